@@ -1,0 +1,84 @@
+"""Pins of the brute-force DAG expansion (event tensor = parametric task DAG)
+against hand-enumerated graphs, and of the trace checker against planted
+mistakes.
+
+"Event Tensor：用“事件张量”编译动态 Megakernel": §Graph Function (maps
+"ij->i" / "i->i"), §Event Tensor 的本质：参数化的 Task DAG,
+§Data-dependent event update, §Data-dependent task triggering.
+"""
+import numpy as np
+
+from oracle import dag
+
+
+def test_splitk_two_tiles_by_hand():
+    g = dag.splitk_graph(rows=64, cols=128, chunk=32, tile_rows=32, sched="static")
+    P, F = dag.OP_SK_PARTIAL, dag.OP_SK_FINAL
+    want_edges = {((P, i, j), (F, i, 0)) for i in range(2) for j in range(4)}
+    assert g.edges == want_edges
+    assert len(g.tasks) == 10
+    # every event gets exactly its wait count of producers (E = ETensor((n,), wait_count=4))
+    for i in range(2):
+        assert len(g.event_producers[("E", i)]) == g.wait_count[("E", i)] == 4
+
+
+def test_splitk_unfused_is_a_barrier():
+    g = dag.splitk_graph(rows=64, cols=128, chunk=32, tile_rows=32, sched="unfused")
+    assert len(g.edges) == 8 * 2  # every partial -> every final
+
+
+def test_moe_tiny_by_hand():
+    # T=2 tokens, k=2, E=3 experts, one token tile, one expert chunk, bm=1
+    topk = np.array([[2, 0], [0, 1]])
+    g, mtiles = dag.moe_graph(topk, E=3, hidden=4, inter=4, tt=2, ec=4, bm=1,
+                              n1_tile=4, n2_tile=4, cb=1, sched="dynamic")
+    # grouping: expert 0 <- (0,1),(1,0); expert 1 <- (1,1); expert 2 <- (0,0); bm=1 -> 4 m-tiles
+    assert [(e, m, rows) for (e, m, rows) in mtiles] == [
+        (0, 0, [(0, 1)]), (0, 1, [(1, 0)]), (1, 0, [(1, 1)]), (2, 0, [(0, 0)])]
+    R, TK, SC, GR, S1, S2, CB = (dag.OP_MOE_ROUTER, dag.OP_MOE_TOPK, dag.OP_MOE_SCAN, dag.OP_MOE_GROUP,
+                                 dag.OP_MOE_S1, dag.OP_MOE_S2, dag.OP_MOE_COMBINE)
+    want = {((R, 0, 0), (TK, 0, 0)), ((TK, 0, 0), (SC, 0, 0)), ((SC, 0, 0), (GR, 0, 0))}
+    want |= {((GR, 0, 0), (S1, f, 0)) for f in range(4)}
+    want |= {((S1, f, 0), (S2, f, 0)) for f in range(4)}
+    # combine block b = token b (cb = 1): rows of m-tile f belong to tokens 0,1,1,0
+    want |= {((S2, 0, 0), (CB, 0, 0)), ((S2, 1, 0), (CB, 1, 0)), ((S2, 2, 0), (CB, 1, 0)),
+             ((S2, 3, 0), (CB, 0, 0))}
+    assert g.edges == want
+    # expert event counts = number of pairs routed to the expert
+    assert len(g.event_producers[("E_exp", 0)]) == 2
+    assert len(g.event_producers[("E_exp", 1)]) == 1
+    assert len(g.event_producers[("E_exp", 2)]) == 1
+
+
+def _trace_from_order(graph):
+    """A valid trace: tasks in a topological order, one after another."""
+    indeg = {t: 0 for t in graph.tasks}
+    succ = {t: [] for t in graph.tasks}
+    for p, c in graph.edges:
+        indeg[c] += 1
+        succ[p].append(c)
+    ready = [t for t in graph.tasks if indeg[t] == 0]
+    recs, tick = [], 0
+    while ready:
+        t = ready.pop()
+        recs.append((t[0], t[1], t[2], 0, tick, tick + 1))
+        tick += 2
+        for c in succ[t]:
+            indeg[c] -= 1
+            if indeg[c] == 0:
+                ready.append(c)
+    return recs
+
+
+def test_checker_accepts_valid_and_catches_planted_mistakes():
+    g = dag.mlp_graph(B=2, hidden=256, inter=256, gu_tile=64, down_tile=128, kchunk=128, sched="static")
+    recs = _trace_from_order(g)
+    assert dag.check_trace(g, recs) == []
+    # a consumer that starts before its producer ended
+    bad = [list(r) for r in recs]
+    i_red = next(i for i, r in enumerate(bad) if r[0] == dag.OP_MLP_REDUCE)
+    bad[i_red][4] = -5
+    assert any("edge violated" in e for e in dag.check_trace(g, bad))
+    # a missing task and a duplicated task
+    assert any("never ran" in e for e in dag.check_trace(g, recs[1:]))
+    assert any("twice" in e for e in dag.check_trace(g, recs + recs[:1]))
