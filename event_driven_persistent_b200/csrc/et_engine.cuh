@@ -1,0 +1,407 @@
+// The persistent megakernel skeleton shared by the three workloads.
+//
+// One CTA per SM runs until its task source is exhausted ("Event Tensor：用
+// “事件张量”编译动态 Megakernel", §Minimal runtime: dispatch, wait, notify
+// and push/pop are compiled into the kernel; the only mutable run-time state
+// is the event counters and the queue).  Roles inside a CTA:
+//
+//   warp 0, lane 0  task source + TMA producer.  Static: walks this CTA's
+//                   task list.  Dynamic: pops the ready queue in batches.
+//                   For a tensor-core task it issues the weight (A) tiles of
+//                   the first pipeline stages BEFORE waiting on the task's
+//                   input event (weights never depend on activations, so
+//                   they stream while the producer tasks finish), then
+//                   waits, then loads the activation (B) tiles.
+//   warp 1, lane 0  tcgen05.mma issuer: D[tmem] += A[smem] * B[smem]^T,
+//                   bf16 in, fp32 accumulate, two TMEM accumulators so the
+//                   epilogue of one task overlaps the main loop of the next.
+//   warps 2..5      epilogues (tcgen05.ld of the accumulator, fused
+//                   element-wise math, stores, notify/push) and all CUDA-core
+//                   tasks (norm, reductions, top-k, grouping, combine).
+//
+// Tasks flow from warp 0 to the others through a 2-deep ring in shared
+// memory guarded by mbarriers.
+#pragma once
+#include "et_device.cuh"
+
+namespace et {
+
+constexpr uint32_t kExitWord = 0xFFFFFFFFu;
+
+struct TaskDesc {
+    uint32_t word;   // task word, kExitWord = stop
+    int valid;       // 0 = a static slot with nothing to do at this size
+    uint32_t start;  // trace ticket taken after the task's wait
+    int gemm;        // 1 = tensor-core task
+    int a_map, a_row0, a_row1;  // A: tensor map id, rows of the two 64-row boxes
+    int b_map, b_row0;          // B: tensor map id, first row
+    int n;                      // MMA N (multiple of 16, <= kMaxN)
+    int k0, nk;                 // first K element, number of 64-wide K stages
+    int p[6];                   // workload-specific
+};
+
+struct SmemCtl {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t ring_full[kRing];
+    uint64_t ring_empty[kRing];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int start_status;
+    int bcast[8];
+    TaskDesc ring[kRing];
+};
+
+// Everything a role needs besides the workload parameters.
+struct Ctx {
+    Ctl* ctl;
+    uint64_t timeout_ns;
+    int* ctr;            // this run's counter set
+    Queue q;
+    int dynamic;         // 1 = ready queue, 0 = static lists
+    int debug;           // ET_DEBUG_* bits
+    TraceRec* trace;
+    int trace_cap;
+    uint8_t* stages;     // kStages x kStageBytes, 1024-aligned
+    float* epi;          // gate/up exchange staging
+    uint8_t* simt;       // CUDA-core task scratch
+    SmemCtl* sc;
+    int tid;             // exec-group thread index 0..127 (exec warps only)
+};
+
+__device__ __forceinline__ void exec_bar() { named_bar_sync(1, kExecThreads); }
+
+// Push n consumer tasks from the exec group (all 128 threads call; n uniform).
+template <class Gen>
+__device__ __forceinline__ void group_push(Ctx& x, int n, Gen gen) {
+    if (n <= 0) return;
+    if (x.tid == 0) x.sc->bcast[0] = q_reserve(x.q, n);
+    exec_bar();
+    int base = x.sc->bcast[0];
+    for (int i = x.tid; i < n; i += kExecThreads) q_publish(x.q, base + i, gen(i));
+    exec_bar();
+}
+
+// Push n tasks from a single thread.
+template <class Gen>
+__device__ __forceinline__ void thread_push(Ctx& x, int n, Gen gen) {
+    if (n <= 0) return;
+    int base = q_reserve(x.q, n);
+    for (int i = 0; i < n; ++i) q_publish(x.q, base + i, gen(i));
+}
+
+// End of a task in the exec group: every thread has written its outputs.
+// Thread 0 records the trace and adds `n` to one event counter; returns (to
+// all threads) whether this notify completed the event (counter == target).
+__device__ __forceinline__ bool group_finish_notify(Ctx& x, const TaskDesc& d, int* ctr, int n, int target) {
+    exec_bar();
+    if (x.tid == 0) {
+        int fired = 0;
+        if (x.debug & ET_DEBUG_TRACE) {
+            uint32_t end = take_ticket(x.ctl);
+            trace_write(x.ctl, x.trace, x.trace_cap, task_op(d.word), task_a(d.word), task_b(d.word), d.start, end);
+        }
+        if (ctr) fired = notify(ctr, n) == target;
+        x.sc->bcast[1] = fired;
+    }
+    exec_bar();
+    return x.sc->bcast[1] != 0;
+}
+
+// Exec-group wait on an event (SIMT tasks).  Returns false on timeout/abort.
+__device__ __forceinline__ bool group_wait(Ctx& x, TaskDesc& d, const int* ctr, int target, int where) {
+    if (x.tid == 0) {
+        bool ok = ctr == nullptr || wait_geq(ctr, target, x.ctl, x.timeout_ns, where, task_word(0, 0, 0) ^ d.word);
+        if (ok && (x.debug & ET_DEBUG_TRACE)) d.start = take_ticket(x.ctl);
+        x.sc->bcast[2] = ok;
+        x.sc->bcast[3] = (int)d.start;
+    }
+    exec_bar();
+    bool ok = x.sc->bcast[2] != 0;
+    d.start = (uint32_t)x.sc->bcast[3];
+    exec_bar();
+    return ok;
+}
+
+// Megakernel body.  W supplies the task semantics:
+//   W::fetch_init(p, idx)              initial dynamic task word for slot idx
+//   W::derive(p, x, word, d)           fill a TaskDesc (warp 0; may wait in
+//                                      static mode); false = abort
+//   W::gemm_wait(p, x, d)              the GEMM task's input wait (warp 0)
+//   W::a_map(p, id), W::b_map(p, id)   tensor maps
+//   W::epilogue(p, x, d, acc_taddr)    exec group, after the accumulator is ready
+//   W::simt(p, x, d)                   exec group, a CUDA-core task
+template <class W>
+__device__ __forceinline__ void megakernel_body(const typename W::Params& p, const RunArgs& ra) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = base;
+    float* epi = reinterpret_cast<float*>(base + kStages * kStageBytes);
+    uint8_t* simt = base + kStages * kStageBytes + kEpiBytes;
+    SmemCtl* sc = reinterpret_cast<SmemCtl*>(simt + kSimtBytes);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    Ctl* ctl = ra.ctl;
+
+    // zero the other parity's counter set for the next run
+    {
+        int* other = ra.ctr_next;
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < ra.n_ctr; i += gridDim.x * blockDim.x) other[i] = 0;
+    }
+    if (threadIdx.x == 0) {
+        sc->start_status = ld_volatile(&ctl->status);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sc->full[s], 1);
+            mbar_init(&sc->empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sc->acc_full[b], 1);
+            mbar_init(&sc->acc_empty[b], kExecThreads / 32);
+        }
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(&sc->ring_full[r], 1);
+            mbar_init(&sc->ring_empty[r], 2);  // MMA warp + exec group
+        }
+        mbar_init(&sc->drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 1 && W::kGemm) {
+        tmem_alloc(&sc->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const bool skip = sc->start_status != 0;  // an earlier run failed: do nothing until the host resets
+
+    Ctx x;
+    x.ctl = ctl;
+    x.timeout_ns = ra.timeout_ns;
+    x.ctr = ra.ctr;
+    x.q.slots = ra.qslots;
+    x.q.cap = ra.qcap;
+    x.q.head = ra.ctr + 0;
+    x.q.tail = ra.ctr + 1;
+    x.q.total = ra.ctr + 2;
+    x.q.epoch = ra.epoch;
+    x.q.n_init = ra.n_init;
+    x.q.total_static = ra.total_static;
+    x.dynamic = ra.dynamic;
+    x.debug = ra.debug;
+    x.trace = ra.trace;
+    x.trace_cap = ra.trace_cap;
+    x.stages = stages;
+    x.epi = epi;
+    x.simt = simt;
+    x.sc = sc;
+    x.tid = threadIdx.x - kExecWarp0 * 32;
+
+    uint32_t armed[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) armed[s] = 0;
+
+    if (!skip && warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ task source + TMA
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_a = policy_evict_last();
+            int lpos = 0, lend = 0;
+            if (!x.dynamic) {
+                lpos = ra.lists.off[blockIdx.x];
+                lend = ra.lists.off[blockIdx.x + 1];
+            }
+            int qn = 0, qe = 0;
+            uint32_t st = 0;  // stages armed so far (ring position)
+            for (uint32_t it = 0;; ++it) {
+                TaskDesc d;
+                d.word = kExitWord;
+                d.valid = 0;
+                d.gemm = 0;
+                d.start = 0;
+                int r;
+                if (!x.dynamic) {
+                    r = lpos < lend ? 1 : 0;
+                    if (r) d.word = ra.lists.words[lpos++];
+                } else {
+                    if (qn == qe) {
+                        qn = atom_add_relaxed(x.q.head, ra.fetch_batch);
+                        qe = qn + ra.fetch_batch;
+                    }
+                    uint32_t w;
+                    r = q_resolve(x.q, qn, &w, [&](int i) { return W::fetch_init(p, i); }, ctl, x.timeout_ns);
+                    ++qn;
+                    if (r == 1) d.word = w;
+                }
+                if (r < 0) break;
+                if (r == 1 && !W::derive(p, x, d)) break;
+                const uint32_t slot = it % kRing;
+                if (!mbar_wait(&sc->ring_empty[slot], ((it / kRing) & 1) ^ 1, ctl, x.timeout_ns, 901)) break;
+                if (r == 1 && d.valid && d.gemm) {
+                    const CUtensorMap* am = W::a_map(p, d.a_map);
+                    const CUtensorMap* bm = W::b_map(p, d.b_map);
+                    const uint32_t bbytes = (uint32_t)d.n * 128u;
+                    const int npre = d.nk < kStages ? d.nk : kStages;
+                    bool ok = true;
+                    for (int s = 0; s < npre && ok; ++s) {  // weights first
+                        const uint32_t ss = (st + s) % kStages;
+                        ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 902);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
+                        ++armed[ss];
+                        uint8_t* dst = stages + ss * kStageBytes;
+                        const int kx = d.k0 + s * kTileK;
+                        tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
+                        tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
+                    }
+                    if (ok) ok = W::gemm_wait(p, x, d);  // the task's input event
+                    if (ok && (x.debug & ET_DEBUG_TRACE)) d.start = take_ticket(ctl);
+                    if (ok) fence_proxy_async_global();
+                    sc->ring[slot] = d;
+                    mbar_arrive(&sc->ring_full[slot]);
+                    if (!ok) {
+                        // the consumers see the abort flag; stop issuing
+                        st += npre;
+                        break;
+                    }
+                    for (int s = 0; s < d.nk && ok; ++s) {
+                        const uint32_t ss = (st + s) % kStages;
+                        uint8_t* dst = stages + ss * kStageBytes;
+                        const int kx = d.k0 + s * kTileK;
+                        if (s >= npre) {
+                            ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 903);
+                            if (!ok) break;
+                            mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
+                            ++armed[ss];
+                            tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
+                            tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
+                        }
+                        for (int rb = 0; rb < d.n; rb += 16)
+                            tma_load_2d(dst + kAStageBytes + rb * 128, bm, &sc->full[ss], kx, d.b_row0 + rb, pol_a);
+                    }
+                    st += d.nk;
+                    if (!ok) break;
+                } else {
+                    sc->ring[slot] = d;
+                    mbar_arrive(&sc->ring_full[slot]);
+                }
+                if (r == 0) break;
+            }
+            // drain: every armed stage's TMA must land before the CTA exits
+            for (int s = 0; s < kStages; ++s)
+                if (armed[s]) {
+                    uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait(&sc->full[s], (armed[s] - 1) & 1) && globaltimer() - t0 < 200000000ull) {
+                    }
+                }
+        }
+        __syncwarp();
+    } else if (!skip && warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------------ MMA issuer
+            uint32_t st = 0, g = 0;
+            bool issued_any = false;
+            for (uint32_t it = 0;; ++it) {
+                const uint32_t slot = it % kRing;
+                if (!mbar_wait(&sc->ring_full[slot], (it / kRing) & 1, ctl, x.timeout_ns, 910)) break;
+                TaskDesc d = sc->ring[slot];
+                mbar_arrive(&sc->ring_empty[slot]);
+                if (d.word == kExitWord) break;
+                if (!(d.valid && d.gemm)) continue;
+                const uint32_t buf = g & 1;
+                if (!mbar_wait(&sc->acc_empty[buf], ((g >> 1) & 1) ^ 1, ctl, x.timeout_ns, 911)) break;
+                tc_fence_after();
+                const uint32_t dt = sc->tmem_base + buf * kMaxN;
+                const uint32_t idesc = idesc_bf16_f32(128, d.n);
+                bool ok = true;
+                for (int s = 0; s < d.nk; ++s) {
+                    const uint32_t ss = (st + s) % kStages;
+                    if (!mbar_wait(&sc->full[ss], ((st + s) / kStages) & 1, ctl, x.timeout_ns, 912)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(stages + ss * kStageBytes);
+                    const uint64_t ad = sdesc_k128(a0);
+                    const uint64_t bd = sdesc_k128(a0 + kAStageBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kTileK / 16; ++kk)
+                        tc_mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, idesc, (s | kk) ? 1u : 0u);
+                    tc_commit(&sc->empty[ss]);
+                    issued_any = true;
+                }
+                if (!ok) break;
+                st += d.nk;
+                tc_commit(&sc->acc_full[buf]);
+                ++g;
+            }
+            if (issued_any) {  // every MMA must finish before TMEM is released
+                tc_commit(&sc->drain);
+                uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(&sc->drain, 0) && globaltimer() - t0 < 200000000ull) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (!skip && warp >= kExecWarp0) {
+        // ------------------------------------------------- epilogue / CUDA-core
+        // Every decision that can end the loop is taken by exec thread 0 and
+        // broadcast, so the four warps never split around a named barrier.
+        uint32_t g = 0;
+        for (uint32_t it = 0;; ++it) {
+            const uint32_t slot = it % kRing;
+            if (x.tid == 0) sc->bcast[4] = mbar_wait(&sc->ring_full[slot], (it / kRing) & 1, ctl, x.timeout_ns, 920);
+            exec_bar();
+            if (!sc->bcast[4]) break;
+            TaskDesc d = sc->ring[slot];
+            exec_bar();
+            if (x.tid == 0) mbar_arrive(&sc->ring_empty[slot]);
+            if (d.word == kExitWord) break;
+            if (!d.valid) continue;
+            if (x.debug & ET_DEBUG_DELAY) debug_delay(d.word ^ (ra.epoch * 977u));
+            if (d.gemm) {
+                const uint32_t buf = g & 1;
+                const uint32_t par = (g >> 1) & 1;
+                if (x.tid == 0) sc->bcast[5] = mbar_wait(&sc->acc_full[buf], par, ctl, x.timeout_ns, 921);
+                exec_bar();
+                if (!sc->bcast[5]) break;
+                while (!mbar_try_wait(&sc->acc_full[buf], par)) {
+                }
+                tc_fence_after();
+                const uint32_t taddr = sc->tmem_base + buf * kMaxN + ((uint32_t)((warp & 3) * 32) << 16);
+                if (!W::epilogue(p, x, d, taddr, &sc->acc_empty[buf])) break;
+                ++g;
+            } else {
+                if (!W::simt(p, x, d)) break;
+            }
+            if (x.tid == 0) sc->bcast[6] = aborted(ctl);
+            exec_bar();
+            if (sc->bcast[6]) break;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1 && W::kGemm) {
+        tc_fence_after();
+        tmem_dealloc(sc->tmem_base, kTmemCols);
+    }
+}
+
+// Epilogue helper: read this warp's 32 lanes x 16 columns [c0, c0+16) of
+// the accumulator into v (thread = lane).
+__device__ __forceinline__ void acc_load16(uint32_t taddr, int c0, float (&v)[16]) {
+    __syncwarp();  // tcgen05.ld is .sync.aligned: the warp must be converged
+    tmem_ld16(taddr + (uint32_t)c0, v);
+    tmem_ld_wait();
+}
+
+// Release the accumulator after this warp's last tcgen05.ld.
+__device__ __forceinline__ void acc_release(uint64_t* acc_empty) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(acc_empty);
+}
+
+}  // namespace et

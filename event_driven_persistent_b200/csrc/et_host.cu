@@ -1,0 +1,648 @@
+// Host half of libet: the C ABI (include/et.h), the graph builder (static
+// per-SM task lists per size bucket, workspace), tensor-map encoding and the
+// launches.  No torch types cross this boundary.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <functional>
+#include <queue>
+#include <vector>
+
+#include "et_params.h"
+
+namespace et {
+cudaError_t splitk_setup(int* max_blocks_per_sm);
+cudaError_t launch_splitk(const SplitKParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
+cudaError_t mlp_setup(int* max_blocks_per_sm);
+cudaError_t launch_mlp(const MlpParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
+cudaError_t moe_setup(int* max_blocks_per_sm);
+cudaError_t launch_moe(const MoeParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
+}  // namespace et
+
+using namespace et;
+
+namespace {
+
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+inline int next_pow2(int v) {
+    int b = 1;
+    while (b < v) b <<= 1;
+    return b;
+}
+
+// -------------------------------------------------------- tensor maps ----
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool load_encode() {
+    if (g_encode) return true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return true;
+}
+
+// bf16 [rows, cols] row-major, 128-byte swizzle, box = box_rows x 64 columns.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    if (!load_encode()) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+struct MapCache {
+    const void* ptr = nullptr;
+    uint64_t rows = 0, cols = 0;
+    uint32_t box = 0;
+    CUtensorMap map;
+    bool get(CUtensorMap* out, const void* p, uint64_t r, uint64_t c, uint32_t b) {
+        if (p != ptr || r != rows || c != cols || b != box) {
+            if (!make_map(&map, p, r, c, b)) return false;
+            ptr = p;
+            rows = r;
+            cols = c;
+            box = b;
+        }
+        *out = map;
+        return true;
+    }
+};
+
+// ------------------------------------------------------- static lists ----
+struct Slot {
+    uint32_t word;
+    float cost;
+};
+
+inline uint32_t tw(int op, int a, int b) {
+    return ((uint32_t)op << 26) | ((uint32_t)(a & 0xFFFF) << 10) | (uint32_t)(b & 0x3FF);
+}
+
+// Assign level-ordered slots to CTAs: each slot goes to the CTA with the
+// least accumulated cost (ties -> lower CTA), so every CTA's list stays in
+// level order (a task only waits on lower levels: no deadlock when all CTAs
+// are resident).
+void assign(const std::vector<Slot>& slots, int n_ctas, std::vector<int>& off, std::vector<uint32_t>& words) {
+    std::vector<std::vector<uint32_t>> per(n_ctas);
+    typedef std::pair<double, int> E;
+    std::priority_queue<E, std::vector<E>, std::greater<E>> pq;
+    for (int c = 0; c < n_ctas; ++c) pq.push(E(0.0, c));
+    for (const Slot& s : slots) {
+        E e = pq.top();
+        pq.pop();
+        per[e.second].push_back(s.word);
+        pq.push(E(e.first + s.cost, e.second));
+    }
+    off.assign(n_ctas + 1, 0);
+    words.clear();
+    for (int c = 0; c < n_ctas; ++c) {
+        off[c] = (int)words.size();
+        words.insert(words.end(), per[c].begin(), per[c].end());
+    }
+    off[n_ctas] = (int)words.size();
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- graph ----
+struct et_graph {
+    et_graph_desc d;
+    et_graph_info info;
+    int dev = 0, n_sm = 0, n_ctas = 0;
+    Ctl* ctl = nullptr;
+    int* ctr[2] = {nullptr, nullptr};
+    int n_ctr = 0;
+    unsigned long long* qslots = nullptr;
+    int qcap = 0;
+    TraceRec* trace = nullptr;
+    int trace_cap = 0;
+    uint32_t epoch = 0;
+    // static lists: one CSR per bucket, concatenated
+    std::vector<int> bucket_T;
+    std::vector<size_t> off_at, words_at;
+    int* lists_off = nullptr;
+    uint32_t* lists_words = nullptr;
+    std::vector<void*> allocs;
+    // workload state
+    SplitKParams sk;
+    MlpParams mlp;
+    MoeParams moe;
+    MapCache mc[6];
+    int bucket_of(int T) const {
+        for (size_t i = 0; i < bucket_T.size(); ++i)
+            if (bucket_T[i] >= T) return (int)i;
+        return (int)bucket_T.size() - 1;
+    }
+};
+
+namespace {
+
+et_status cuda_fail(cudaError_t e) {
+    if (e == cudaErrorMemoryAllocation) return ET_ERR_OOM;
+    return ET_ERR_CUDA;
+}
+
+#define ET_CU(call)                                   \
+    do {                                              \
+        cudaError_t e_ = (call);                      \
+        if (e_ != cudaSuccess) return cuda_fail(e_);  \
+    } while (0)
+
+template <class T>
+et_status galloc(et_graph* g, T** p, size_t n) {
+    void* q = nullptr;
+    if (n == 0) n = 1;
+    cudaError_t e = cudaMalloc(&q, n * sizeof(T));
+    if (e != cudaSuccess) return cuda_fail(e);
+    g->allocs.push_back(q);
+    e = cudaMemset(q, 0, n * sizeof(T));
+    if (e != cudaSuccess) return cuda_fail(e);
+    *p = static_cast<T*>(q);
+    return ET_OK;
+}
+
+#define ET_TRY(x)                      \
+    do {                               \
+        et_status s_ = (x);            \
+        if (s_ != ET_OK) return s_;    \
+    } while (0)
+
+bool aligned16(const void* p) { return p && ((uintptr_t)p & 15) == 0; }
+
+// Build every bucket's lists with `gen(T_b, slots)`, upload them.
+et_status build_lists(et_graph* g, const std::function<void(int, std::vector<Slot>&)>& gen) {
+    std::vector<int> all_off;
+    std::vector<uint32_t> all_words;
+    for (int T = 1;; T <<= 1) {
+        int Tb = std::min(T, g->d.max_T);
+        std::vector<Slot> slots;
+        gen(Tb, slots);
+        std::vector<int> off;
+        std::vector<uint32_t> words;
+        assign(slots, g->n_ctas, off, words);
+        g->bucket_T.push_back(Tb);
+        g->off_at.push_back(all_off.size());
+        g->words_at.push_back(all_words.size());
+        for (int o : off) all_off.push_back(o);
+        all_words.insert(all_words.end(), words.begin(), words.end());
+        if (Tb >= g->d.max_T) break;
+    }
+    ET_TRY(galloc(g, &g->lists_off, all_off.size()));
+    ET_TRY(galloc(g, &g->lists_words, all_words.size()));
+    ET_CU(cudaMemcpy(g->lists_off, all_off.data(), all_off.size() * sizeof(int), cudaMemcpyHostToDevice));
+    ET_CU(cudaMemcpy(g->lists_words, all_words.data(), all_words.size() * sizeof(uint32_t), cudaMemcpyHostToDevice));
+    return ET_OK;
+}
+
+RunArgs run_args(et_graph* g, int T, int n_init, int total_static) {
+    RunArgs ra;
+    memset(&ra, 0, sizeof(ra));
+    ++g->epoch;
+    ra.ctl = g->ctl;
+    ra.ctr = g->ctr[g->epoch & 1];
+    ra.ctr_next = g->ctr[(g->epoch + 1) & 1];
+    ra.n_ctr = g->n_ctr;
+    ra.qslots = g->qslots;
+    ra.qcap = g->qcap;
+    ra.epoch = g->epoch;
+    ra.n_init = n_init;
+    ra.total_static = total_static;
+    ra.dynamic = g->d.sched == ET_SCHED_DYNAMIC;
+    ra.fetch_batch = g->d.fetch_batch;
+    ra.debug = g->d.debug_flags;
+    ra.trace = g->trace;
+    ra.trace_cap = g->trace_cap;
+    int b = g->bucket_of(T);
+    ra.lists.off = g->lists_off + g->off_at[b];
+    ra.lists.words = g->lists_words + g->words_at[b];
+    ra.timeout_ns = (unsigned long long)((double)g->d.timeout_ms * 1e6);
+    return ra;
+}
+
+et_status pre_run(et_graph* g, cudaStream_t s) {
+    if (g->d.debug_flags & ET_DEBUG_TRACE) {
+        // the trace of one run: clear the record counter and tickets
+        ET_CU(cudaMemsetAsync(&g->ctl->ticket, 0, 2 * sizeof(int), s));
+    }
+    return ET_OK;
+}
+
+// ------------------------------------------------------------- split-K ----
+et_status build_splitk(et_graph* g) {
+    et_graph_desc& d = g->d;
+    if (d.splitk_cols <= 0) d.splitk_cols = 128;
+    if (d.splitk_chunk <= 0) d.splitk_chunk = 32;
+    if (d.splitk_tile_rows <= 0) d.splitk_tile_rows = 32;
+    if (d.fetch_batch <= 0) d.fetch_batch = 4;
+    const int nt_max = cdiv(d.max_T, d.splitk_tile_rows);
+    const int nch = cdiv(d.splitk_cols, d.splitk_chunk);
+    if (nt_max > 0xFFFF || nch > 0x3FF) return ET_ERR_UNSUPPORTED;
+    SplitKParams& p = g->sk;
+    memset(&p, 0, sizeof(p));
+    p.cols = d.splitk_cols;
+    p.chunk = d.splitk_chunk;
+    p.tile_rows = d.splitk_tile_rows;
+    p.n_chunks = nch;
+    p.ev_base = kCtrFirstEvent;
+    p.ev_all = kCtrFirstEvent + nt_max;
+    p.unfused = d.sched == ET_SCHED_UNFUSED;
+    p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
+    g->n_ctr = p.ev_all + 1;
+    g->qcap = nt_max * nch + nt_max + g->n_ctas * d.fetch_batch + 64;
+    int mb = 0;
+    ET_CU(splitk_setup(&mb));
+    if (mb < 1) return ET_ERR_UNSUPPORTED;
+    return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
+        int nt = cdiv(Tb, d.splitk_tile_rows);
+        for (int i = 0; i < nt; ++i)
+            for (int j = 0; j < nch; ++j) s.push_back({tw(ET_OP_SK_PARTIAL, i, j), 1.0f});
+        for (int i = 0; i < nt; ++i) s.push_back({tw(ET_OP_SK_FINAL, i, 0), 0.5f});
+    });
+}
+
+// ----------------------------------------------------------------- MLP ----
+et_status build_mlp(et_graph* g) {
+    et_graph_desc& d = g->d;
+    if (d.hidden <= 0) d.hidden = 4096;
+    if (d.inter <= 0) d.inter = 14336;
+    if (d.rms_eps <= 0.f) d.rms_eps = 1e-5f;
+    if (d.fetch_batch <= 0) d.fetch_batch = 1;
+    if (d.max_T > kMaxN) return ET_ERR_UNSUPPORTED;  // one token tile
+    if (d.hidden % 128 || d.inter % 64) return ET_ERR_UNSUPPORTED;
+    MlpParams& p = g->mlp;
+    memset(&p, 0, sizeof(p));
+    p.hidden = d.hidden;
+    p.inter = d.inter;
+    p.maxB = d.max_T;
+    p.eps = d.rms_eps;
+    p.gu_tile = 64;
+    p.down_tile = 128;
+    p.kchunk = d.inter % 1024 == 0 ? 1024 : (d.inter % 256 == 0 ? 256 : 64);
+    p.n_gu = d.inter / p.gu_tile;
+    p.n_m = d.hidden / p.down_tile;
+    p.n_c = d.inter / p.kchunk;
+    p.gu_per_chunk = p.kchunk / p.gu_tile;
+    if (p.n_gu > 0xFFFF || p.n_c > 0x3FF) return ET_ERR_UNSUPPORTED;
+    p.ev_norm = kCtrFirstEvent;
+    p.ev_h = p.ev_norm + 1;
+    p.ev_y = p.ev_h + p.n_c;
+    p.ev_gu_all = p.ev_y + p.n_m;
+    p.ev_down_all = p.ev_gu_all + 1;
+    p.unfused = d.sched == ET_SCHED_UNFUSED;
+    p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
+    g->n_ctr = p.ev_down_all + 1;
+    g->qcap = d.max_T + p.n_gu + p.n_m * p.n_c + p.n_m + g->n_ctas * d.fetch_batch + 64;
+    ET_TRY(galloc(g, &p.xn, (size_t)p.maxB * p.hidden));
+    ET_TRY(galloc(g, &p.h, (size_t)p.maxB * p.inter));
+    ET_TRY(galloc(g, &p.part, (size_t)p.n_c * p.maxB * p.hidden));
+    if (!make_map(&p.tm_xn, p.xn, p.maxB, p.hidden, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_h, p.h, p.maxB, p.inter, 16)) return ET_ERR_CUDA;
+    int mb = 0;
+    ET_CU(mlp_setup(&mb));
+    if (mb < 1) return ET_ERR_UNSUPPORTED;
+    // cost ~ bytes streamed per task (KB)
+    const float c_gu = 2.f * p.gu_tile * p.hidden * 2 / 1024.f, c_dn = (float)p.down_tile * p.kchunk * 2 / 1024.f;
+    return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
+        for (int b = 0; b < Tb; ++b) s.push_back({tw(ET_OP_MLP_NORM, b, 0), 1.f});
+        for (int n = 0; n < p.n_gu; ++n) s.push_back({tw(ET_OP_MLP_GATEUP, n, 0), c_gu});
+        for (int c = 0; c < p.n_c; ++c)
+            for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_MLP_DOWN, m, c), c_dn});
+        for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_MLP_REDUCE, m, 0), 2.f});
+    });
+}
+
+// ----------------------------------------------------------------- MoE ----
+struct MoeShape {
+    int n_tt, n_kc, n_g, n_cb, f_max;
+};
+
+MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
+    MoeShape m;
+    m.n_tt = cdiv(T, p.tt);
+    // router K split: enough (token tile, chunk) tasks to cover the SMs
+    int kc = 1;
+    while (kc < 8 && m.n_tt * kc * 2 <= g->n_ctas && (p.hidden / (kc * 2)) % kTileK == 0) kc *= 2;
+    m.n_kc = kc;
+    m.n_g = cdiv(T, p.gt);
+    m.n_cb = cdiv(T, p.cb);
+    const int pairs = p.k * T;
+    m.f_max = std::min(pairs, std::min(p.E, pairs) + cdiv(pairs, p.bm));
+    return m;
+}
+
+et_status build_moe(et_graph* g) {
+    et_graph_desc& d = g->d;
+    if (d.hidden <= 0) d.hidden = 2048;
+    if (d.inter <= 0) d.inter = 768;
+    if (d.n_experts <= 0) d.n_experts = 128;
+    if (d.top_k <= 0) d.top_k = 8;
+    if (d.fetch_batch <= 0) d.fetch_batch = 1;
+    if (d.n_experts > 128 || d.top_k > 32 || d.top_k > d.n_experts) return ET_ERR_UNSUPPORTED;
+    if (d.hidden % 128 || d.inter % 64) return ET_ERR_UNSUPPORTED;
+    MoeParams& p = g->moe;
+    memset(&p, 0, sizeof(p));
+    p.hidden = d.hidden;
+    p.inter = d.inter;
+    p.E = d.n_experts;
+    p.k = d.top_k;
+    p.maxT = d.max_T;
+    p.tt = 128;
+    p.gt = std::max(1, 128 / p.k);
+    p.bm = 128;
+    p.n1_tile = 64;
+    p.n_n1 = p.inter / p.n1_tile;
+    p.n2_tile = 128;
+    p.n_n2 = p.hidden / p.n2_tile;
+    p.cb = 16;
+    p.sched = d.sched;
+    p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
+    const MoeShape mx = moe_shape(g, p, d.max_T);
+    if (mx.f_max > 0xFFFF || mx.n_g > 0xFFFF || p.n_n1 > 0x3FF || p.n_n2 > 0x3FF) return ET_ERR_UNSUPPORTED;
+    int ev = kCtrFirstEvent;
+    p.ev_tk = ev++;
+    p.ev_sc = ev++;
+    p.ev_grp = ev++;
+    p.ev_rt_all = ev++;
+    p.ev_s1_all = ev++;
+    p.ev_s2_all = ev++;
+    p.ev_rt = ev;
+    ev += mx.n_tt;
+    p.ev_exp = ev;
+    ev += p.E;
+    p.ev_s1 = ev;
+    ev += mx.f_max;
+    p.ev_cb = ev;
+    ev += mx.n_cb;
+    g->n_ctr = ev;
+    g->qcap = mx.n_tt * 8 + mx.n_tt + 1 + mx.n_g + mx.f_max * (p.n_n1 + p.n_n2) + mx.n_cb + g->n_ctas * d.fetch_batch + 64;
+    const size_t pairs = (size_t)p.maxT * p.k;
+    ET_TRY(galloc(g, &p.lpart, (size_t)8 * p.maxT * p.E));
+    ET_TRY(galloc(g, &p.logits, (size_t)p.maxT * p.E));
+    ET_TRY(galloc(g, &p.topk, pairs));
+    ET_TRY(galloc(g, &p.topw, pairs));
+    ET_TRY(galloc(g, &p.gcnt, (size_t)mx.n_g * p.E));
+    ET_TRY(galloc(g, &p.goff, (size_t)mx.n_g * p.E));
+    ET_TRY(galloc(g, &p.counts, (size_t)p.E));
+    ET_TRY(galloc(g, &p.indptr, (size_t)p.E + 1));
+    ET_TRY(galloc(g, &p.tindptr, (size_t)p.E + 1));
+    ET_TRY(galloc(g, &p.mt_expert, (size_t)mx.f_max));
+    ET_TRY(galloc(g, &p.perm, pairs));
+    ET_TRY(galloc(g, &p.pos, pairs));
+    ET_TRY(galloc(g, &p.scal, 8));
+    ET_TRY(galloc(g, &p.Xp, pairs * p.hidden));
+    ET_TRY(galloc(g, &p.Hm, pairs * p.inter));
+    ET_TRY(galloc(g, &p.Yacc, (size_t)p.maxT * p.hidden));
+    if (!make_map(&p.tm_xp, p.Xp, pairs, p.hidden, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_hm, p.Hm, pairs, p.inter, 16)) return ET_ERR_CUDA;
+    int mb = 0;
+    ET_CU(moe_setup(&mb));
+    if (mb < 1) return ET_ERR_UNSUPPORTED;
+    const float c_s1 = 2.f * p.n1_tile * p.hidden * 2 / 1024.f, c_s2 = (float)p.n2_tile * p.inter * 2 / 1024.f;
+    return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
+        MoeShape m = moe_shape(g, p, Tb);
+        const float c_rt = (float)p.E * p.hidden * 2 / m.n_kc / 1024.f;
+        for (int t = 0; t < m.n_tt; ++t)
+            for (int c = 0; c < m.n_kc; ++c) s.push_back({tw(ET_OP_MOE_ROUTER, t, c), c_rt});
+        for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_TOPK, t, 0), 8.f});
+        s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 16.f});
+        for (int q = 0; q < m.n_g; ++q) s.push_back({tw(ET_OP_MOE_GROUP, q, 0), (float)p.gt * p.k * p.hidden * 2 / 1024.f});
+        for (int f = 0; f < m.f_max; ++f)
+            for (int n = 0; n < p.n_n1; ++n) s.push_back({tw(ET_OP_MOE_S1, f, n), c_s1});
+        for (int f = 0; f < m.f_max; ++f)
+            for (int n = 0; n < p.n_n2; ++n) s.push_back({tw(ET_OP_MOE_S2, f, n), c_s2});
+        for (int b = 0; b < m.n_cb; ++b) s.push_back({tw(ET_OP_MOE_COMBINE, b, 0), 2.f});
+    });
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+extern "C" {
+
+const char* et_status_str(et_status s) {
+    switch (s) {
+        case ET_OK: return "ok";
+        case ET_ERR_INVALID: return "invalid argument";
+        case ET_ERR_CUDA: return "CUDA error";
+        case ET_ERR_TIMEOUT: return "device wait timed out";
+        case ET_ERR_OOM: return "out of device memory";
+        case ET_ERR_UNSUPPORTED: return "unsupported device or dims";
+        case ET_ERR_PENDING: return "an earlier run failed";
+    }
+    return "unknown status";
+}
+
+
+
+et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
+    if (!desc || !out) return ET_ERR_INVALID;
+    *out = nullptr;
+    if (desc->max_T < 1 || desc->kind < 0 || desc->kind > 2 || desc->sched < 0 || desc->sched > 2)
+        return ET_ERR_INVALID;
+    et_graph* g = new et_graph();
+    g->d = *desc;
+    if (g->d.timeout_ms <= 0) g->d.timeout_ms = 1000.f;
+    auto fail = [&](et_status s) {
+        et_destroy_graph(g);
+        return s;
+    };
+    if (cudaSetDevice(desc->device) != cudaSuccess) return fail(ET_ERR_CUDA);
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, desc->device) != cudaSuccess) return fail(ET_ERR_CUDA);
+    if (prop.major != 10) return fail(ET_ERR_UNSUPPORTED);
+    g->dev = desc->device;
+    g->n_sm = prop.multiProcessorCount;
+    g->n_ctas = desc->n_ctas > 0 ? std::min(desc->n_ctas, g->n_sm) : g->n_sm;
+    et_status st = ET_ERR_INVALID;
+    if (desc->kind == ET_GRAPH_SPLITK) st = build_splitk(g);
+    else if (desc->kind == ET_GRAPH_MLP) st = build_mlp(g);
+    else st = build_moe(g);
+    if (st != ET_OK) return fail(st);
+    // common workspace
+    if ((st = galloc(g, &g->ctl, 1)) != ET_OK) return fail(st);
+    if ((st = galloc(g, &g->ctr[0], g->n_ctr)) != ET_OK) return fail(st);
+    if ((st = galloc(g, &g->ctr[1], g->n_ctr)) != ET_OK) return fail(st);
+    if ((st = galloc(g, &g->qslots, g->qcap)) != ET_OK) return fail(st);
+    g->trace_cap = (g->d.debug_flags & ET_DEBUG_TRACE) ? g->qcap + 1024 : 1;
+    if ((st = galloc(g, &g->trace, g->trace_cap)) != ET_OK) return fail(st);
+    if (cudaDeviceSynchronize() != cudaSuccess) return fail(ET_ERR_CUDA);
+    // info
+    et_graph_info& in = g->info;
+    memset(&in, 0, sizeof(in));
+    in.kind = g->d.kind;
+    in.sched = g->d.sched;
+    in.max_T = g->d.max_T;
+    in.n_ctas = g->n_ctas;
+    in.threads = kThreads;
+    in.smem_bytes = kSmemBytes;
+    in.fetch_batch = g->d.fetch_batch;
+    in.hidden = g->d.hidden;
+    in.inter = g->d.inter;
+    in.n_experts = g->d.n_experts;
+    in.top_k = g->d.top_k;
+    in.splitk_cols = g->d.splitk_cols;
+    in.splitk_chunk = g->d.splitk_chunk;
+    in.splitk_tile_rows = g->d.splitk_tile_rows;
+    if (desc->kind == ET_GRAPH_MLP) {
+        in.mlp_gu_tile = g->mlp.gu_tile;
+        in.mlp_down_tile = g->mlp.down_tile;
+        in.mlp_kchunk = g->mlp.kchunk;
+    }
+    if (desc->kind == ET_GRAPH_MOE) {
+        in.moe_tt = g->moe.tt;
+        in.moe_gt = g->moe.gt;
+        in.moe_bm = g->moe.bm;
+        in.moe_n1_tile = g->moe.n1_tile;
+        in.moe_n2_tile = g->moe.n2_tile;
+        in.moe_cb = g->moe.cb;
+        in.moe_router_kc = g->moe.n_kc;
+    }
+    *out = g;
+    return ET_OK;
+}
+
+void et_destroy_graph(et_graph* g) {
+    if (!g) return;
+    cudaSetDevice(g->dev);
+    cudaDeviceSynchronize();
+    for (void* p : g->allocs) cudaFree(p);
+    delete g;
+}
+
+et_status et_get_info(const et_graph* g, et_graph_info* info) {
+    if (!g || !info) return ET_ERR_INVALID;
+    *info = g->info;
+    return ET_OK;
+}
+
+et_status et_run_splitk(et_graph* g, const float* A, int n_rows, float* Bpart, float* C, void* stream) {
+    if (!g || g->d.kind != ET_GRAPH_SPLITK) return ET_ERR_INVALID;
+    if (n_rows < 0 || n_rows > g->d.max_T) return ET_ERR_INVALID;
+    if (n_rows == 0) return ET_OK;
+    if (!aligned16(A) || !aligned16(Bpart) || !aligned16(C)) return ET_ERR_INVALID;
+    cudaStream_t s = (cudaStream_t)stream;
+    ET_CU(cudaSetDevice(g->dev));
+    SplitKParams p = g->sk;
+    p.A = A;
+    p.Bp = Bpart;
+    p.C = C;
+    p.rows = n_rows;
+    p.n_tiles = cdiv(n_rows, p.tile_rows);
+    ET_TRY(pre_run(g, s));
+    const int n_init = p.n_tiles * p.n_chunks;
+    RunArgs ra = run_args(g, n_rows, n_init, n_init + p.n_tiles);
+    ET_CU(launch_splitk(p, ra, g->n_ctas, s));
+    return ET_OK;
+}
+
+et_status et_run_mlp(et_graph* g, int B, const uint16_t* X, const uint16_t* gamma, const uint16_t* Wgu,
+                     const uint16_t* Wd, uint16_t* Y, void* stream) {
+    if (!g || g->d.kind != ET_GRAPH_MLP) return ET_ERR_INVALID;
+    if (B < 1 || B > g->d.max_T) return ET_ERR_INVALID;
+    if (!aligned16(X) || !aligned16(gamma) || !aligned16(Wgu) || !aligned16(Wd) || !aligned16(Y))
+        return ET_ERR_INVALID;
+    cudaStream_t s = (cudaStream_t)stream;
+    ET_CU(cudaSetDevice(g->dev));
+    MlpParams& p = g->mlp;
+    if (!g->mc[0].get(&p.tm_wgu, Wgu, 2ull * p.inter, p.hidden, 64)) return ET_ERR_CUDA;
+    if (!g->mc[1].get(&p.tm_wd, Wd, p.hidden, p.inter, 64)) return ET_ERR_CUDA;
+    p.X = X;
+    p.gamma = gamma;
+    p.Y = Y;
+    p.B = B;
+    ET_TRY(pre_run(g, s));
+    const int total = B + p.n_gu + p.n_m * p.n_c + p.n_m;
+    RunArgs ra = run_args(g, B, B, total);
+    ET_CU(launch_mlp(p, ra, g->n_ctas, s));
+    return ET_OK;
+}
+
+et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
+                     const uint16_t* W1, const uint16_t* W2, uint16_t* Y, int32_t* topk, float* topk_w,
+                     int32_t* indptr, int32_t* perm, float* logits, void* stream) {
+    if (!g || g->d.kind != ET_GRAPH_MOE) return ET_ERR_INVALID;
+    if (T < 1 || T > g->d.max_T) return ET_ERR_INVALID;
+    if (!aligned16(X) || !aligned16(Wr) || !bias || !aligned16(W1) || !aligned16(W2) || !aligned16(Y))
+        return ET_ERR_INVALID;
+    cudaStream_t s = (cudaStream_t)stream;
+    ET_CU(cudaSetDevice(g->dev));
+    MoeParams& p = g->moe;
+    if (!g->mc[0].get(&p.tm_wr, Wr, p.E, p.hidden, 64)) return ET_ERR_CUDA;
+    if (!g->mc[1].get(&p.tm_w1, W1, (uint64_t)p.E * 2 * p.inter, p.hidden, 64)) return ET_ERR_CUDA;
+    if (!g->mc[2].get(&p.tm_w2, W2, (uint64_t)p.E * p.hidden, p.inter, 64)) return ET_ERR_CUDA;
+    if (!g->mc[3].get(&p.tm_x, X, T, p.hidden, 16)) return ET_ERR_CUDA;
+    p.X = X;
+    p.bias = bias;
+    p.Y = Y;
+    p.out_topk = topk;
+    p.out_w = topk_w;
+    p.out_indptr = indptr;
+    p.out_perm = perm;
+    p.out_logits = logits;
+    p.T = T;
+    const int b = g->bucket_of(T);
+    const MoeShape mb = moe_shape(g, p, g->bucket_T[b]);
+    const MoeShape mt = moe_shape(g, p, T);
+    p.n_kc = mb.n_kc;  // the bucket fixes the router split (static lists and dynamic alike)
+    p.n_tt = mt.n_tt;
+    p.n_g = mt.n_g;
+    p.n_cb = mt.n_cb;
+    p.f_max = mb.f_max;
+    ET_TRY(pre_run(g, s));
+    RunArgs ra = run_args(g, T, p.n_tt * p.n_kc, 0);
+    ET_CU(launch_moe(p, ra, g->n_ctas, s));
+    return ET_OK;
+}
+
+et_status et_sync_status(et_graph* g, void* stream) {
+    if (!g) return ET_ERR_INVALID;
+    ET_CU(cudaSetDevice(g->dev));
+    ET_CU(cudaStreamSynchronize((cudaStream_t)stream));
+    Ctl h;
+    ET_CU(cudaMemcpy(&h, g->ctl, sizeof(Ctl), cudaMemcpyDeviceToHost));
+    if (h.status == 0) return ET_OK;
+    // reset: status, abort flag, counters, scratch that must start at zero
+    ET_CU(cudaMemset(g->ctl, 0, sizeof(Ctl)));
+    ET_CU(cudaMemset(g->ctr[0], 0, g->n_ctr * sizeof(int)));
+    ET_CU(cudaMemset(g->ctr[1], 0, g->n_ctr * sizeof(int)));
+    if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc)
+        ET_CU(cudaMemset(g->moe.Yacc, 0, (size_t)g->moe.maxT * g->moe.hidden * sizeof(float)));
+    ET_CU(cudaDeviceSynchronize());
+    // keep the diagnostic words readable through et_get_diag
+    ET_CU(cudaMemcpy(g->ctl->diag, h.diag, sizeof(h.diag), cudaMemcpyHostToDevice));
+    return (et_status)h.status;
+}
+
+et_status et_get_trace(et_graph* g, void* host_buf, size_t bytes, int* n_records) {
+    if (!g || !n_records) return ET_ERR_INVALID;
+    ET_CU(cudaSetDevice(g->dev));
+    ET_CU(cudaDeviceSynchronize());
+    Ctl h;
+    ET_CU(cudaMemcpy(&h, g->ctl, sizeof(Ctl), cudaMemcpyDeviceToHost));
+    int n = std::min(h.n_trace, g->trace_cap);
+    *n_records = n;
+    size_t want = std::min((size_t)n * sizeof(TraceRec), bytes);
+    if (host_buf && want) ET_CU(cudaMemcpy(host_buf, g->trace, want, cudaMemcpyDeviceToHost));
+    return ET_OK;
+}
+
+et_status et_get_diag(et_graph* g, int32_t* out8) {
+    if (!g || !out8) return ET_ERR_INVALID;
+    ET_CU(cudaSetDevice(g->dev));
+    ET_CU(cudaDeviceSynchronize());
+    ET_CU(cudaMemcpy(out8, g->ctl->diag, 8 * sizeof(int32_t), cudaMemcpyDeviceToHost));
+    return ET_OK;
+}
+
+}  // extern "C"

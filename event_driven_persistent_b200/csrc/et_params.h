@@ -1,0 +1,96 @@
+// Kernel parameter blocks of the three megakernels (host and device).
+#pragma once
+#include <cuda.h>
+#include <stdint.h>
+
+#include "et_shared.h"
+
+namespace et {
+
+// ------------------------------------------------------------------ split-K
+// Tasks: P(i, j) partial of row tile i, K-chunk j; F(i) final of row tile i.
+// Events (counter-set index): E[i] = ev_base + i; unfused barrier = ev_all.
+struct SplitKParams {
+    const float* A;
+    float* Bp;
+    float* C;
+    int rows, cols, chunk, tile_rows;
+    int n_tiles, n_chunks;
+    int ev_base, ev_all;
+    int unfused;
+    int bad_count;
+};
+
+// ---------------------------------------------------------------------- MLP
+// Tasks: NORM(b), GU(n) gate/up tile n, DOWN(m, c), RED(m).
+// Events: E_norm (count B), E_h[c] (count gu_per_chunk), E_y[m] (count
+// n_chunks); unfused: E_gu_all (count n_gu), E_down_all (count n_m*n_c).
+enum { MLP_MAP_WGU = 0, MLP_MAP_WD = 1, MLP_MAP_XN = 2, MLP_MAP_H = 3 };
+struct MlpParams {
+    CUtensorMap tm_wgu;  // Wgu [2I, H], box 64 x 64
+    CUtensorMap tm_wd;   // Wd  [H, I], box 64 x 64
+    CUtensorMap tm_xn;   // xn  [maxB, H] (workspace), box 64 x 16
+    CUtensorMap tm_h;    // h   [maxB, I] (workspace), box 64 x 16
+    const uint16_t* X;
+    const uint16_t* gamma;
+    uint16_t* xn;
+    uint16_t* h;
+    float* part;         // [n_c, maxB, H] fp32 partial sums of the down GEMM
+    uint16_t* Y;
+    int B, hidden, inter, maxB;
+    float eps;
+    int gu_tile, down_tile, kchunk;
+    int n_gu, n_m, n_c, gu_per_chunk;
+    int ev_norm, ev_h, ev_y, ev_gu_all, ev_down_all;
+    int unfused;
+    int bad_count;
+};
+
+// ---------------------------------------------------------------------- MoE
+// Tasks: RT(tt, kc) router partial (tensor core), TK(tt) top-k,
+// SC scan, GR(g) grouping, S1(f, n) stage-1 tile, S2(f, n) stage-2 tile,
+// CB(b) combine.
+enum { MOE_MAP_WR = 0, MOE_MAP_W1 = 1, MOE_MAP_W2 = 2, MOE_MAP_X = 3, MOE_MAP_XP = 4, MOE_MAP_HM = 5 };
+struct MoeParams {
+    CUtensorMap tm_wr;  // Wr [E, H], box 64 x 64
+    CUtensorMap tm_w1;  // W1 [E*2I, H], box 64 x 64
+    CUtensorMap tm_w2;  // W2 [E*H, I], box 64 x 64
+    CUtensorMap tm_x;   // X  [T, H], box 64 x 16
+    CUtensorMap tm_xp;  // Xp [maxT*k, H] (workspace), box 64 x 16
+    CUtensorMap tm_hm;  // Hm [maxT*k, I] (workspace), box 64 x 16
+    const uint16_t* X;
+    const float* bias;
+    uint16_t* Y;
+    // optional exports
+    int32_t* out_topk;
+    float* out_w;
+    int32_t* out_indptr;
+    int32_t* out_perm;
+    float* out_logits;
+    // workspace
+    float* lpart;       // [n_kc, maxT, E] router partial logits
+    float* logits;      // [maxT, E]
+    int32_t* topk;      // [maxT, k]
+    float* topw;        // [maxT, k]
+    int32_t* gcnt;      // [n_g, E] pairs of group tile g per expert
+    int32_t* goff;      // [n_g, E] first grouped row of tile g's pairs of expert e
+    int32_t* counts;    // [E]
+    int32_t* indptr;    // [E+1]
+    int32_t* tindptr;   // [E+1] m-tile CSR
+    int32_t* mt_expert; // [F_max] expert of flat m-tile f
+    int32_t* perm;      // [maxT*k]
+    int32_t* pos;       // [maxT*k]
+    int32_t* scal;      // [8]: 0 = total m-tiles
+    uint16_t* Xp;       // [maxT*k, H] grouped token rows
+    uint16_t* Hm;       // [maxT*k, I] stage-1 output, grouped order
+    float* Yacc;        // [maxT, H] fp32 combine accumulator (kept zero between runs)
+    int T, hidden, inter, E, k, maxT;
+    int tt, n_tt, n_kc, gt, n_g, bm, n1_tile, n_n1, n2_tile, n_n2, cb, n_cb;
+    int f_max;          // static: m-tile slots of this bucket
+    // events
+    int ev_rt, ev_tk, ev_sc, ev_grp, ev_exp, ev_s1, ev_cb, ev_rt_all, ev_s1_all, ev_s2_all;
+    int sched;          // et_sched
+    int bad_count;
+};
+
+}  // namespace et

@@ -1,0 +1,67 @@
+// Types shared by the host and device halves of libet (not part of the C ABI).
+#pragma once
+#include <stdint.h>
+
+#include "../../include/et.h"
+
+namespace et {
+
+typedef et_trace_record TraceRec;
+
+// Launch shape of every megakernel: warp 0 fetches tasks and drives TMA,
+// warp 1 issues tcgen05 MMAs, warps 2..5 run epilogues and CUDA-core tasks.
+constexpr int kThreads = 192;
+constexpr int kExecThreads = 128;
+constexpr int kExecWarp0 = 2;
+constexpr int kRing = 2;           // task ring depth (warp 0 runs one task ahead)
+constexpr int kStages = 6;         // smem pipeline stages of the GEMM engine
+constexpr int kTileK = 64;         // K elements per stage (one 128-byte swizzle row)
+constexpr int kAStageBytes = 128 * 128;  // 128 rows x 128 B
+constexpr int kBStageBytes = 128 * 128;  // up to 128 rows x 128 B
+constexpr int kStageBytes = kAStageBytes + kBStageBytes;
+constexpr int kMaxN = 128;         // largest MMA N (token rows per tile)
+constexpr int kTmemCols = 256;     // two accumulators of kMaxN fp32 columns
+constexpr int kEpiBytes = 64 * 32 * 4;   // gate/up exchange staging
+constexpr int kSimtBytes = 16384;        // scratch for CUDA-core tasks
+constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + kSimtBytes + 1024 /*barriers*/;
+
+// Per-bucket static task lists: CSR over CTAs.
+struct StaticLists {
+    const int* off;    // [n_ctas + 1]
+    const uint32_t* words;
+};
+
+// Device control block of a graph (lives in its workspace).
+struct Ctl {
+    int status;       // sticky error code (0 = ok), cleared by the host
+    int abort;        // raised with status; every spin checks it
+    int diag[8];      // where the first error happened
+    unsigned ticket;  // trace ticket counter
+    int n_trace;      // trace records written
+    int pad[4];
+};
+
+// Per-run arguments common to every megakernel.
+struct RunArgs {
+    Ctl* ctl;
+    int* ctr;                  // this run's counter set (zero at entry)
+    int* ctr_next;             // the other set, zeroed during this run
+    int n_ctr;
+    unsigned long long* qslots;
+    int qcap;
+    uint32_t epoch;            // run number, >= 1
+    int n_init;                // dynamic: initial tasks (implicit slots)
+    int total_static;          // dynamic: task count when known at launch (else 0)
+    int dynamic;
+    int fetch_batch;
+    int debug;
+    TraceRec* trace;
+    int trace_cap;
+    StaticLists lists;         // static / unfused: this size bucket's lists
+    unsigned long long timeout_ns;
+};
+
+// Counter-set slots every workload reserves at the front.
+constexpr int kCtrHead = 0, kCtrTail = 1, kCtrTotal = 2, kCtrFirstEvent = 4;
+
+}  // namespace et

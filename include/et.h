@@ -1,0 +1,205 @@
+/*
+ * et.h -- C ABI of the event-tensor megakernel library (libet.so).
+ *
+ * One persistent kernel launch runs every tiled task of a small operator
+ * graph.  Tasks are ordered by event tensors: arrays of counters with a
+ * symbolic shape; a producer task notifies an event, a consumer task runs
+ * once the event has received its wait count of notifications.  Sources,
+ * cited by page title and section:
+ *   [ETN] "Event Tensor：用“事件张量”编译动态 Megakernel" (reading notes on
+ *         "Event Tensor: A Unified Abstraction for Compiling Dynamic
+ *         Megakernel", MLSys 2026)
+ *   [ETS] hyper.ai summary of the same paper, §方法
+ *   [WV]  "MoE Kernel动态SM调度：从静态分配到任务池，4卡H100加速2.89×"
+ *         (batched atomic pops, §2.2)
+ *
+ * Conventions for every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *    contiguous, 16-byte aligned.  bf16 tensors are passed as uint16_t bit
+ *    patterns.  The library never frees or retains them past the call.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Runs are
+ *    asynchronous: et_run_* returns after the launch; device-side errors
+ *    (a wait that timed out) are reported by et_sync_status.
+ *  - The token / batch count T (or B, or the split-K row count) is a plain
+ *    run-time int: the same graph and binary serve every value up to
+ *    max_T with no recompile and no graph capture ([ETN] §Shape dynamism).
+ *  - A graph owns its workspace (event counters, ready queue, static task
+ *    lists, scratch tensors, status word, trace buffer).  Runs of one graph
+ *    must be issued on one stream, one after another; the library is not
+ *    re-entrant per graph.  Different graphs are independent.
+ *  - Errors: every function returns an et_status; ET_OK = 0.
+ */
+#ifndef ET_H_
+#define ET_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ET_OK = 0,
+    ET_ERR_INVALID = 1,     /* bad argument: null/misaligned pointer, T out of range, wrong graph kind */
+    ET_ERR_CUDA = 2,        /* a CUDA runtime/driver call failed */
+    ET_ERR_TIMEOUT = 3,     /* a device-side wait exceeded its time limit (see et_sync_status) */
+    ET_ERR_OOM = 4,         /* workspace allocation failed */
+    ET_ERR_UNSUPPORTED = 5, /* device is not sm_100, or dims outside what the kernels tile */
+    ET_ERR_PENDING = 6      /* an earlier run failed and its error was not yet collected by et_sync_status */
+} et_status;
+
+/* How tasks are ordered on the SMs ([ETN] §静态调度, §动态调度, §静态与动态调度的消融). */
+typedef enum {
+    ET_SCHED_STATIC = 0,  /* per-SM task lists fixed at build time (one set per power-of-two
+                             size bucket); consumers spin-wait on their events */
+    ET_SCHED_DYNAMIC = 1, /* a device-side ready queue: a producer that brings an event to its
+                             wait count pushes the consumers; SMs pop in batches */
+    ET_SCHED_UNFUSED = 2  /* control: the static lists with one barrier event between
+                             consecutive operators (the "unfused megakernel" baseline) */
+} et_sched;
+
+typedef enum { ET_GRAPH_SPLITK = 0, ET_GRAPH_MLP = 1, ET_GRAPH_MOE = 2 } et_graph_kind;
+
+/* debug_flags bits */
+#define ET_DEBUG_TRACE 1      /* record one et_trace_record per task (tickets from one global counter) */
+#define ET_DEBUG_DELAY 2      /* each task first spins a pseudo-random 0..~20 us, to perturb the order */
+#define ET_DEBUG_BAD_COUNT 4  /* raise one event's wait count by one: a run must then end in
+                                 ET_ERR_TIMEOUT (used to test the timeout path) */
+
+typedef struct {
+    int kind;            /* et_graph_kind */
+    int sched;           /* et_sched */
+    int max_T;           /* largest T (MoE tokens), B (MLP batch) or split-K row count */
+    /* dims; 0 = the default in brackets */
+    int hidden;          /* MLP [4096] / MoE [2048] model width */
+    int inter;           /* MLP [14336] / MoE [768] intermediate width */
+    int n_experts;       /* MoE [128] */
+    int top_k;           /* MoE [8] */
+    int splitk_cols;     /* split-K columns [128] */
+    int splitk_chunk;    /* split-K K-chunk [32] */
+    int splitk_tile_rows;/* split-K rows per task [32] */
+    float rms_eps;       /* MLP RMSNorm epsilon [1e-5] */
+    int fetch_batch;     /* dynamic: tasks claimed per atomic pop [workload default] */
+    int debug_flags;     /* ET_DEBUG_* */
+    int device;          /* CUDA device ordinal */
+    int n_ctas;          /* persistent CTAs [0 = one per SM] */
+    float timeout_ms;    /* per-wait device time limit [1000] */
+} et_graph_desc;
+
+typedef struct et_graph et_graph; /* opaque, library-owned */
+
+/* Tile parameters of a built graph (what the task coordinates mean). */
+typedef struct {
+    int kind, sched, max_T, n_ctas, threads, smem_bytes, fetch_batch;
+    int hidden, inter, n_experts, top_k;
+    int splitk_cols, splitk_chunk, splitk_tile_rows;
+    int mlp_gu_tile;     /* intermediate columns per gate/up task */
+    int mlp_down_tile;   /* output columns per down task */
+    int mlp_kchunk;      /* K (intermediate) columns per down task */
+    int moe_tt;          /* tokens per router/top-k tile */
+    int moe_gt;          /* tokens per grouping task */
+    int moe_bm;          /* rows (token, slot pairs) per expert m-tile */
+    int moe_n1_tile;     /* intermediate columns per stage-1 task */
+    int moe_n2_tile;     /* output columns per stage-2 task */
+    int moe_cb;          /* tokens per combine task */
+    int moe_router_kc;   /* router K-chunks at this graph's max_T bucket */
+} et_graph_info;
+
+/* Trace record (ET_DEBUG_TRACE): one per executed task. */
+typedef struct {
+    int32_t op, a, b, sm;
+    uint32_t start; /* ticket taken after the task's wait succeeded */
+    uint32_t end;   /* ticket taken after its outputs were written, before its notify */
+} et_trace_record;
+
+/* trace op codes */
+#define ET_OP_SK_PARTIAL 1
+#define ET_OP_SK_FINAL 2
+#define ET_OP_MLP_NORM 10
+#define ET_OP_MLP_GATEUP 11
+#define ET_OP_MLP_DOWN 12
+#define ET_OP_MLP_REDUCE 13
+#define ET_OP_MOE_ROUTER 20
+#define ET_OP_MOE_TOPK 21
+#define ET_OP_MOE_SCAN 22
+#define ET_OP_MOE_GROUP 23
+#define ET_OP_MOE_S1 24
+#define ET_OP_MOE_S2 25
+#define ET_OP_MOE_COMBINE 26
+
+/* Build a graph: validate dims, allocate its workspace for max_T, build the
+ * static per-SM task lists for every power-of-two bucket up to max_T
+ * ([ETN] §静态调度: "per-SM task queue" materialised at build time; an
+ * unsampled size reuses the next larger bucket).  Host-side, once.
+ * Errors: ET_ERR_INVALID (bad desc), ET_ERR_UNSUPPORTED (not sm_100 or dims
+ * the tiles do not cover), ET_ERR_OOM, ET_ERR_CUDA. */
+et_status et_build_graph(const et_graph_desc* desc, et_graph** out);
+
+/* Two-stage split-K reduction ([ETN] §Split-K reduction 示例):
+ *   Bpart[i,j] = sum_{k=chunk*j}^{chunk*j+chunk-1} A[i,k]   (j < ceil(cols/chunk))
+ *   C[i]       = sum_j Bpart[i,j]
+ * One task per (row tile i, chunk j) notifies E[i] ("ij->i"); the final
+ * task of row tile i waits for E[i] ("i->i"), wait count = #chunks.
+ * A: fp32 [n_rows, cols]; Bpart: fp32 [n_rows, nchunk]; C: fp32 [n_rows].
+ * 0 <= n_rows <= max_T (n_rows = 0 launches nothing). */
+et_status et_run_splitk(et_graph* g, const float* A, int n_rows, float* Bpart, float* C,
+                        void* stream);
+
+/* Fused decode MLP (RMSNorm -> gate/up GEMM -> SiLU*mul -> down GEMM) of
+ * [ETN] §端到端低 batch serving ("Norm, MLP" of the decoding pipeline,
+ * weights prefetched before activations arrive):
+ *   xn = bf16(x * rsqrt(mean(x^2) + eps) * gamma)
+ *   h  = bf16(silu(xn Wg^T) * (xn Wu^T))
+ *   Y  = bf16(h Wd^T)                 (fp32 accumulation throughout)
+ * X bf16 [B, hidden]; gamma bf16 [hidden]; Wgu bf16 [2*inter, hidden]
+ * (gate rows first, then up rows); Wd bf16 [hidden, inter]; Y bf16
+ * [B, hidden].  1 <= B <= max_T <= 128. */
+et_status et_run_mlp(et_graph* g, int B, const uint16_t* X, const uint16_t* gamma,
+                     const uint16_t* Wgu, const uint16_t* Wd, uint16_t* Y, void* stream);
+
+/* MoE layer ([ETN] §Data-dependent event update, §Data-dependent task
+ * triggering, §完整 MoE layer): router -> top-k -> token grouping ->
+ * stage-1 grouped GEMM + SiLU*mul -> stage-2 grouped GEMM -> weighted
+ * combine, in one launch.
+ *   logits[t,e] = x_t . Wr_e + bias[e]           (fp32)
+ *   topk[t,:]   = the top_k experts by logit, ties -> lower index, in order
+ *   w[t,:]      = softmax of the selected logits  (fp32)
+ *   h           = bf16(silu(x W1g_e^T) * (x W1u_e^T)),  o = h W2_e^T
+ *   Y[t]        = bf16(sum_s w[t,s] * o[t,s])
+ * X bf16 [T, hidden]; Wr bf16 [E, hidden]; bias fp32 [E]; W1 bf16
+ * [E, 2*inter, hidden] (gate rows first); W2 bf16 [E, hidden, inter];
+ * Y bf16 [T, hidden].  Optional outputs (NULL to skip): topk int32 [T,k],
+ * topk_w fp32 [T,k], indptr int32 [E+1] (pairs per expert, CSR), perm int32
+ * [T*k] (pairs t*k+s grouped by expert, ascending t), logits fp32 [T,E].
+ * 1 <= T <= max_T. */
+et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
+                     const uint16_t* W1, const uint16_t* W2, uint16_t* Y, int32_t* topk,
+                     float* topk_w, int32_t* indptr, int32_t* perm, float* logits, void* stream);
+
+/* Synchronise `stream`, then read and clear the graph's sticky device
+ * status.  Returns ET_OK, or ET_ERR_TIMEOUT if a wait of any run since the
+ * last call gave up (every CTA then drained and exited; no trap).  After a
+ * device error the workspace (counters, scratch) is reset here, so the next
+ * run starts clean; until then et_run_* refuses with ET_ERR_PENDING. */
+et_status et_sync_status(et_graph* g, void* stream);
+
+/* Copy the trace of the last run (ET_DEBUG_TRACE) to host memory.
+ * Synchronises the device.  *n_records receives the record count; at most
+ * bytes / sizeof(et_trace_record) records are copied. */
+et_status et_get_trace(et_graph* g, void* host_buf, size_t bytes, int* n_records);
+
+/* Tile parameters of a built graph. */
+et_status et_get_info(const et_graph* g, et_graph_info* info);
+
+/* Diagnostic words of the last device error (which wait, which task);
+ * 8 ints.  Synchronises the device. */
+et_status et_get_diag(et_graph* g, int32_t* out8);
+
+void et_destroy_graph(et_graph* g);
+const char* et_status_str(et_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ET_H_ */

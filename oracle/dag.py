@@ -120,20 +120,20 @@ def mlp_graph(B, hidden, inter, gu_tile, down_tile, kchunk, sched):
     return g.finish()
 
 
-def moe_graph(topk, E, hidden, inter, tt, ec, bm, n1_tile, n2_tile, cb, sched):
+def moe_graph(topk, E, tt, n_kc, gt, bm, n_n1, n_n2, cb, sched):
     """MoE layer, expanded with the runtime routing `topk` [T, k]:
-      router (t, c)   --"tc->t"-->           E_rt[t]         (count = #expert chunks)
+      router (t, c)   --"tc->t"-->           E_rt[t]         (count = #K chunks)
       E_rt[t]         --"t->t"-->            topk t
       topk t          --"t->"-->             E_tk            (count = #token tiles)
       E_tk            -->                    scan
       scan            -->                    E_sc            (count 1)
-      E_sc            --"->t"-->             group t
-      group t         --> E_exp[topk[i,:]] for every token i of tile t
+      E_sc            --"->g"-->             group g
+      group g         --> E_exp[topk[i,:]] for every token i of group g
                                                (count of E_exp[e] = #pairs routed to e)
       E_exp[e]        --> stage1 tasks[task_indptr[e] : task_indptr[e+1]] x n1 tiles
       stage1 (f, n)   --"fn->f"-->           E_s1[f]         (count = #n1 tiles)
       E_s1[f]         --"f->fn"-->           stage2 (f, n)
-      stage2 (f, n)   --> E_cb[i // cb] for every row i of m-tile f (data-dependent)
+      stage2 (f, n)   --> E_cb[i // cb] for every row (token i) of m-tile f
       E_cb[b]         -->                    combine b
     Static scheduling replaces group -> E_exp -> stage1 by one coarse event
     (every group task -> every stage1 task).  Unfused replaces every
@@ -142,9 +142,7 @@ def moe_graph(topk, E, hidden, inter, tt, ec, bm, n1_tile, n2_tile, cb, sched):
     T, k = topk.shape
     g = Graph()
     n_tt = _cdiv(T, tt)
-    n_ec = _cdiv(E, ec)
-    n_n1 = _cdiv(inter, n1_tile)
-    n_n2 = _cdiv(hidden, n2_tile)
+    n_g = _cdiv(T, gt)
     n_cb = _cdiv(T, cb)
     unf = sched == "unfused"
     static = sched == "static"
@@ -159,7 +157,7 @@ def moe_graph(topk, E, hidden, inter, tt, ec, bm, n1_tile, n2_tile, cb, sched):
         for m in range(_cdiv(len(r), bm)):
             mtiles.append((e, m, r[m * bm:(m + 1) * bm]))
     for t in range(n_tt):
-        for c in range(n_ec):
+        for c in range(n_kc):
             task = (OP_MOE_ROUTER, t, c)
             g.add_task(task)
             g.produce(task, ("E_rt_all",) if unf else ("E_rt", t))
@@ -172,14 +170,14 @@ def moe_graph(topk, E, hidden, inter, tt, ec, bm, n1_tile, n2_tile, cb, sched):
     g.add_task(scan)
     g.consume(scan, ("E_tk",))
     g.produce(scan, ("E_sc",))
-    for t in range(n_tt):
-        task = (OP_MOE_GROUP, t, 0)
+    for q in range(n_g):
+        task = (OP_MOE_GROUP, q, 0)
         g.add_task(task)
         g.consume(task, ("E_sc",))
         if unf or static:
             g.produce(task, ("E_grp",))
         else:
-            for i in range(t * tt, min(T, (t + 1) * tt)):
+            for i in range(q * gt, min(T, (q + 1) * gt)):
                 for s in range(k):
                     g.produce(task, ("E_exp", int(topk[i, s])))
     for f, (e, m, rows) in enumerate(mtiles):

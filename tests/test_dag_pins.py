@@ -28,10 +28,9 @@ def test_splitk_unfused_is_a_barrier():
 
 
 def test_moe_tiny_by_hand():
-    # T=2 tokens, k=2, E=3 experts, one token tile, one expert chunk, bm=1
+    # T=2 tokens, k=2, E=3 experts, one token tile, one K chunk, one group, bm=1
     topk = np.array([[2, 0], [0, 1]])
-    g, mtiles = dag.moe_graph(topk, E=3, hidden=4, inter=4, tt=2, ec=4, bm=1,
-                              n1_tile=4, n2_tile=4, cb=1, sched="dynamic")
+    g, mtiles = dag.moe_graph(topk, E=3, tt=2, n_kc=1, gt=2, bm=1, n_n1=1, n_n2=1, cb=1, sched="dynamic")
     # grouping: expert 0 <- (0,1),(1,0); expert 1 <- (1,1); expert 2 <- (0,0); bm=1 -> 4 m-tiles
     assert [(e, m, rows) for (e, m, rows) in mtiles] == [
         (0, 0, [(0, 1)]), (0, 1, [(1, 0)]), (1, 0, [(1, 1)]), (2, 0, [(0, 0)])]
