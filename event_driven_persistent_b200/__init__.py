@@ -44,12 +44,13 @@ class et_graph_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "kind", "sched", "max_T", "n_ctas", "threads", "smem_bytes", "fetch_batch", "hidden", "inter",
         "n_experts", "top_k", "splitk_cols", "splitk_chunk", "splitk_tile_rows", "mlp_gu_tile", "mlp_down_tile",
-        "mlp_kchunk", "moe_tt", "moe_gt", "moe_bm", "moe_n1_tile", "moe_n2_tile", "moe_cb", "moe_router_kc")]
+        "mlp_kchunk", "moe_tt", "moe_gt", "moe_tkt", "moe_bm", "moe_n1_tile", "moe_n2_tile", "moe_cb", "moe_router_kc")]
 
 
 class et_trace_record(ctypes.Structure):
     _fields_ = [("op", ctypes.c_int32), ("a", ctypes.c_int32), ("b", ctypes.c_int32), ("sm", ctypes.c_int32),
-                ("start", ctypes.c_uint32), ("end", ctypes.c_uint32)]
+                ("start", ctypes.c_uint32), ("end", ctypes.c_uint32), ("t_fetch", ctypes.c_uint64),
+                ("t_ready", ctypes.c_uint64), ("t_acc", ctypes.c_uint64), ("t_end", ctypes.c_uint64)]
 
 
 _P = ctypes.c_void_p
@@ -129,12 +130,13 @@ def et_sync_status(g, stream=None):
 
 
 def et_get_trace(g):
-    """List of (op, a, b, sm, start, end) tuples of the last traced run."""
+    """List of (op, a, b, sm, start, end, t_fetch, t_ready, t_acc, t_end)
+    tuples of the last traced run (tickets, then %globaltimer ns)."""
     n = _I(0)
     _check(_lib.et_get_trace(g, None, 0, ctypes.byref(n)), "et_get_trace")
     buf = (et_trace_record * max(n.value, 1))()
     _check(_lib.et_get_trace(g, ctypes.cast(buf, _P), ctypes.sizeof(buf), ctypes.byref(n)), "et_get_trace")
-    return [(r.op, r.a, r.b, r.sm, r.start, r.end) for r in buf[:n.value]]
+    return [(r.op, r.a, r.b, r.sm, r.start, r.end, r.t_fetch, r.t_ready, r.t_acc, r.t_end) for r in buf[:n.value]]
 
 
 def et_get_info(g):

@@ -64,6 +64,29 @@ __device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned l
 
 __device__ __forceinline__ int ld_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
 
+__device__ __forceinline__ int ld_relaxed(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+// after a relaxed load observed a released value: acquire (fence) once
+__device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Spin back-off: 148 SMs polling a few counters must not flood the L2 slice
+// that holds them (which slows every other access to that slice).
+struct Backoff {
+    uint32_t ns = 32;
+    __device__ __forceinline__ void pause() {
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+    }
+};
+
 // atomic add, acquire+release at GPU scope; returns the old value
 __device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
     int old;
@@ -112,6 +135,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+
+// ------------------------------------------------------------- cp.async ----
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// the mbarrier's next phase also waits for every cp.async this thread issued
+// so far (the pending count is raised now and lowered when they land)
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* b) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // ----------------------------------------------------------------- TMA ----
 
@@ -227,9 +262,13 @@ static __device__ __noinline__ bool wait_geq(const int* ctr, int target, Ctl* ct
                                       int ev) {
     if (ld_acquire(ctr) >= target) return true;
     uint64_t t0 = globaltimer();
+    Backoff bo;
     for (uint32_t it = 1;; ++it) {
-        __nanosleep(64);
-        if (ld_acquire(ctr) >= target) return true;
+        bo.pause();
+        if (ld_relaxed(ctr) >= target) {
+            fence_acquire();
+            return true;
+        }
         if ((it & 31) == 0) {
             if (aborted(ctl)) return false;
             if (globaltimer() - t0 > timeout_ns || it > kMaxSpinIters) {
@@ -248,8 +287,9 @@ __device__ __forceinline__ int notify(int* ctr, int n) {
     return atom_add_acq_rel(ctr, n) + n;
 }
 
-// bounded mbarrier wait (parity); false on timeout/abort
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Ctl* ctl, uint64_t timeout_ns, int where) {
+// bounded mbarrier wait (parity); false on timeout/abort.  Out of line: it
+// has many call sites and the megakernel's instruction footprint matters.
+static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Ctl* ctl, uint64_t timeout_ns, int where) {
     if (mbar_try_wait(b, parity)) return true;
     uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
@@ -268,23 +308,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Ctl* ctl
 
 __device__ __forceinline__ uint32_t take_ticket(Ctl* ctl) { return atomicAdd(&ctl->ticket, 1u); }
 
-__device__ __forceinline__ void trace_write(Ctl* ctl, TraceRec* buf, int cap, int op, int a, int b,
-                                            uint32_t start, uint32_t end) {
+__device__ __forceinline__ void trace_write(Ctl* ctl, TraceRec* buf, int cap, const TraceRec& r) {
     int i = atomicAdd(&ctl->n_trace, 1);
-    if (i < cap) {
-        TraceRec r;
-        r.op = op;
-        r.a = a;
-        r.b = b;
-        r.sm = (int)smid();
-        r.start = start;
-        r.end = end;
-        buf[i] = r;
-    }
+    if (i < cap) buf[i] = r;
 }
 
 // pseudo-random delay (debug): 0 .. ~20 us
-__device__ __forceinline__ void debug_delay(uint32_t key) {
+static __device__ __noinline__ void debug_delay(uint32_t key) {
     uint32_t h = key * 2654435761u;
     h ^= h >> 15;
     h *= 2246822519u;
@@ -323,6 +353,13 @@ __device__ __forceinline__ int q_reserve(const Queue& q, int n) { return q.n_ini
 __device__ __forceinline__ void q_publish(const Queue& q, int idx, uint32_t word) {
     if (idx < q.cap) st_release_u64(&q.slots[idx], ((unsigned long long)q.epoch << 32) | word);
 }
+// Publish after the caller issued one release fence for the whole batch.
+__device__ __forceinline__ void q_publish_after_fence(const Queue& q, int idx, uint32_t word) {
+    if (idx < q.cap)
+        asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(&q.slots[idx]),
+                     "l"(((unsigned long long)q.epoch << 32) | word)
+                     : "memory");
+}
 
 // Resolve slot `idx`: 1 = task in *word, 0 = no more tasks (idx beyond the
 // run's total), -1 = timeout/abort.
@@ -336,16 +373,18 @@ __device__ __forceinline__ int q_resolve(const Queue& q, int idx, uint32_t* word
     if (idx >= q.cap) return 0;  // beyond any run's last task
     const unsigned long long* s = &q.slots[idx];
     uint64_t t0 = 0;
+    Backoff bo;
     for (uint32_t it = 0;; ++it) {
-        unsigned long long v = ld_acquire_u64(s);
+        unsigned long long v = ld_relaxed_u64(s);
         if ((uint32_t)(v >> 32) == q.epoch) {
+            fence_acquire();
             *word = (uint32_t)v;
             return 1;
         }
-        int tot = q.total_static > 0 ? q.total_static + 1 : ld_acquire(q.total);
+        int tot = q.total_static > 0 ? q.total_static + 1 : ld_relaxed(q.total);
         if (tot > 0 && idx >= tot - 1) return 0;
         if (it == 0) t0 = globaltimer();
-        __nanosleep(32);
+        bo.pause();
         if ((it & 31) == 31) {
             if (aborted(ctl)) return -1;
             if (globaltimer() - t0 > timeout_ns || it > kMaxSpinIters) {

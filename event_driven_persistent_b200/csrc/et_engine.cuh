@@ -33,6 +33,8 @@ struct TaskDesc {
     int valid;       // 0 = a static slot with nothing to do at this size
     uint32_t start;  // trace ticket taken after the task's wait
     int gemm;        // 1 = tensor-core task
+    int gather;      // 1 = B rows gathered through W::gather_row (cp.async), else B by TMA
+    uint64_t t_fetch, t_ready, t_acc;  // trace timestamps (ns)
     int a_map, a_row0, a_row1;  // A: tensor map id, rows of the two 64-row boxes
     int b_map, b_row0;          // B: tensor map id, first row
     int n;                      // MMA N (multiple of 16, <= kMaxN)
@@ -51,7 +53,10 @@ struct SmemCtl {
     uint32_t tmem_base;
     int start_status;
     int bcast[8];
+    uint64_t bcast64[2];
     TaskDesc ring[kRing];
+    TaskDesc pd;  // warp 0: the task lane 0 fetched, for the other lanes
+    int pr, pbrk, pok;
 };
 
 // Everything a role needs besides the workload parameters.
@@ -80,7 +85,8 @@ __device__ __forceinline__ void group_push(Ctx& x, int n, Gen gen) {
     if (x.tid == 0) x.sc->bcast[0] = q_reserve(x.q, n);
     exec_bar();
     int base = x.sc->bcast[0];
-    for (int i = x.tid; i < n; i += kExecThreads) q_publish(x.q, base + i, gen(i));
+    if (x.tid < n) __threadfence();  // release: this task's writes before its pushes
+    for (int i = x.tid; i < n; i += kExecThreads) q_publish_after_fence(x.q, base + i, gen(i));
     exec_bar();
 }
 
@@ -89,7 +95,8 @@ template <class Gen>
 __device__ __forceinline__ void thread_push(Ctx& x, int n, Gen gen) {
     if (n <= 0) return;
     int base = q_reserve(x.q, n);
-    for (int i = 0; i < n; ++i) q_publish(x.q, base + i, gen(i));
+    __threadfence();
+    for (int i = 0; i < n; ++i) q_publish_after_fence(x.q, base + i, gen(i));
 }
 
 // End of a task in the exec group: every thread has written its outputs.
@@ -100,8 +107,18 @@ __device__ __forceinline__ bool group_finish_notify(Ctx& x, const TaskDesc& d, i
     if (x.tid == 0) {
         int fired = 0;
         if (x.debug & ET_DEBUG_TRACE) {
-            uint32_t end = take_ticket(x.ctl);
-            trace_write(x.ctl, x.trace, x.trace_cap, task_op(d.word), task_a(d.word), task_b(d.word), d.start, end);
+            TraceRec r;
+            r.end = take_ticket(x.ctl);
+            r.t_end = globaltimer();
+            r.op = task_op(d.word);
+            r.a = task_a(d.word);
+            r.b = task_b(d.word);
+            r.sm = (int)smid();
+            r.start = d.start;
+            r.t_fetch = d.t_fetch;
+            r.t_ready = d.t_ready;
+            r.t_acc = d.t_acc;
+            trace_write(x.ctl, x.trace, x.trace_cap, r);
         }
         if (ctr) fired = notify(ctr, n) == target;
         x.sc->bcast[1] = fired;
@@ -114,13 +131,18 @@ __device__ __forceinline__ bool group_finish_notify(Ctx& x, const TaskDesc& d, i
 __device__ __forceinline__ bool group_wait(Ctx& x, TaskDesc& d, const int* ctr, int target, int where) {
     if (x.tid == 0) {
         bool ok = ctr == nullptr || wait_geq(ctr, target, x.ctl, x.timeout_ns, where, task_word(0, 0, 0) ^ d.word);
-        if (ok && (x.debug & ET_DEBUG_TRACE)) d.start = take_ticket(x.ctl);
+        if (ok && (x.debug & ET_DEBUG_TRACE)) {
+            d.start = take_ticket(x.ctl);
+            d.t_ready = globaltimer();
+        }
         x.sc->bcast[2] = ok;
         x.sc->bcast[3] = (int)d.start;
+        x.sc->bcast64[0] = d.t_ready;
     }
     exec_bar();
     bool ok = x.sc->bcast[2] != 0;
     d.start = (uint32_t)x.sc->bcast[3];
+    d.t_ready = x.sc->bcast64[0];
     exec_bar();
     return ok;
 }
@@ -130,6 +152,7 @@ __device__ __forceinline__ bool group_wait(Ctx& x, TaskDesc& d, const int* ctr, 
 //   W::derive(p, x, word, d)           fill a TaskDesc (warp 0; may wait in
 //                                      static mode); false = abort
 //   W::gemm_wait(p, x, d)              the GEMM task's input wait (warp 0)
+//   W::gather_row(p, d, r)             B row r of a gather task (d.gather)
 //   W::a_map(p, id), W::b_map(p, id)   tensor maps
 //   W::epilogue(p, x, d, acc_taddr)    exec group, after the accumulator is ready
 //   W::simt(p, x, d)                   exec group, a CUDA-core task
@@ -204,23 +227,29 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     for (int s = 0; s < kStages; ++s) armed[s] = 0;
 
     if (!skip && warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------ task source + TMA
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_a = policy_evict_last();
-            int lpos = 0, lend = 0;
-            if (!x.dynamic) {
-                lpos = ra.lists.off[blockIdx.x];
-                lend = ra.lists.off[blockIdx.x + 1];
-            }
-            int qn = 0, qe = 0;
-            uint32_t st = 0;  // stages armed so far (ring position)
-            for (uint32_t it = 0;; ++it) {
+        // ---------------------------------------------------- task source + loads
+        // Lane 0 leads (task fetch, waits, TMA, ring); for tasks whose B rows
+        // are gathered through an index list, all 32 lanes issue the row copies.
+        const uint64_t pol_w = policy_evict_first();
+        const uint64_t pol_a = policy_evict_last();
+        int lpos = 0, lend = 0;
+        if (!x.dynamic) {
+            lpos = ra.lists.off[blockIdx.x];
+            lend = ra.lists.off[blockIdx.x + 1];
+        }
+        int qn = 0, qe = 0;
+        uint32_t st = 0;  // stages armed so far (ring position)
+        bool any_gather = false;
+        for (uint32_t it = 0;; ++it) {
+            const uint32_t slot = it % kRing;
+            if (lane == 0) {
                 TaskDesc d;
                 d.word = kExitWord;
                 d.valid = 0;
                 d.gemm = 0;
+                d.gather = 0;
                 d.start = 0;
+                d.t_fetch = d.t_ready = d.t_acc = 0;
                 int r;
                 if (!x.dynamic) {
                     r = lpos < lend ? 1 : 0;
@@ -235,68 +264,143 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     ++qn;
                     if (r == 1) d.word = w;
                 }
-                if (r < 0) break;
-                if (r == 1 && !W::derive(p, x, d)) break;
-                const uint32_t slot = it % kRing;
-                if (!mbar_wait(&sc->ring_empty[slot], ((it / kRing) & 1) ^ 1, ctl, x.timeout_ns, 901)) break;
-                if (r == 1 && d.valid && d.gemm) {
-                    const CUtensorMap* am = W::a_map(p, d.a_map);
-                    const CUtensorMap* bm = W::b_map(p, d.b_map);
-                    const uint32_t bbytes = (uint32_t)d.n * 128u;
-                    const int npre = d.nk < kStages ? d.nk : kStages;
+                bool brk = r < 0;
+                if (!brk && (x.debug & ET_DEBUG_TRACE)) d.t_fetch = globaltimer();
+                if (!brk && r == 1 && !W::derive(p, x, d)) brk = true;
+                if (!brk && !mbar_wait(&sc->ring_empty[slot], ((it / kRing) & 1) ^ 1, ctl, x.timeout_ns, 901))
+                    brk = true;
+                sc->pd = d;
+                sc->pr = r;
+                sc->pbrk = brk;
+            }
+            __syncwarp();
+            const bool brk = sc->pbrk;
+            const int r = sc->pr;
+            TaskDesc d = sc->pd;
+            __syncwarp();
+            if (brk) break;
+            if (r == 1 && d.valid && d.gemm) {
+                const CUtensorMap* am = W::a_map(p, d.a_map);
+                const uint32_t bbytes = (uint32_t)d.n * 128u;
+                if (!d.gather) {
+                    // weights (A) of the first stages before the input wait, then B by TMA
                     bool ok = true;
-                    for (int s = 0; s < npre && ok; ++s) {  // weights first
-                        const uint32_t ss = (st + s) % kStages;
-                        ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 902);
-                        if (!ok) break;
-                        mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
-                        ++armed[ss];
-                        uint8_t* dst = stages + ss * kStageBytes;
-                        const int kx = d.k0 + s * kTileK;
-                        tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
-                        tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
+                    if (lane == 0) {
+                        const CUtensorMap* bm = W::b_map(p, d.b_map);
+                        const int npre = d.nk < kStages ? d.nk : kStages;
+                        for (int s = 0; s < npre && ok; ++s) {
+                            const uint32_t ss = (st + s) % kStages;
+                            ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 902);
+                            if (!ok) break;
+                            mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
+                            ++armed[ss];
+                            uint8_t* dst = stages + ss * kStageBytes;
+                            const int kx = d.k0 + s * kTileK;
+                            tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
+                            tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
+                        }
+                        if (ok) ok = W::gemm_wait(p, x, d);  // the task's input event
+                        if (ok && (x.debug & ET_DEBUG_TRACE)) {
+                            d.start = take_ticket(ctl);
+                            d.t_ready = globaltimer();
+                        }
+                        if (ok) fence_proxy_async_global();
+                        sc->ring[slot] = d;
+                        mbar_arrive(&sc->ring_full[slot]);
+                        for (int s = 0; s < d.nk && ok; ++s) {
+                            const uint32_t ss = (st + s) % kStages;
+                            uint8_t* dst = stages + ss * kStageBytes;
+                            const int kx = d.k0 + s * kTileK;
+                            if (s >= npre) {
+                                ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 903);
+                                if (!ok) break;
+                                mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
+                                ++armed[ss];
+                                tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
+                                tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
+                            }
+                            for (int rb = 0; rb < d.n; rb += 16)
+                                tma_load_2d(dst + kAStageBytes + rb * 128, bm, &sc->full[ss], kx, d.b_row0 + rb, pol_a);
+                        }
+                        sc->pok = ok;
                     }
-                    if (ok) ok = W::gemm_wait(p, x, d);  // the task's input event
-                    if (ok && (x.debug & ET_DEBUG_TRACE)) d.start = take_ticket(ctl);
-                    if (ok) fence_proxy_async_global();
-                    sc->ring[slot] = d;
-                    mbar_arrive(&sc->ring_full[slot]);
-                    if (!ok) {
-                        // the consumers see the abort flag; stop issuing
-                        st += npre;
-                        break;
+                    __syncwarp();
+                    ok = sc->pok;
+                    __syncwarp();
+                    st += d.nk;
+                    if (!ok) break;
+                } else {
+                    // B rows gathered through an index list: every lane copies
+                    // up to 4 rows per stage with cp.async into the 128-byte
+                    // swizzled layout; lane 0 adds the weight tile by TMA.
+                    any_gather = true;
+                    const uint16_t* rows[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) rows[i] = W::gather_row(p, d, lane + 32 * i);
+                    bool ok = true;
+                    if (lane == 0) {
+                        ok = W::gemm_wait(p, x, d);
+                        if (ok && (x.debug & ET_DEBUG_TRACE)) {
+                            d.start = take_ticket(ctl);
+                            d.t_ready = globaltimer();
+                        }
+                        sc->ring[slot] = d;
+                        mbar_arrive(&sc->ring_full[slot]);
+                        sc->pok = ok;
                     }
+                    __syncwarp();
+                    ok = sc->pok;
+                    __syncwarp();
                     for (int s = 0; s < d.nk && ok; ++s) {
                         const uint32_t ss = (st + s) % kStages;
                         uint8_t* dst = stages + ss * kStageBytes;
                         const int kx = d.k0 + s * kTileK;
-                        if (s >= npre) {
-                            ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 903);
-                            if (!ok) break;
-                            mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
+                        if (lane == 0)
+                            sc->pok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 904);
+                        __syncwarp();
+                        ok = sc->pok;
+                        __syncwarp();
+                        if (!ok) break;
+                        uint8_t* bdst = dst + kAStageBytes;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = lane + 32 * i;
+                            if (rows[i]) {
+                                const uint16_t* src = rows[i] + kx;
+#pragma unroll
+                                for (int c = 0; c < 8; ++c)
+                                    cp_async16(bdst + rr * 128 + ((c ^ (rr & 7)) << 4), src + c * 8);
+                            }
+                        }
+                        cp_async_mbar_arrive(&sc->full[ss]);
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes);
                             ++armed[ss];
                             tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
                             tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
                         }
-                        for (int rb = 0; rb < d.n; rb += 16)
-                            tma_load_2d(dst + kAStageBytes + rb * 128, bm, &sc->full[ss], kx, d.b_row0 + rb, pol_a);
                     }
                     st += d.nk;
                     if (!ok) break;
-                } else {
+                }
+            } else {
+                if (lane == 0) {
                     sc->ring[slot] = d;
                     mbar_arrive(&sc->ring_full[slot]);
                 }
-                if (r == 0) break;
             }
-            // drain: every armed stage's TMA must land before the CTA exits
+            if (r == 0) break;
+        }
+        // drain: every armed stage's copies must land before the CTA exits
+        if (any_gather) cp_async_wait_all();
+        if (lane == 0)
             for (int s = 0; s < kStages; ++s)
                 if (armed[s]) {
                     uint64_t t0 = globaltimer();
                     while (!mbar_try_wait(&sc->full[s], (armed[s] - 1) & 1) && globaltimer() - t0 < 200000000ull) {
                     }
                 }
-        }
         __syncwarp();
     } else if (!skip && warp == 1) {
         if (lane == 0) {
@@ -323,6 +427,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         break;
                     }
                     tc_fence_after();
+                    fence_proxy_async_smem();  // rows copied by cp.async (generic proxy) -> tensor core
                     const uint32_t a0 = smem_u32(stages + ss * kStageBytes);
                     const uint64_t ad = sdesc_k128(a0);
                     const uint64_t bd = sdesc_k128(a0 + kAStageBytes);
@@ -369,6 +474,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 if (!sc->bcast[5]) break;
                 while (!mbar_try_wait(&sc->acc_full[buf], par)) {
                 }
+                if (x.debug & ET_DEBUG_TRACE) d.t_acc = globaltimer();
                 tc_fence_after();
                 const uint32_t taddr = sc->tmem_base + buf * kMaxN + ((uint32_t)((warp & 3) * 32) << 16);
                 if (!W::epilogue(p, x, d, taddr, &sc->acc_empty[buf])) break;

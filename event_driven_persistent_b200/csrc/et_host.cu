@@ -324,7 +324,7 @@ et_status build_mlp(et_graph* g) {
 
 // ----------------------------------------------------------------- MoE ----
 struct MoeShape {
-    int n_tt, n_kc, n_g, n_cb, f_max;
+    int n_tt, n_kc, n_tk, n_cb, f_max;
 };
 
 MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
@@ -334,8 +334,8 @@ MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
     int kc = 1;
     while (kc < 8 && m.n_tt * kc * 2 <= g->n_ctas && (p.hidden / (kc * 2)) % kTileK == 0) kc *= 2;
     m.n_kc = kc;
-    m.n_g = cdiv(T, p.gt);
     m.n_cb = cdiv(T, p.cb);
+    m.n_tk = cdiv(T, p.tkt);
     const int pairs = p.k * T;
     m.f_max = std::min(pairs, std::min(p.E, pairs) + cdiv(pairs, p.bm));
     return m;
@@ -348,7 +348,7 @@ et_status build_moe(et_graph* g) {
     if (d.n_experts <= 0) d.n_experts = 128;
     if (d.top_k <= 0) d.top_k = 8;
     if (d.fetch_batch <= 0) d.fetch_batch = 1;
-    if (d.n_experts > 128 || d.top_k > 32 || d.top_k > d.n_experts) return ET_ERR_UNSUPPORTED;
+    if (d.n_experts > 128 || d.n_experts % 8 || d.top_k > 8 || d.top_k > d.n_experts) return ET_ERR_UNSUPPORTED;
     if (d.hidden % 128 || d.inter % 64) return ET_ERR_UNSUPPORTED;
     MoeParams& p = g->moe;
     memset(&p, 0, sizeof(p));
@@ -358,7 +358,7 @@ et_status build_moe(et_graph* g) {
     p.k = d.top_k;
     p.maxT = d.max_T;
     p.tt = 128;
-    p.gt = std::max(1, 128 / p.k);
+    p.tkt = 16;
     p.bm = 128;
     p.n1_tile = 64;
     p.n_n1 = p.inter / p.n1_tile;
@@ -366,9 +366,10 @@ et_status build_moe(et_graph* g) {
     p.n_n2 = p.hidden / p.n2_tile;
     p.cb = 16;
     p.sched = d.sched;
+    p.early_max = 2 * g->n_ctas;
     p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
     const MoeShape mx = moe_shape(g, p, d.max_T);
-    if (mx.f_max > 0xFFFF || mx.n_g > 0xFFFF || p.n_n1 > 0x3FF || p.n_n2 > 0x3FF) return ET_ERR_UNSUPPORTED;
+    if (mx.f_max > 0xFFFF || mx.n_tt > 0xFFFF || p.n_n1 > 0x3FF || p.n_n2 > 0x3FF) return ET_ERR_UNSUPPORTED;
     int ev = kCtrFirstEvent;
     p.ev_tk = ev++;
     p.ev_sc = ev++;
@@ -384,15 +385,15 @@ et_status build_moe(et_graph* g) {
     ev += mx.f_max;
     p.ev_cb = ev;
     ev += mx.n_cb;
+    p.ev_gcnt = ev;
+    ev += mx.n_tt * p.E;
     g->n_ctr = ev;
-    g->qcap = mx.n_tt * 8 + mx.n_tt + 1 + mx.n_g + mx.f_max * (p.n_n1 + p.n_n2) + mx.n_cb + g->n_ctas * d.fetch_batch + 64;
+    g->qcap = mx.n_tt * 8 + mx.n_tk + mx.n_tt + 1 + mx.f_max * (p.n_n1 + p.n_n2) + mx.n_cb + g->n_ctas * d.fetch_batch + 64;
     const size_t pairs = (size_t)p.maxT * p.k;
-    ET_TRY(galloc(g, &p.lpart, (size_t)8 * p.maxT * p.E));
-    ET_TRY(galloc(g, &p.logits, (size_t)p.maxT * p.E));
+    ET_TRY(galloc(g, &p.lacc, (size_t)p.maxT * p.E));
     ET_TRY(galloc(g, &p.topk, pairs));
     ET_TRY(galloc(g, &p.topw, pairs));
-    ET_TRY(galloc(g, &p.gcnt, (size_t)mx.n_g * p.E));
-    ET_TRY(galloc(g, &p.goff, (size_t)mx.n_g * p.E));
+    ET_TRY(galloc(g, &p.goff, (size_t)mx.n_tt * p.E));
     ET_TRY(galloc(g, &p.counts, (size_t)p.E));
     ET_TRY(galloc(g, &p.indptr, (size_t)p.E + 1));
     ET_TRY(galloc(g, &p.tindptr, (size_t)p.E + 1));
@@ -400,10 +401,8 @@ et_status build_moe(et_graph* g) {
     ET_TRY(galloc(g, &p.perm, pairs));
     ET_TRY(galloc(g, &p.pos, pairs));
     ET_TRY(galloc(g, &p.scal, 8));
-    ET_TRY(galloc(g, &p.Xp, pairs * p.hidden));
     ET_TRY(galloc(g, &p.Hm, pairs * p.inter));
     ET_TRY(galloc(g, &p.Yacc, (size_t)p.maxT * p.hidden));
-    if (!make_map(&p.tm_xp, p.Xp, pairs, p.hidden, 16)) return ET_ERR_CUDA;
     if (!make_map(&p.tm_hm, p.Hm, pairs, p.inter, 16)) return ET_ERR_CUDA;
     int mb = 0;
     ET_CU(moe_setup(&mb));
@@ -414,9 +413,10 @@ et_status build_moe(et_graph* g) {
         const float c_rt = (float)p.E * p.hidden * 2 / m.n_kc / 1024.f;
         for (int t = 0; t < m.n_tt; ++t)
             for (int c = 0; c < m.n_kc; ++c) s.push_back({tw(ET_OP_MOE_ROUTER, t, c), c_rt});
-        for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_TOPK, t, 0), 8.f});
-        s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 16.f});
-        for (int q = 0; q < m.n_g; ++q) s.push_back({tw(ET_OP_MOE_GROUP, q, 0), (float)p.gt * p.k * p.hidden * 2 / 1024.f});
+        for (int j = 0; j < m.n_tk; ++j) s.push_back({tw(ET_OP_MOE_TOPK, j, 0), 8.f});
+        s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 8.f});
+        if (m.n_tt > 1)
+            for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_GROUP, t, 0), 8.f});
         for (int f = 0; f < m.f_max; ++f)
             for (int n = 0; n < p.n_n1; ++n) s.push_back({tw(ET_OP_MOE_S1, f, n), c_s1});
         for (int f = 0; f < m.f_max; ++f)
@@ -501,7 +501,8 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     }
     if (desc->kind == ET_GRAPH_MOE) {
         in.moe_tt = g->moe.tt;
-        in.moe_gt = g->moe.gt;
+        in.moe_gt = g->moe.tt;
+        in.moe_tkt = g->moe.tkt;
         in.moe_bm = g->moe.bm;
         in.moe_n1_tile = g->moe.n1_tile;
         in.moe_n2_tile = g->moe.n2_tile;
@@ -596,7 +597,7 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
     const MoeShape mt = moe_shape(g, p, T);
     p.n_kc = mb.n_kc;  // the bucket fixes the router split (static lists and dynamic alike)
     p.n_tt = mt.n_tt;
-    p.n_g = mt.n_g;
+    p.n_tk = mt.n_tk;
     p.n_cb = mt.n_cb;
     p.f_max = mb.f_max;
     ET_TRY(pre_run(g, s));
@@ -616,8 +617,10 @@ et_status et_sync_status(et_graph* g, void* stream) {
     ET_CU(cudaMemset(g->ctl, 0, sizeof(Ctl)));
     ET_CU(cudaMemset(g->ctr[0], 0, g->n_ctr * sizeof(int)));
     ET_CU(cudaMemset(g->ctr[1], 0, g->n_ctr * sizeof(int)));
-    if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc)
+    if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc) {
         ET_CU(cudaMemset(g->moe.Yacc, 0, (size_t)g->moe.maxT * g->moe.hidden * sizeof(float)));
+        ET_CU(cudaMemset(g->moe.lacc, 0, (size_t)g->moe.maxT * g->moe.E * sizeof(float)));
+    }
     ET_CU(cudaDeviceSynchronize());
     // keep the diagnostic words readable through et_get_diag
     ET_CU(cudaMemcpy(g->ctl->diag, h.diag, sizeof(h.diag), cudaMemcpyHostToDevice));

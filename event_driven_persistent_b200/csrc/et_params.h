@@ -47,16 +47,16 @@ struct MlpParams {
 };
 
 // ---------------------------------------------------------------------- MoE
-// Tasks: RT(tt, kc) router partial (tensor core), TK(tt) top-k,
-// SC scan, GR(g) grouping, S1(f, n) stage-1 tile, S2(f, n) stage-2 tile,
-// CB(b) combine.
-enum { MOE_MAP_WR = 0, MOE_MAP_W1 = 1, MOE_MAP_W2 = 2, MOE_MAP_X = 3, MOE_MAP_XP = 4, MOE_MAP_HM = 5 };
+// Tasks: RT(tt, kc) router partial (tensor core), TK(tt) top-k (and, when
+// one token tile covers T, the whole grouping), SC scan, GR(g) grouping,
+// S1(f, n) stage-1 tile (token rows gathered from X), S2(f, n) stage-2
+// tile, CB(b) combine.
+enum { MOE_MAP_WR = 0, MOE_MAP_W1 = 1, MOE_MAP_W2 = 2, MOE_MAP_X = 3, MOE_MAP_HM = 4 };
 struct MoeParams {
     CUtensorMap tm_wr;  // Wr [E, H], box 64 x 64
     CUtensorMap tm_w1;  // W1 [E*2I, H], box 64 x 64
     CUtensorMap tm_w2;  // W2 [E*H, I], box 64 x 64
     CUtensorMap tm_x;   // X  [T, H], box 64 x 16
-    CUtensorMap tm_xp;  // Xp [maxT*k, H] (workspace), box 64 x 16
     CUtensorMap tm_hm;  // Hm [maxT*k, I] (workspace), box 64 x 16
     const uint16_t* X;
     const float* bias;
@@ -68,27 +68,28 @@ struct MoeParams {
     int32_t* out_perm;
     float* out_logits;
     // workspace
-    float* lpart;       // [n_kc, maxT, E] router partial logits
-    float* logits;      // [maxT, E]
+    float* lacc;        // [maxT, E] router logits without bias: the K-chunk tasks add
+                        // their partials here (fp32 red.add); the top-k task reads and
+                        // re-zeroes it, so it is zero between runs
     int32_t* topk;      // [maxT, k]
     float* topw;        // [maxT, k]
-    int32_t* gcnt;      // [n_g, E] pairs of group tile g per expert
-    int32_t* goff;      // [n_g, E] first grouped row of tile g's pairs of expert e
+    int32_t* goff;      // [n_tt, E] first grouped row of tile g's pairs of expert e
     int32_t* counts;    // [E]
     int32_t* indptr;    // [E+1]
     int32_t* tindptr;   // [E+1] m-tile CSR
     int32_t* mt_expert; // [F_max] expert of flat m-tile f
     int32_t* perm;      // [maxT*k]
     int32_t* pos;       // [maxT*k]
-    int32_t* scal;      // [8]: 0 = total m-tiles
-    uint16_t* Xp;       // [maxT*k, H] grouped token rows
+    int32_t* scal;      // [8]: 0 = total m-tiles, 1 = stage-2 tasks were pushed early
     uint16_t* Hm;       // [maxT*k, I] stage-1 output, grouped order
     float* Yacc;        // [maxT, H] fp32 combine accumulator (kept zero between runs)
     int T, hidden, inter, E, k, maxT;
-    int tt, n_tt, n_kc, gt, n_g, bm, n1_tile, n_n1, n2_tile, n_n2, cb, n_cb;
+    int tt, n_tt, n_kc, tkt, n_tk, bm, n1_tile, n_n1, n2_tile, n_n2, cb, n_cb;
     int f_max;          // static: m-tile slots of this bucket
+    int early_max;      // dynamic: push stage-2 tasks with stage 1 when #stage-1 tasks <= this
     // events
     int ev_rt, ev_tk, ev_sc, ev_grp, ev_exp, ev_s1, ev_cb, ev_rt_all, ev_s1_all, ev_s2_all;
+    int ev_gcnt;        // counter-set block [n_tt, E]: pairs of 128-token tile g per expert
     int sched;          // et_sched
     int bad_count;
 };

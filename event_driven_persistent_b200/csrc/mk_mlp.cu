@@ -63,6 +63,7 @@ struct Mlp {
         return true;
     }
 
+    __device__ static const uint16_t* gather_row(const Params&, const TaskDesc&, int) { return nullptr; }
     __device__ static bool gemm_wait(const Params& p, Ctx& x, TaskDesc& d) {
         const int op = task_op(d.word);
         if (op == ET_OP_MLP_GATEUP)

@@ -11,13 +11,19 @@
 //     with no global barrier between the two stages.
 //   §静态调度: data-dependent edges fall back to a coarse event under
 //     static scheduling (here: every grouping task -> every stage-1 slot).
+//   §动态调度 (appendix, early push): consumers may be queued once their
+//     producers are dispatched and wait on the event before running; used
+//     for stage 2 when the stage-1 tasks do not fill the SMs, so stage-2
+//     weights stream while stage 1 computes.
 //
-// Task graph (counts in brackets; dynamic schedule):
+// Task graph (counts in brackets; dynamic schedule; tiles of 128 tokens):
 //   RT(t, c)  router partial logits of token tile t, K chunk c   -> E_rt[t] [#chunks]
-//   TK(t)     sum partials + bias, top-k, softmax, tile histograms -> E_tk [#tiles]
-//   SC        expert counts, CSR (indptr, m-tile indptr), E_exp counts -> E_sc [1]
-//   GR(g)     place the pairs of token group g, copy their rows   -> E_exp[topk[i,:]]
-//   S1(f, n)  m-tile f (expert e, up to 128 rows) x 64 intermediate cols -> E_s1[f] [#n1]
+//   TK(j)     16 tokens: sum partials + bias, top-k, softmax, tile counts -> E_tk [#top-k tasks]
+//   SC        expert counts, CSR (indptr, m-tile indptr), tile offsets -> E_sc [1]
+//             (run by the task that completes E_tk; with T <= 128 it is also the
+//             grouping task -> E_exp[topk[i,:]])
+//   GR(t)     grouped row of every pair of token tile t          -> E_exp[topk[i,:]]
+//   S1(f, n)  m-tile f (expert e, <= 128 rows gathered from X) x 64 intermediate cols -> E_s1[f] [#n1]
 //   S2(f, n)  m-tile f x 128 output cols, weighted red.add into Yacc -> E_cb[t / cb]
 //   CB(b)     Y = bf16(Yacc) for a block of cb tokens, Yacc = 0
 #include <cuda_bf16.h>
@@ -35,13 +41,35 @@ __device__ __forceinline__ void red_add(float* p, float v) {
 }
 // (value desc, index asc) total order
 __device__ __forceinline__ bool better(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
+
+// Exclusive prefix sum over the 128 exec threads (value v of thread tid);
+// returns the prefix, *total gets the sum.  `tmp` holds 4 ints of smem.
+__device__ __forceinline__ int exec_scan(int v, int tid, int* tmp, int* total) {
+    const int lane = tid & 31, w = tid >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) tmp[w] = inc;
+    exec_bar();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < kExecThreads / 32; ++i) {
+        base += i < w ? tmp[i] : 0;
+        tot += tmp[i];
+    }
+    exec_bar();
+    *total = tot;
+    return base + inc - v;
+}
 }  // namespace
 
 struct Moe {
     using Params = MoeParams;
     static constexpr bool kGemm = true;
 
-    __device__ static bool is_static(const Params& p) { return p.sched == ET_SCHED_STATIC; }
     __device__ static bool is_unfused(const Params& p) { return p.sched == ET_SCHED_UNFUSED; }
 
     __device__ static uint32_t fetch_init(const Params& p, int idx) {
@@ -73,15 +101,15 @@ struct Moe {
             d.nk = p.hidden / p.n_kc / kTileK;
             d.k0 = b * (p.hidden / p.n_kc);
         } else if (op == ET_OP_MOE_TOPK) {
-            d.valid = a < p.n_tt;
+            d.valid = a < p.n_tk;
         } else if (op == ET_OP_MOE_GROUP) {
-            d.valid = a < p.n_g;
+            d.valid = p.n_tt > 1 && a < p.n_tt;  // one tile: the scan task groups
         } else if (op == ET_OP_MOE_COMBINE) {
             d.valid = a < p.n_cb;
         } else if (op == ET_OP_MOE_S1 || op == ET_OP_MOE_S2) {
             if (!x.dynamic) {
                 // coarse: the whole grouping must be done before any stage slot
-                if (!wait_geq(x.ctr + p.ev_grp, p.n_g, x.ctl, x.timeout_ns, 200, 0)) return false;
+                if (!wait_geq(x.ctr + p.ev_grp, p.n_tt, x.ctl, x.timeout_ns, 200, 0)) return false;
                 fence_proxy_async_global();
                 if (a >= ld_volatile(p.scal)) {
                     d.valid = 0;
@@ -101,7 +129,7 @@ struct Moe {
                 d.a_map = MOE_MAP_W1;
                 d.a_row0 = e * 2 * p.inter + b * p.n1_tile;
                 d.a_row1 = e * 2 * p.inter + p.inter + b * p.n1_tile;
-                d.b_map = MOE_MAP_XP;
+                d.gather = 1;  // token rows straight from X through perm
                 d.nk = p.hidden / kTileK;
             } else {
                 d.a_map = MOE_MAP_W2;
@@ -114,13 +142,20 @@ struct Moe {
         return true;
     }
 
+    // stage-1 B row r of the task: token perm[row0 + r] / k of X
+    __device__ static const uint16_t* gather_row(const Params& p, const TaskDesc& d, int r) {
+        if (r >= d.p[2]) return nullptr;
+        return p.X + (size_t)(p.perm[d.p[1] + r] / p.k) * p.hidden;
+    }
+
     __device__ static bool gemm_wait(const Params& p, Ctx& x, TaskDesc& d) {
         const int op = task_op(d.word), f = task_a(d.word);
-        if (op != ET_OP_MOE_S2 || x.dynamic) return true;  // router: no input; S1 waited in derive
+        if (op != ET_OP_MOE_S2) return true;  // router: no input; stage 1: waited before derive
         if (is_unfused(p)) {
             const int mt_total = ld_volatile(p.scal);
             return wait_geq(x.ctr + p.ev_s1_all, mt_total * p.n_n1, x.ctl, x.timeout_ns, 201, 0);
         }
+        // static, and dynamic with stage 2 pushed early: wait for the m-tile's stage 1
         return wait_geq(x.ctr + p.ev_s1 + f, p.n_n1, x.ctl, x.timeout_ns, 202, f);
     }
 
@@ -128,7 +163,19 @@ struct Moe {
         return id == MOE_MAP_WR ? &p.tm_wr : (id == MOE_MAP_W1 ? &p.tm_w1 : &p.tm_w2);
     }
     __device__ static const CUtensorMap* b_map(const Params& p, int id) {
-        return id == MOE_MAP_X ? &p.tm_x : (id == MOE_MAP_XP ? &p.tm_xp : &p.tm_hm);
+        return id == MOE_MAP_X ? &p.tm_x : &p.tm_hm;
+    }
+
+    // Push the stage-1 tasks of m-tiles [f0, f0 + nf) and, when stage 2 goes
+    // early, their stage-2 tasks right after (exec group or single thread).
+    __device__ static int n_stage_tasks(const Params& p, int nf, bool early) {
+        return nf * (p.n_n1 + (early ? p.n_n2 : 0));
+    }
+    __device__ static uint32_t stage_task(const Params& p, int f0, int nf, int i) {
+        const int n1 = nf * p.n_n1;
+        if (i < n1) return task_word(ET_OP_MOE_S1, f0 + i / p.n_n1, i % p.n_n1);
+        i -= n1;
+        return task_word(ET_OP_MOE_S2, f0 + i / p.n_n2, i % p.n_n2);
     }
 
     __device__ static bool epilogue(const Params& p, Ctx& x, TaskDesc& d, uint32_t taddr, uint64_t* acc_empty) {
@@ -137,10 +184,10 @@ struct Moe {
         const int q = (w + kExecWarp0) & 3;
         const int r = q * 32 + lane;
         if (op == ET_OP_MOE_ROUTER) {
-            // rows = experts, columns = tokens of tile a; partial logits of K chunk b
+            // rows = experts, columns = tokens of tile a: add K chunk b's partial
+            // logits into lacc (the L2 performs the reduction over the chunks)
             const int t0 = a * p.tt;
             const int cnt = min(p.tt, p.T - t0);
-            float* lp = p.lpart + (size_t)b * p.maxT * p.E;
             for (int c0 = 0; c0 < d.n; c0 += 16) {
                 float v[16];
                 acc_load16(taddr, c0, v);
@@ -148,13 +195,16 @@ struct Moe {
                 if (r < p.E) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        if (c0 + i < cnt) lp[(size_t)(t0 + c0 + i) * p.E + r] = v[i];
+                        if (c0 + i < cnt) red_add(p.lacc + (size_t)(t0 + c0 + i) * p.E + r, v[i]);
                 }
             }
             int* ev = x.ctr + (is_unfused(p) ? p.ev_rt_all : p.ev_rt + a);
             const int tgt = is_unfused(p) ? p.n_tt * p.n_kc : p.n_kc;
             const bool fired = group_finish_notify(x, d, ev, 1, tgt);
-            if (fired && x.dynamic) group_push(x, 1, [&](int) { return task_word(ET_OP_MOE_TOPK, a, 0); });
+            if (fired && x.dynamic) {
+                const int j0 = a * (p.tt / p.tkt), nj = min(p.tt / p.tkt, p.n_tk - j0);
+                group_push(x, nj, [&](int i) { return task_word(ET_OP_MOE_TOPK, j0 + i, 0); });
+            }
         } else if (op == ET_OP_MOE_S1) {
             const int row0 = d.p[1], cnt = d.p[2];
             const bool is_up = q >= 2;
@@ -188,11 +238,19 @@ struct Moe {
             int* ev = x.ctr + (is_unfused(p) ? p.ev_s1_all : p.ev_s1 + a);
             const int tgt = is_unfused(p) ? ld_volatile(p.scal) * p.n_n1 : p.n_n1;
             const bool fired = group_finish_notify(x, d, ev, 1, tgt);
-            if (fired && x.dynamic)
+            if (fired && x.dynamic && !ld_volatile(p.scal + 1))
                 group_push(x, p.n_n2, [&](int n2) { return task_word(ET_OP_MOE_S2, a, n2); });
         } else {  // S2
             const int row0 = d.p[1], cnt = d.p[2];
             const int col = b * p.n2_tile + r;
+            int* s_tok = reinterpret_cast<int*>(x.simt);  // [128] token of each row
+            float* s_w = reinterpret_cast<float*>(s_tok + 128);
+            if (x.tid < cnt) {
+                const int pp = p.perm[row0 + x.tid];
+                s_tok[x.tid] = pp / p.k;
+                s_w[x.tid] = p.topw[pp];
+            }
+            exec_bar();
             for (int c0 = 0; c0 < d.n; c0 += 16) {
                 float v[16];
                 acc_load16(taddr, c0, v);
@@ -200,11 +258,7 @@ struct Moe {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int c = c0 + i;
-                    if (c < cnt) {
-                        const int pp = p.perm[row0 + c];
-                        const int t = pp / p.k;
-                        red_add(p.Yacc + (size_t)t * p.hidden + col, p.topw[pp] * v[i]);
-                    }
+                    if (c < cnt) red_add(p.Yacc + (size_t)s_tok[c] * p.hidden + col, s_w[c] * v[i]);
                 }
             }
             if (is_unfused(p)) {
@@ -214,17 +268,18 @@ struct Moe {
                 // one notify per run of rows in the same combine block
                 if (x.tid < cnt) {
                     const int c = x.tid;
-                    const int blk = (p.perm[row0 + c] / p.k) / p.cb;
-                    const bool head = c == 0 || (p.perm[row0 + c - 1] / p.k) / p.cb != blk;
+                    const int blk = s_tok[c] / p.cb;
+                    const bool head = c == 0 || s_tok[c - 1] / p.cb != blk;
                     if (head) {
                         int len = 1;
-                        while (c + len < cnt && (p.perm[row0 + c + len] / p.k) / p.cb == blk) ++len;
+                        while (c + len < cnt && s_tok[c + len] / p.cb == blk) ++len;
                         const int ntok = min(p.cb, p.T - blk * p.cb);
                         const int tgt = p.k * p.n_n2 * ntok;
                         if (notify(x.ctr + p.ev_cb + blk, len) == tgt && x.dynamic)
                             thread_push(x, 1, [&](int) { return task_word(ET_OP_MOE_COMBINE, blk, 0); });
                     }
                 }
+                exec_bar();  // s_tok is reused by the next task
             }
         }
         return true;
@@ -232,215 +287,335 @@ struct Moe {
 
     __device__ static bool simt(const Params& p, Ctx& x, TaskDesc& d) {
         const int op = task_op(d.word), a = task_a(d.word);
-        const int w = x.tid >> 5, lane = x.tid & 31;
-        if (op == ET_OP_MOE_TOPK) return topk_task(p, x, d, a, w, lane);
+        if (op == ET_OP_MOE_TOPK) return topk_task(p, x, d, a);
         if (op == ET_OP_MOE_SCAN) return scan_task(p, x, d);
         if (op == ET_OP_MOE_GROUP) return group_task(p, x, d, a);
         // COMBINE
         const int t0 = a * p.cb;
         const int ntok = min(p.cb, p.T - t0);
         if (is_unfused(p)) {
-            if (!group_wait(x, d, x.ctr + p.ev_grp, p.n_g, 210)) return false;
+            if (!group_wait(x, d, x.ctr + p.ev_grp, p.n_tt, 210)) return false;
             const int mt_total = ld_volatile(p.scal);
             if (!group_wait(x, d, x.ctr + p.ev_s2_all, mt_total * p.n_n2, 211)) return false;
         } else {
             if (!group_wait(x, d, x.ctr + p.ev_cb + a, p.k * p.n_n2 * ntok, 212)) return false;
         }
-        const int nv = p.hidden / 4;
-        for (int i = x.tid; i < ntok * nv; i += kExecThreads) {
-            const int t = t0 + i / nv, j = (i % nv) * 4;
-            float4* src = reinterpret_cast<float4*>(p.Yacc + (size_t)t * p.hidden + j);
-            float4 v = __ldcg(src);
-            __stcg(src, make_float4(0.f, 0.f, 0.f, 0.f));
-            ushort4 o;
-            o.x = bf16_bits(v.x);
-            o.y = bf16_bits(v.y);
-            o.z = bf16_bits(v.z);
-            o.w = bf16_bits(v.w);
-            *reinterpret_cast<ushort4*>(p.Y + (size_t)t * p.hidden + j) = o;
+        // eight float4 loads in flight per thread, then zero + convert + store
+        const int nv = p.hidden / 4, total = ntok * nv;
+        for (int base = x.tid; base < total; base += kExecThreads * 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * kExecThreads;
+                if (i < total) v[u] = __ldcg(reinterpret_cast<const float4*>(p.Yacc + (size_t)(t0 + i / nv) * p.hidden) + i % nv);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * kExecThreads;
+                if (i < total) {
+                    const size_t off = (size_t)(t0 + i / nv) * p.hidden + (i % nv) * 4;
+                    __stcg(reinterpret_cast<float4*>(p.Yacc + off), make_float4(0.f, 0.f, 0.f, 0.f));
+                    ushort4 o;
+                    o.x = bf16_bits(v[u].x);
+                    o.y = bf16_bits(v[u].y);
+                    o.z = bf16_bits(v[u].z);
+                    o.w = bf16_bits(v[u].w);
+                    *reinterpret_cast<ushort4*>(p.Y + off) = o;
+                }
+            }
         }
         group_finish_notify(x, d, nullptr, 0, 0);
         return true;
     }
 
-    // TK(tt): logits = sum of the K-chunk partials (chunk order) + bias; top-k
-    // by (value desc, index asc); softmax of the selected logits; per-group
-    // tile histograms of the routed experts.
-    __device__ static bool topk_task(const Params& p, Ctx& x, TaskDesc& d, int tt, int w, int lane) {
-        const int* ev = x.ctr + (is_unfused(p) ? p.ev_rt_all : p.ev_rt + tt);
-        const int tgt = is_unfused(p) ? p.n_tt * p.n_kc : p.n_kc;
+    // Exec-group scratch of the routing tasks (x.epi and x.simt, which are
+    // contiguous and free while the exec group runs a CUDA-core task):
+    //   L     [16][132] fp32  logits of 16 tokens; expert e of token t at
+    //                         t*132 + (e/32)*33 + e%32 (bank-conflict free);
+    //                         reused for the per-quarter top-8 lists
+    //   tk    [128 * k] int   selected experts of a 128-token tile, pair order
+    //   emask [128][4]  u32   per expert: bit t = token t of the tile picked it
+    //   base  [128] int       first grouped row per expert (placement)
+    //   hist  [128] int       pairs per expert of a top-k task
+    //   misc  [8] int
+    struct RouteSmem {
+        float* L;
+        int* tk;
+        uint32_t* emask;
+        int* base;
+        int* hist;
+        int* misc;
+    };
+    __device__ static RouteSmem route_smem(Ctx& x) {
+        RouteSmem s;
+        s.L = x.epi;
+        s.tk = reinterpret_cast<int*>(x.epi + 16 * 132);
+        s.emask = reinterpret_cast<uint32_t*>(s.tk + 128 * 8);
+        s.base = reinterpret_cast<int*>(s.emask + 128 * 4);
+        s.hist = s.base + 128;
+        s.misc = s.hist + 128;
+        return s;
+    }
+
+    // Insert candidate (v, i) into a descending top-8 list (order: logit
+    // desc, index asc).  The list keeps the 8 best candidates seen so far.
+    __device__ static void ins8(float (&tv)[8], int (&ti)[8], float v, int i) {
+        if (!better(v, i, tv[7], ti[7])) return;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const bool c = better(v, i, tv[s], ti[s]);
+            const float ov = tv[s];
+            const int oi = ti[s];
+            tv[s] = c ? v : ov;
+            ti[s] = c ? i : oi;
+            v = c ? ov : v;
+            i = c ? oi : i;
+        }
+    }
+
+    // TK(j): tokens [16j, 16j+16).  logits = (sum of the K-chunk partials) +
+    // bias; top-k by (logit desc, index asc); softmax of the selected logits;
+    // pair counts per expert of the token's 128-token tile.  Thread (g, q)
+    // takes token g and experts 32q .. 32q+31, keeps a top-8 list of its
+    // quarter, and the q = 0 thread merges the four lists.  Loops stay
+    // rolled: this code runs once per task and must stay small in the
+    // instruction cache.  The task that completes E_tk runs the scan itself
+    // (dynamic schedule), with no trip through the queue.
+    __device__ static bool topk_task(const Params& p, Ctx& x, TaskDesc& d, int j) {
+        const int tile = j * p.tkt / p.tt;
+        const int* ev = x.ctr + (is_unfused(p) ? p.ev_rt_all : p.ev_rt + tile);
+        const int tgt = (is_unfused(p) ? p.n_tt * p.n_kc : p.n_kc) + p.bad_count;
         if (!group_wait(x, d, ev, tgt, 220)) return false;
-        const int t0 = tt * p.tt;
-        const int ntok = min(p.tt, p.T - t0);
-        const int g0 = t0 / p.gt;
-        const int ng = (ntok + p.gt - 1) / p.gt;
-        int* hist = reinterpret_cast<int*>(x.simt);  // [ng][E]
-        for (int i = x.tid; i < ng * p.E; i += kExecThreads) hist[i] = 0;
+        RouteSmem sm = route_smem(x);
+        const int tg = x.tid >> 2, q = x.tid & 3;
+        const int t0 = j * p.tkt;
+        const int ntok = min(p.tkt, p.T - t0);
+        const bool valid = tg < ntok;
+        const int t = t0 + tg;
+        if (x.tid < 128) sm.hist[x.tid] = 0;
+        float* row = sm.L + tg * 132 + q * 33;
+        // logits of this thread's token quarter (and re-zero the accumulator)
+#pragma unroll 1
+        for (int sub = 0; sub < 4; ++sub) {
+            const int e0 = q * 32 + sub * 8;
+            if (!valid || e0 >= p.E) break;
+            float4* src = reinterpret_cast<float4*>(p.lacc + (size_t)t * p.E + e0);
+            const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
+            const float4 b0 = *reinterpret_cast<const float4*>(p.bias + e0);
+            const float4 b1 = *reinterpret_cast<const float4*>(p.bias + e0 + 4);
+            __stcg(src, make_float4(0.f, 0.f, 0.f, 0.f));
+            __stcg(src + 1, make_float4(0.f, 0.f, 0.f, 0.f));
+            const float4 l0 = make_float4(a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w);
+            const float4 l1 = make_float4(a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w);
+            float* r8 = row + sub * 8;
+            r8[0] = l0.x;
+            r8[1] = l0.y;
+            r8[2] = l0.z;
+            r8[3] = l0.w;
+            r8[4] = l1.x;
+            r8[5] = l1.y;
+            r8[6] = l1.z;
+            r8[7] = l1.w;
+            if (p.out_logits) {
+                float4* o = reinterpret_cast<float4*>(p.out_logits + (size_t)t * p.E + e0);
+                o[0] = l0;
+                o[1] = l1;
+            }
+        }
+        float tv[8];
+        int ti[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            tv[s] = -INFINITY;
+            ti[s] = 0x7fffffff;
+        }
+        const int ne = valid ? max(0, min(32, p.E - q * 32)) : 0;
+#pragma unroll 1
+        for (int i = 0; i < ne; ++i) ins8(tv, ti, row[i], q * 32 + i);
+        exec_bar();  // every thread is done with L: reuse it for the lists
+        float* lst = sm.L + x.tid * 16;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            lst[s] = tv[s];
+            reinterpret_cast<int*>(lst)[8 + s] = ti[s];
+        }
         exec_bar();
-        for (int lt = w; lt < ntok; lt += kExecThreads / 32) {
-            const int t = t0 + lt;
-            float v[4];
-            bool taken[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e = lane + 32 * i;
-                taken[i] = e >= p.E;
-                float s = -INFINITY;
-                if (e < p.E) {
-                    s = 0.f;
-                    for (int c = 0; c < p.n_kc; ++c) s += p.lpart[((size_t)c * p.maxT + t) * p.E + e];
-                    s += p.bias[e];
-                    p.logits[(size_t)t * p.E + e] = s;
-                    if (p.out_logits) p.out_logits[(size_t)t * p.E + e] = s;
-                }
-                v[i] = s;
+        if (q == 0 && valid) {
+#pragma unroll 1
+            for (int qq = 1; qq < 4; ++qq) {
+                const float* o = sm.L + (tg * 4 + qq) * 16;
+#pragma unroll 1
+                for (int s = 0; s < 8; ++s) ins8(tv, ti, o[s], reinterpret_cast<const int*>(o)[8 + s]);
             }
-            int seli = 0;
-            float m0 = 0.f;
-            float z = 0.f;
-            float my_ex = 0.f;
-            for (int s = 0; s < p.k; ++s) {
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
+            float ex[8], z = 0.f;
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (!taken[i] && better(v[i], lane + 32 * i, bv, bi)) {
-                        bv = v[i];
-                        bi = lane + 32 * i;
-                    }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                    if (better(ov, oi, bv, bi)) {
-                        bv = ov;
-                        bi = oi;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (bi == lane + 32 * i) taken[i] = true;
-                if (s == 0) m0 = bv;
-                const float ex = expf(bv - m0);
-                z += ex;
-                if (lane == s) {
-                    seli = bi;
-                    my_ex = ex;
-                }
+            for (int s = 0; s < 8; ++s) {
+                ex[s] = s < p.k ? expf(tv[s] - tv[0]) : 0.f;
+                z += ex[s];
             }
-            if (lane < p.k) {
-                const float wt = my_ex / z;
-                p.topk[(size_t)t * p.k + lane] = seli;
-                p.topw[(size_t)t * p.k + lane] = wt;
-                if (p.out_topk) p.out_topk[(size_t)t * p.k + lane] = seli;
-                if (p.out_w) p.out_w[(size_t)t * p.k + lane] = wt;
-                atomicAdd(&hist[(lt / p.gt) * p.E + seli], 1);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                if (s >= p.k) break;
+                const size_t pi = (size_t)t * p.k + s;
+                const float wt = ex[s] / z;
+                p.topk[pi] = ti[s];
+                p.topw[pi] = wt;
+                if (p.out_topk) p.out_topk[pi] = ti[s];
+                if (p.out_w) p.out_w[pi] = wt;
+                atomicAdd(&sm.hist[ti[s]], 1);
             }
         }
         exec_bar();
-        for (int i = x.tid; i < ng * p.E; i += kExecThreads) p.gcnt[(size_t)g0 * p.E + i] = hist[i];
-        const bool fired = group_finish_notify(x, d, x.ctr + p.ev_tk, 1, p.n_tt);
-        if (fired && x.dynamic) group_push(x, 1, [&](int) { return task_word(ET_OP_MOE_SCAN, 0, 0); });
+        if (x.tid < p.E && sm.hist[x.tid] > 0) atomicAdd(x.ctr + p.ev_gcnt + tile * p.E + x.tid, sm.hist[x.tid]);
+        const bool fired = group_finish_notify(x, d, x.ctr + p.ev_tk, 1, p.n_tk);
+        if (fired && x.dynamic) {
+            // this task completed E_tk: run the scan task here
+            TaskDesc sd = d;
+            sd.word = task_word(ET_OP_MOE_SCAN, 0, 0);
+            sd.t_fetch = sd.t_acc = 0;
+            if (x.debug & ET_DEBUG_TRACE) sd.t_fetch = globaltimer();
+            return scan_task(p, x, sd);
+        }
         return true;
     }
 
-    // SC: counts, pair CSR (indptr), per-group offsets, m-tile CSR and the
-    // m-tile -> expert map; the data-dependent counts of the expert events.
-    __device__ static bool scan_task(const Params& p, Ctx& x, TaskDesc& d) {
-        if (!group_wait(x, d, x.ctr + p.ev_tk, p.n_tt + p.bad_count, 230)) return false;
-        int* s_cnt = reinterpret_cast<int*>(x.simt);  // [E]
-        int* s_ptr = s_cnt + 128;                      // [E+1]
-        int* s_tptr = s_ptr + 132;                     // [E+1]
+    __device__ static int tile_count(const RouteSmem& sm, int e) {
+        return __popc(sm.emask[e * 4]) + __popc(sm.emask[e * 4 + 1]) + __popc(sm.emask[e * 4 + 2]) +
+               __popc(sm.emask[e * 4 + 3]);
+    }
+
+    // Expert counts -> CSR of pairs (indptr), CSR of m-tiles (tindptr), the
+    // m-tile -> expert map, the run's task total and the early-push choice.
+    // Exec group; thread e owns expert e.  Returns the number of m-tiles.
+    __device__ static int build_csr(const Params& p, Ctx& x, RouteSmem& sm, int cnt, int* ex_out) {
         const int e = x.tid;
-        int cnt = 0;
-        if (e < p.E)
-            for (int g = 0; g < p.n_g; ++g) cnt += p.gcnt[(size_t)g * p.E + e];
-        if (e < p.E) s_cnt[e] = cnt;
-        exec_bar();
+        int tot, ttot;
+        const int ex = exec_scan(cnt, x.tid, sm.misc, &tot);
+        const int nt = (cnt + p.bm - 1) / p.bm;
+        const int tex = exec_scan(nt, x.tid, sm.misc, &ttot);
+        if (e < p.E) {
+            p.counts[e] = cnt;
+            p.indptr[e] = ex;
+            p.tindptr[e] = tex;
+            if (p.out_indptr) p.out_indptr[e] = ex;
+            for (int f = tex; f < tex + nt; ++f) p.mt_expert[f] = e;
+        }
         if (x.tid == 0) {
-            int acc = 0, tacc = 0;
-            for (int i = 0; i < p.E; ++i) {
-                s_ptr[i] = acc;
-                s_tptr[i] = tacc;
-                acc += s_cnt[i];
-                tacc += (s_cnt[i] + p.bm - 1) / p.bm;
-            }
-            s_ptr[p.E] = acc;
-            s_tptr[p.E] = tacc;
-            p.indptr[p.E] = acc;
-            p.tindptr[p.E] = tacc;
-            if (p.out_indptr) p.out_indptr[p.E] = acc;
-            p.scal[0] = tacc;
+            p.indptr[p.E] = tot;
+            p.tindptr[p.E] = ttot;
+            if (p.out_indptr) p.out_indptr[p.E] = tot;
+            p.scal[0] = ttot;
+            const bool early = x.dynamic && n_stage_tasks(p, ttot, false) <= p.early_max;
+            p.scal[1] = early;
             if (x.dynamic) {
-                const int total = p.n_tt * p.n_kc + p.n_tt + 1 + p.n_g + tacc * (p.n_n1 + p.n_n2) + p.n_cb;
+                // queued tasks of the run: router, top-k, group (several tiles),
+                // stage 1 and 2, combine (the scan runs inline)
+                const int total = p.n_tt * p.n_kc + p.n_tk + (p.n_tt > 1 ? p.n_tt : 0) +
+                                  ttot * (p.n_n1 + p.n_n2) + p.n_cb;
                 __threadfence();
                 atomicExch(x.ctr + kCtrTotal, total + 1);
             }
+            sm.misc[4] = ttot;
+            sm.misc[5] = early;
         }
         exec_bar();
-        if (e < p.E) {
-            p.counts[e] = cnt;
-            p.indptr[e] = s_ptr[e];
-            p.tindptr[e] = s_tptr[e];
-            if (p.out_indptr) p.out_indptr[e] = s_ptr[e];
-            for (int f = s_tptr[e]; f < s_tptr[e + 1]; ++f) p.mt_expert[f] = e;
-            int run = s_ptr[e];
-            for (int g = 0; g < p.n_g; ++g) {
-                p.goff[(size_t)g * p.E + e] = run;
-                run += p.gcnt[(size_t)g * p.E + e];
-            }
-        }
-        const bool fired = group_finish_notify(x, d, x.ctr + p.ev_sc, 1, 1);
-        if (fired && x.dynamic) group_push(x, p.n_g, [&](int g) { return task_word(ET_OP_MOE_GROUP, g, 0); });
-        return true;
+        *ex_out = ex;
+        return sm.misc[4];
     }
 
-    // GR(g): grouped row of each (token, slot) pair of group g (stable:
-    // ascending token inside an expert), perm/pos, and the token rows copied
-    // to their grouped positions; then the expert events.
-    __device__ static bool group_task(const Params& p, Ctx& x, TaskDesc& d, int g) {
-        if (!group_wait(x, d, x.ctr + p.ev_sc, 1, 240)) return false;
-        const int t0 = g * p.gt;
-        const int ntok = min(p.gt, p.T - t0);
-        const int np = ntok * p.k;
-        int* s_e = reinterpret_cast<int*>(x.simt);  // [128] expert of pair i
-        int* s_row = s_e + 128;                      // [128] grouped row of pair i
-        if (x.tid < np) s_e[x.tid] = p.topk[(size_t)t0 * p.k + x.tid];
+    // Load a 128-token tile's picks (pair order) into sm.tk and build the
+    // per-expert token masks.  Exec group.
+    __device__ static void load_tile_picks(const Params& p, Ctx& x, RouteSmem& sm, int t0, int ntok) {
+        for (int i = x.tid; i < 128 * 4; i += kExecThreads) sm.emask[i] = 0;
         exec_bar();
-        if (x.tid < np) {
-            const int i = x.tid, e = s_e[i];
-            int rank = 0;
-            for (int j = 0; j < i; ++j) rank += s_e[j] == e;
-            const int row = p.goff[(size_t)g * p.E + e] + rank;
-            s_row[i] = row;
-            const int pair = t0 * p.k + i;
+        for (int i = x.tid; i < ntok * p.k; i += kExecThreads) {
+            const int ee = __ldcg(p.topk + (size_t)t0 * p.k + i);
+            const int tl = i / p.k;
+            sm.tk[i] = ee;
+            atomicOr(&sm.emask[ee * 4 + (tl >> 5)], 1u << (tl & 31));
+        }
+        exec_bar();
+    }
+
+    // Stable placement of one tile's pairs: thread t owns token t of the tile;
+    // the grouped row of (t, s) with expert e is base[e] + the number of the
+    // tile's tokens before t that picked e (a popcount of e's token mask).
+    __device__ static void place_pairs(const Params& p, Ctx& x, RouteSmem& sm, int t0, int ntok) {
+        const int t = x.tid;
+        if (t >= ntok) return;
+        const int wd = t >> 5;
+        const uint32_t below = (1u << (t & 31)) - 1u;
+        for (int s = 0; s < p.k; ++s) {
+            const int e = sm.tk[t * p.k + s];
+            const uint32_t* m = sm.emask + e * 4;
+            int rank = __popc(m[wd] & below);
+            for (int j = 0; j < wd; ++j) rank += __popc(m[j]);
+            const int pair = (t0 + t) * p.k + s, row = sm.base[e] + rank;
             p.perm[row] = pair;
             p.pos[pair] = row;
             if (p.out_perm) p.out_perm[row] = pair;
         }
-        exec_bar();
-        const int nv = p.hidden / 8;  // uint4 per row
-        for (int i = x.tid; i < np * nv; i += kExecThreads) {
-            const int pi = i / nv, j = i % nv;
-            const int t = t0 + pi / p.k;
-            const uint4 v = *reinterpret_cast<const uint4*>(p.X + (size_t)t * p.hidden + j * 8);
-            *reinterpret_cast<uint4*>(p.Xp + (size_t)s_row[pi] * p.hidden + j * 8) = v;
+    }
+
+    // SC: expert counts from the per-tile pair counts, the CSRs and each
+    // tile's first grouped row per expert.  With one 128-token tile it is
+    // also the grouping task (placement, then the stage tasks / E_grp).
+    __device__ static bool scan_task(const Params& p, Ctx& x, TaskDesc& d) {
+        if (!group_wait(x, d, x.ctr + p.ev_tk, p.n_tk, 230)) return false;
+        RouteSmem sm = route_smem(x);
+        const int e = x.tid;
+        int cnt = 0;
+        if (e < p.E)
+            for (int g = 0; g < p.n_tt; ++g) cnt += ld_relaxed(x.ctr + p.ev_gcnt + g * p.E + e);
+        int ex;
+        const int ttot = build_csr(p, x, sm, cnt, &ex);
+        if (p.n_tt == 1) {
+            if (e < p.E) sm.base[e] = ex;
+            load_tile_picks(p, x, sm, 0, p.T);
+            place_pairs(p, x, sm, 0, p.T);
+            if (!x.dynamic) {
+                group_finish_notify(x, d, x.ctr + p.ev_grp, 1, p.n_tt);
+                return true;
+            }
+            group_finish_notify(x, d, nullptr, 0, 0);
+            const bool early = sm.misc[5] != 0;
+            group_push(x, n_stage_tasks(p, ttot, early), [&](int i) { return stage_task(p, 0, ttot, i); });
+            return true;
         }
-        fence_proxy_async_global();  // Xp is read by TMA in stage 1
+        if (e < p.E) {
+            int run = ex;
+            for (int g = 0; g < p.n_tt; ++g) {
+                p.goff[(size_t)g * p.E + e] = run;
+                run += ld_relaxed(x.ctr + p.ev_gcnt + g * p.E + e);
+            }
+        }
+        const bool fired = group_finish_notify(x, d, x.ctr + p.ev_sc, 1, 1);
+        if (fired && x.dynamic) group_push(x, p.n_tt, [&](int g) { return task_word(ET_OP_MOE_GROUP, g, 0); });
+        return true;
+    }
+
+    // GR(g) (several tiles): grouped rows of 128-token tile g's pairs, then
+    // the expert events (grouping_task[g] -> E[topk[i,:]], one add of the
+    // tile's pair count per expert it touches).
+    __device__ static bool group_task(const Params& p, Ctx& x, TaskDesc& d, int g) {
+        if (!group_wait(x, d, x.ctr + p.ev_sc, 1, 240)) return false;
+        RouteSmem sm = route_smem(x);
+        const int t0 = g * p.tt;
+        const int ntok = min(p.tt, p.T - t0);
+        const int e = x.tid;
+        if (e < p.E) sm.base[e] = __ldcg(p.goff + (size_t)g * p.E + e);
+        load_tile_picks(p, x, sm, t0, ntok);
+        place_pairs(p, x, sm, t0, ntok);
+        const int cnt = e < p.E ? tile_count(sm, e) : 0;
         if (!x.dynamic) {
-            group_finish_notify(x, d, x.ctr + p.ev_grp, 1, p.n_g);
+            group_finish_notify(x, d, x.ctr + p.ev_grp, 1, p.n_tt);
             return true;
         }
         group_finish_notify(x, d, nullptr, 0, 0);
-        // grouping_task[g] -> E[topk[i,:]] for the tokens i of group g: one add
-        // of the group's pair count per expert it touches
-        if (x.tid < p.E) {
-            const int e = x.tid;
-            const int c = p.gcnt[(size_t)g * p.E + e];
-            if (c > 0 && notify(x.ctr + p.ev_exp + e, c) == p.counts[e]) {
-                const int f0 = p.tindptr[e], nf = p.tindptr[e + 1] - f0;
-                thread_push(x, nf * p.n_n1, [&](int i) { return task_word(ET_OP_MOE_S1, f0 + i / p.n_n1, i % p.n_n1); });
-            }
+        if (cnt > 0 && notify(x.ctr + p.ev_exp + e, cnt) == __ldcg(p.counts + e)) {
+            const int f0 = __ldcg(p.tindptr + e), nf = __ldcg(p.tindptr + e + 1) - f0;
+            const bool early = ld_volatile(p.scal + 1) != 0;
+            thread_push(x, n_stage_tasks(p, nf, early), [&](int i) { return stage_task(p, f0, nf, i); });
         }
         return true;
     }

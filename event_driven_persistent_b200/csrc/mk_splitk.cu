@@ -26,6 +26,7 @@ struct SplitK {
         d.gemm = 0;
         return true;
     }
+    __device__ static const uint16_t* gather_row(const Params&, const TaskDesc&, int) { return nullptr; }
     __device__ static bool gemm_wait(const Params&, Ctx&, TaskDesc&) { return true; }
     __device__ static const CUtensorMap* a_map(const Params&, int) { return nullptr; }
     __device__ static const CUtensorMap* b_map(const Params&, int) { return nullptr; }

@@ -98,7 +98,8 @@ typedef struct {
     int mlp_down_tile;   /* output columns per down task */
     int mlp_kchunk;      /* K (intermediate) columns per down task */
     int moe_tt;          /* tokens per router/top-k tile */
-    int moe_gt;          /* tokens per grouping task */
+    int moe_gt;          /* tokens per grouping task (= moe_tt) */
+    int moe_tkt;         /* tokens per top-k task */
     int moe_bm;          /* rows (token, slot pairs) per expert m-tile */
     int moe_n1_tile;     /* intermediate columns per stage-1 task */
     int moe_n2_tile;     /* output columns per stage-2 task */
@@ -109,8 +110,13 @@ typedef struct {
 /* Trace record (ET_DEBUG_TRACE): one per executed task. */
 typedef struct {
     int32_t op, a, b, sm;
-    uint32_t start; /* ticket taken after the task's wait succeeded */
-    uint32_t end;   /* ticket taken after its outputs were written, before its notify */
+    uint32_t start;   /* ticket taken after the task's wait succeeded */
+    uint32_t end;     /* ticket taken after its outputs were written, before its notify */
+    uint64_t t_fetch; /* %globaltimer (ns): task taken from the static list / ready queue */
+    uint64_t t_ready; /* %globaltimer: input event complete */
+    uint64_t t_acc;   /* %globaltimer: tensor-core accumulator ready (GEMM tasks), end of the
+                         first phase (top-k task), else 0 */
+    uint64_t t_end;   /* %globaltimer: outputs written */
 } et_trace_record;
 
 /* trace op codes */

@@ -120,14 +120,17 @@ def mlp_graph(B, hidden, inter, gu_tile, down_tile, kchunk, sched):
     return g.finish()
 
 
-def moe_graph(topk, E, tt, n_kc, gt, bm, n_n1, n_n2, cb, sched):
+def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
     """MoE layer, expanded with the runtime routing `topk` [T, k]:
-      router (t, c)   --"tc->t"-->           E_rt[t]         (count = #K chunks)
-      E_rt[t]         --"t->t"-->            topk t
-      topk t          --"t->"-->             E_tk            (count = #token tiles)
+      router (t, c)   --"tc->t"-->           E_rt[t]         (count = #K chunks; tt tokens)
+      E_rt[t]         -->                    topk j for the tkt-token tiles j inside tile t
+      topk j          --"j->"-->             E_tk            (count = #top-k tasks)
       E_tk            -->                    scan
+      one router tile (T <= tt): the scan is the grouping task:
+      scan            --> E_exp[topk[i,:]] for every token i
+      several router tiles:
       scan            -->                    E_sc            (count 1)
-      E_sc            --"->g"-->             group g
+      E_sc            --"->g"-->             group g         (gt tokens)
       group g         --> E_exp[topk[i,:]] for every token i of group g
                                                (count of E_exp[e] = #pairs routed to e)
       E_exp[e]        --> stage1 tasks[task_indptr[e] : task_indptr[e+1]] x n1 tiles
@@ -135,13 +138,14 @@ def moe_graph(topk, E, tt, n_kc, gt, bm, n_n1, n_n2, cb, sched):
       E_s1[f]         --"f->fn"-->           stage2 (f, n)
       stage2 (f, n)   --> E_cb[i // cb] for every row (token i) of m-tile f
       E_cb[b]         -->                    combine b
-    Static scheduling replaces group -> E_exp -> stage1 by one coarse event
-    (every group task -> every stage1 task).  Unfused replaces every
+    Static scheduling replaces grouping -> E_exp -> stage1 by one coarse event
+    (every grouping task -> every stage1 task).  Unfused replaces every
     operator boundary by one event."""
     topk = np.asarray(topk)
     T, k = topk.shape
     g = Graph()
     n_tt = _cdiv(T, tt)
+    n_tk = _cdiv(T, tkt)
     n_g = _cdiv(T, gt)
     n_cb = _cdiv(T, cb)
     unf = sched == "unfused"
@@ -161,25 +165,33 @@ def moe_graph(topk, E, tt, n_kc, gt, bm, n_n1, n_n2, cb, sched):
             task = (OP_MOE_ROUTER, t, c)
             g.add_task(task)
             g.produce(task, ("E_rt_all",) if unf else ("E_rt", t))
-    for t in range(n_tt):
-        task = (OP_MOE_TOPK, t, 0)
+    for j in range(n_tk):
+        task = (OP_MOE_TOPK, j, 0)
         g.add_task(task)
-        g.consume(task, ("E_rt_all",) if unf else ("E_rt", t))
+        g.consume(task, ("E_rt_all",) if unf else ("E_rt", (j * tkt) // tt))
         g.produce(task, ("E_tk",))
     scan = (OP_MOE_SCAN, 0, 0)
     g.add_task(scan)
     g.consume(scan, ("E_tk",))
-    g.produce(scan, ("E_sc",))
-    for q in range(n_g):
-        task = (OP_MOE_GROUP, q, 0)
-        g.add_task(task)
-        g.consume(task, ("E_sc",))
+    if n_tt == 1:
         if unf or static:
-            g.produce(task, ("E_grp",))
+            g.produce(scan, ("E_grp",))
         else:
-            for i in range(q * gt, min(T, (q + 1) * gt)):
+            for i in range(T):
                 for s in range(k):
-                    g.produce(task, ("E_exp", int(topk[i, s])))
+                    g.produce(scan, ("E_exp", int(topk[i, s])))
+    else:
+        g.produce(scan, ("E_sc",))
+        for q in range(n_g):
+            task = (OP_MOE_GROUP, q, 0)
+            g.add_task(task)
+            g.consume(task, ("E_sc",))
+            if unf or static:
+                g.produce(task, ("E_grp",))
+            else:
+                for i in range(q * gt, min(T, (q + 1) * gt)):
+                    for s in range(k):
+                        g.produce(task, ("E_exp", int(topk[i, s])))
     for f, (e, m, rows) in enumerate(mtiles):
         for n in range(n_n1):
             task = (OP_MOE_S1, f, n)

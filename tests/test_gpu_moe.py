@@ -125,7 +125,7 @@ def test_moe_dependency_order(small_inputs, sched, T):
         # the router split of a run is fixed by its size bucket; read it from the trace
         rt = [r for r in et.et_get_trace(g) if r[0] == dag.OP_MOE_ROUTER]
         n_kc = max(r[2] for r in rt) + 1
-        graph, _ = dag.moe_graph(out["topk"], 16, info["moe_tt"], n_kc, info["moe_gt"], info["moe_bm"],
+        graph, _ = dag.moe_graph(out["topk"], 16, info["moe_tt"], n_kc, info["moe_tkt"], info["moe_gt"], info["moe_bm"],
                                  128 // info["moe_n1_tile"], 256 // info["moe_n2_tile"], info["moe_cb"], sched)
         errs = dag.check_trace(graph, et.et_get_trace(g))
         assert errs == [], errs[:5]
