@@ -43,8 +43,8 @@ struct TaskDesc {
 };
 
 struct SmemCtl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kSlots];
+    uint64_t empty[kSlots];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t ring_full[kRing];
@@ -57,6 +57,8 @@ struct SmemCtl {
     TaskDesc ring[kRing];
     TaskDesc pd;  // warp 0: the task lane 0 fetched, for the other lanes
     int pr, pbrk, pok;
+    uint32_t pslot, poff;
+    uint32_t r_off[kSlots], r_end[kSlots];  // arena range of the last kSlots stages
 };
 
 // Everything a role needs besides the workload parameters.
@@ -69,7 +71,7 @@ struct Ctx {
     int debug;           // ET_DEBUG_* bits
     TraceRec* trace;
     int trace_cap;
-    uint8_t* stages;     // kStages x kStageBytes, 1024-aligned
+    uint8_t* arena;      // pipeline stages, 1024-aligned
     float* epi;          // gate/up exchange staging
     uint8_t* simt;       // CUDA-core task scratch
     SmemCtl* sc;
@@ -147,6 +149,22 @@ __device__ __forceinline__ bool group_wait(Ctx& x, TaskDesc& d, const int* ctr, 
     return ok;
 }
 
+// Bytes of one pipeline stage: the weight tile, then N activation rows
+// (1 KB multiples keep every tile on the 128-byte swizzle atom).
+__device__ __forceinline__ uint32_t stage_bytes(int n) { return kAStageBytes + ((n * 128 + 1023) & ~1023); }
+
+// Circular allocation of stages in the arena; the producer and the MMA
+// issuer replay the same sequence, so both know every stage's address.
+struct StageAlloc {
+    uint32_t head = 0;
+    __device__ __forceinline__ uint32_t next(uint32_t size) {
+        if (head + size > (uint32_t)kArenaBytes) head = 0;
+        const uint32_t o = head;
+        head += size;
+        return o;
+    }
+};
+
 // Megakernel body.  W supplies the task semantics:
 //   W::fetch_init(p, idx)              initial dynamic task word for slot idx
 //   W::derive(p, x, word, d)           fill a TaskDesc (warp 0; may wait in
@@ -160,10 +178,12 @@ template <class W>
 __device__ __forceinline__ void megakernel_body(const typename W::Params& p, const RunArgs& ra) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* stages = base;
-    float* epi = reinterpret_cast<float*>(base + kStages * kStageBytes);
-    uint8_t* simt = base + kStages * kStageBytes + kEpiBytes;
-    SmemCtl* sc = reinterpret_cast<SmemCtl*>(simt + kSimtBytes);
+    uint8_t* arena = base;
+    uint8_t* scratch = arena + kArenaBytes;
+    float* epi = reinterpret_cast<float*>(scratch);
+    uint8_t* simt = scratch + kEpiBytes;
+    SmemCtl* sc = reinterpret_cast<SmemCtl*>(scratch + kScratchBytes);
+    static_assert(sizeof(SmemCtl) <= kCtlBytes, "control block does not fit");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Ctl* ctl = ra.ctl;
@@ -175,7 +195,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     }
     if (threadIdx.x == 0) {
         sc->start_status = ld_volatile(&ctl->status);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kSlots; ++s) {
             mbar_init(&sc->full[s], 1);
             mbar_init(&sc->empty[s], 1);
         }
@@ -216,15 +236,12 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     x.debug = ra.debug;
     x.trace = ra.trace;
     x.trace_cap = ra.trace_cap;
-    x.stages = stages;
+    x.arena = arena;
     x.epi = epi;
     x.simt = simt;
     x.sc = sc;
     x.tid = threadIdx.x - kExecWarp0 * 32;
 
-    uint32_t armed[kStages];
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) armed[s] = 0;
 
     if (!skip && warp == 0) {
         // ---------------------------------------------------- task source + loads
@@ -238,8 +255,45 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             lend = ra.lists.off[blockIdx.x + 1];
         }
         int qn = 0, qe = 0;
-        uint32_t st = 0;  // stages armed so far (ring position)
         bool any_gather = false;
+        // lane 0: stage bookkeeping (global stage count, arena ranges of the
+        // last kSlots stages, arms per slot for the exit drain)
+        uint32_t nst = 0, tail = 0;  // stages reserved so far; oldest stage not yet seen consumed
+        StageAlloc alloc;
+        uint32_t armed[kSlots];
+        for (int s2 = 0; s2 < kSlots; ++s2) armed[s2] = 0;
+        // Reserve the next stage.  In-flight stages form one circular run of
+        // the arena from the tail stage to the allocation head, so the new
+        // stage can only collide with the oldest ones: consume (wait for)
+        // tail stages until its slot and its bytes are free.  O(1) amortised.
+        auto reserve = [&](int n, uint32_t* slot_out, uint32_t* off_out) -> bool {
+            const uint32_t size = stage_bytes(n);
+            const uint32_t off = alloc.next(size);
+            while (tail < nst) {
+                const uint32_t ts = tail % kSlots;
+                const bool slot_busy = nst - tail >= (uint32_t)kSlots;
+                const bool overlap = off < sc->r_end[ts] && sc->r_off[ts] < off + size;
+                if (!slot_busy && !overlap) break;
+                if (!mbar_wait(&sc->empty[ts], (tail / kSlots) & 1, ctl, x.timeout_ns, 902)) return false;
+                ++tail;
+            }
+            const uint32_t slot2 = nst % kSlots;
+            sc->r_off[slot2] = off;
+            sc->r_end[slot2] = off + size;
+            ++nst;
+            *slot_out = slot2;
+            *off_out = off;
+            return true;
+        };
+        auto issue_a = [&](uint32_t slot2, uint32_t off, const CUtensorMap* am2, const TaskDesc& dd, int stage,
+                           uint32_t tx, uint64_t pol) {
+            mbar_arrive_expect_tx(&sc->full[slot2], tx);
+            ++armed[slot2];
+            uint8_t* dst = arena + off;
+            const int kx = dd.k0 + stage * kTileK;
+            tma_load_2d(dst, am2, &sc->full[slot2], kx, dd.a_row0, pol);
+            tma_load_2d(dst + 64 * 128, am2, &sc->full[slot2], kx, dd.a_row1, pol);
+        };
         for (uint32_t it = 0;; ++it) {
             const uint32_t slot = it % kRing;
             if (lane == 0) {
@@ -282,22 +336,20 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             if (r == 1 && d.valid && d.gemm) {
                 const CUtensorMap* am = W::a_map(p, d.a_map);
                 const uint32_t bbytes = (uint32_t)d.n * 128u;
+                bool ok = true;
                 if (!d.gather) {
-                    // weights (A) of the first stages before the input wait, then B by TMA
-                    bool ok = true;
                     if (lane == 0) {
                         const CUtensorMap* bm = W::b_map(p, d.b_map);
-                        const int npre = d.nk < kStages ? d.nk : kStages;
-                        for (int s = 0; s < npre && ok; ++s) {
-                            const uint32_t ss = (st + s) % kStages;
-                            ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 902);
-                            if (!ok) break;
-                            mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
-                            ++armed[ss];
-                            uint8_t* dst = stages + ss * kStageBytes;
-                            const int kx = d.k0 + s * kTileK;
-                            tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
-                            tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
+                        // 1. weight tiles of the first stages, before the input
+                        //    wait (as many as fit without waiting on themselves)
+                        const int fit = kArenaBytes / (int)stage_bytes(d.n) - 1;
+                        int npre = d.nk < fit ? d.nk : fit;
+                        npre = npre < kSlots - 1 ? npre : kSlots - 1;
+                        uint32_t pslot[kSlots], poff[kSlots];
+                        int s = 0;
+                        for (; s < npre && ok; ++s) {
+                            ok = reserve(d.n, &pslot[s], &poff[s]);
+                            if (ok) issue_a(pslot[s], poff[s], am, d, s, kAStageBytes + bbytes, pol_w);
                         }
                         if (ok) ok = W::gemm_wait(p, x, d);  // the task's input event
                         if (ok && (x.debug & ET_DEBUG_TRACE)) {
@@ -307,28 +359,26 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         if (ok) fence_proxy_async_global();
                         sc->ring[slot] = d;
                         mbar_arrive(&sc->ring_full[slot]);
-                        for (int s = 0; s < d.nk && ok; ++s) {
-                            const uint32_t ss = (st + s) % kStages;
-                            uint8_t* dst = stages + ss * kStageBytes;
-                            const int kx = d.k0 + s * kTileK;
-                            if (s >= npre) {
-                                ok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 903);
-                                if (!ok) break;
-                                mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes + bbytes);
-                                ++armed[ss];
-                                tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
-                                tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
-                            }
+                        // 2. activation tiles of the prefetched stages
+                        for (int i = 0; ok && i < npre; ++i)
                             for (int rb = 0; rb < d.n; rb += 16)
-                                tma_load_2d(dst + kAStageBytes + rb * 128, bm, &sc->full[ss], kx, d.b_row0 + rb, pol_a);
+                                tma_load_2d(arena + poff[i] + kAStageBytes + rb * 128, bm, &sc->full[pslot[i]],
+                                            d.k0 + i * kTileK, d.b_row0 + rb, pol_a);
+                        // 3. the remaining stages, weights and activations together
+                        for (; ok && s < d.nk; ++s) {
+                            uint32_t sl, of;
+                            ok = reserve(d.n, &sl, &of);
+                            if (!ok) break;
+                            issue_a(sl, of, am, d, s, kAStageBytes + bbytes, pol_w);
+                            for (int rb = 0; rb < d.n; rb += 16)
+                                tma_load_2d(arena + of + kAStageBytes + rb * 128, bm, &sc->full[sl], d.k0 + s * kTileK,
+                                            d.b_row0 + rb, pol_a);
                         }
                         sc->pok = ok;
                     }
                     __syncwarp();
                     ok = sc->pok;
                     __syncwarp();
-                    st += d.nk;
-                    if (!ok) break;
                 } else {
                     // B rows gathered through an index list: every lane copies
                     // up to 4 rows per stage with cp.async into the 128-byte
@@ -337,7 +387,6 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     const uint16_t* rows[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) rows[i] = W::gather_row(p, d, lane + 32 * i);
-                    bool ok = true;
                     if (lane == 0) {
                         ok = W::gemm_wait(p, x, d);
                         if (ok && (x.debug & ET_DEBUG_TRACE)) {
@@ -352,16 +401,19 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     ok = sc->pok;
                     __syncwarp();
                     for (int s = 0; s < d.nk && ok; ++s) {
-                        const uint32_t ss = (st + s) % kStages;
-                        uint8_t* dst = stages + ss * kStageBytes;
-                        const int kx = d.k0 + s * kTileK;
-                        if (lane == 0)
-                            sc->pok = mbar_wait(&sc->empty[ss], (((st + s) / kStages) & 1) ^ 1, ctl, x.timeout_ns, 904);
+                        if (lane == 0) {
+                            uint32_t sl = 0, of = 0;
+                            sc->pok = reserve(d.n, &sl, &of);
+                            sc->pslot = sl;
+                            sc->poff = of;
+                        }
                         __syncwarp();
                         ok = sc->pok;
+                        const uint32_t sl = sc->pslot, of = sc->poff;
                         __syncwarp();
                         if (!ok) break;
-                        uint8_t* bdst = dst + kAStageBytes;
+                        const int kx = d.k0 + s * kTileK;
+                        uint8_t* bdst = arena + of + kAStageBytes;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int rr = lane + 32 * i;
@@ -372,18 +424,12 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                                     cp_async16(bdst + rr * 128 + ((c ^ (rr & 7)) << 4), src + c * 8);
                             }
                         }
-                        cp_async_mbar_arrive(&sc->full[ss]);
+                        cp_async_mbar_arrive(&sc->full[sl]);
                         __syncwarp();
-                        if (lane == 0) {
-                            mbar_arrive_expect_tx(&sc->full[ss], kAStageBytes);
-                            ++armed[ss];
-                            tma_load_2d(dst, am, &sc->full[ss], kx, d.a_row0, pol_w);
-                            tma_load_2d(dst + 64 * 128, am, &sc->full[ss], kx, d.a_row1, pol_w);
-                        }
+                        if (lane == 0) issue_a(sl, of, am, d, s, kAStageBytes, pol_w);
                     }
-                    st += d.nk;
-                    if (!ok) break;
                 }
+                if (!ok) break;
             } else {
                 if (lane == 0) {
                     sc->ring[slot] = d;
@@ -395,17 +441,18 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
         // drain: every armed stage's copies must land before the CTA exits
         if (any_gather) cp_async_wait_all();
         if (lane == 0)
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < kSlots; ++s)
                 if (armed[s]) {
-                    uint64_t t0 = globaltimer();
-                    while (!mbar_try_wait(&sc->full[s], (armed[s] - 1) & 1) && globaltimer() - t0 < 200000000ull) {
+                    uint64_t t1 = globaltimer();
+                    while (!mbar_try_wait(&sc->full[s], (armed[s] - 1) & 1) && globaltimer() - t1 < 200000000ull) {
                     }
                 }
         __syncwarp();
     } else if (!skip && warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
-            uint32_t st = 0, g = 0;
+            uint32_t nst = 0, g = 0;
+            StageAlloc alloc;
             bool issued_any = false;
             for (uint32_t it = 0;; ++it) {
                 const uint32_t slot = it % kRing;
@@ -419,16 +466,18 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 tc_fence_after();
                 const uint32_t dt = sc->tmem_base + buf * kMaxN;
                 const uint32_t idesc = idesc_bf16_f32(128, d.n);
+                const uint32_t size = stage_bytes(d.n);
                 bool ok = true;
-                for (int s = 0; s < d.nk; ++s) {
-                    const uint32_t ss = (st + s) % kStages;
-                    if (!mbar_wait(&sc->full[ss], ((st + s) / kStages) & 1, ctl, x.timeout_ns, 912)) {
+                for (int s = 0; s < d.nk; ++s, ++nst) {
+                    const uint32_t ss = nst % kSlots;
+                    const uint32_t off = alloc.next(size);
+                    if (!mbar_wait(&sc->full[ss], (nst / kSlots) & 1, ctl, x.timeout_ns, 912)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     fence_proxy_async_smem();  // rows copied by cp.async (generic proxy) -> tensor core
-                    const uint32_t a0 = smem_u32(stages + ss * kStageBytes);
+                    const uint32_t a0 = smem_u32(arena + off);
                     const uint64_t ad = sdesc_k128(a0);
                     const uint64_t bd = sdesc_k128(a0 + kAStageBytes);
 #pragma unroll
@@ -438,7 +487,6 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     issued_any = true;
                 }
                 if (!ok) break;
-                st += d.nk;
                 tc_commit(&sc->acc_full[buf]);
                 ++g;
             }

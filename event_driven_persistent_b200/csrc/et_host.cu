@@ -364,7 +364,7 @@ et_status build_moe(et_graph* g) {
     p.n_n1 = p.inter / p.n1_tile;
     p.n2_tile = 128;
     p.n_n2 = p.hidden / p.n2_tile;
-    p.cb = 16;
+    p.cb = 8;
     p.sched = d.sched;
     p.early_max = 2 * g->n_ctas;
     p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;

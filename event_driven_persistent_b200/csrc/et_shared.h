@@ -14,16 +14,22 @@ constexpr int kThreads = 192;
 constexpr int kExecThreads = 128;
 constexpr int kExecWarp0 = 2;
 constexpr int kRing = 2;           // task ring depth (warp 0 runs one task ahead)
-constexpr int kStages = 6;         // smem pipeline stages of the GEMM engine
 constexpr int kTileK = 64;         // K elements per stage (one 128-byte swizzle row)
+// Pipeline stages live in a circular smem arena: a stage holds the weight
+// tile (A, 16 KB) followed by the activation tile (B, N x 128 B rounded up to
+// 1 KB), so tasks with few token rows keep more weight bytes in flight
+// (11 stages at N = 16, 6 at N = 128).  kSlots mbarrier pairs track stages.
+constexpr int kSlots = 12;
+constexpr int kArenaBytes = 208 * 1024;
 constexpr int kAStageBytes = 128 * 128;  // 128 rows x 128 B
 constexpr int kBStageBytes = 128 * 128;  // up to 128 rows x 128 B
-constexpr int kStageBytes = kAStageBytes + kBStageBytes;
 constexpr int kMaxN = 128;         // largest MMA N (token rows per tile)
 constexpr int kTmemCols = 256;     // two accumulators of kMaxN fp32 columns
-constexpr int kEpiBytes = 64 * 32 * 4;   // gate/up exchange staging
-constexpr int kSimtBytes = 16384;        // scratch for CUDA-core tasks
-constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + kSimtBytes + 1024 /*barriers*/;
+constexpr int kScratchBytes = 16384;     // epilogue staging and CUDA-core task scratch
+constexpr int kEpiBytes = 64 * 33 * 4;   // gate/up exchange staging (start of the scratch)
+constexpr int kCtlBytes = 2048;          // mbarriers, task ring, broadcast words
+constexpr int kSmemBytes = 1024 /*align slack*/ + kArenaBytes + kScratchBytes + kCtlBytes;
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
 // Per-bucket static task lists: CSR over CTAs.
 struct StaticLists {

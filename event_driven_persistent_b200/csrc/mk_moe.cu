@@ -290,7 +290,13 @@ struct Moe {
         if (op == ET_OP_MOE_TOPK) return topk_task(p, x, d, a);
         if (op == ET_OP_MOE_SCAN) return scan_task(p, x, d);
         if (op == ET_OP_MOE_GROUP) return group_task(p, x, d, a);
-        // COMBINE
+        return combine_task(p, x, d);
+    }
+
+
+    // CB(b): Y = bf16(Yacc) for tokens [cb*b, cb*b + cb), and Yacc back to 0.
+    __device__ static bool combine_task(const Params& p, Ctx& x, TaskDesc& d) {
+        const int a = task_a(d.word);
         const int t0 = a * p.cb;
         const int ntok = min(p.cb, p.T - t0);
         if (is_unfused(p)) {
