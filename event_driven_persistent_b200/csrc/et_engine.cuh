@@ -151,7 +151,8 @@ __device__ __forceinline__ bool group_wait(Ctx& x, TaskDesc& d, const int* ctr, 
 
 // Bytes of one pipeline stage: the weight tile, then N activation rows
 // (1 KB multiples keep every tile on the 128-byte swizzle atom).
-__device__ __forceinline__ uint32_t stage_bytes(int n) { return kAStageBytes + ((n * 128 + 1023) & ~1023); }
+// (per K atom: 128 weight rows, then N activation rows; n is a multiple of 16)
+__device__ __forceinline__ uint32_t stage_bytes(int n) { return kAStageBytes + 2u * (uint32_t)n * 128u; }
 
 // Circular allocation of stages in the arena; the producer and the MMA
 // issuer replay the same sequence, so both know every stage's address.
@@ -285,14 +286,27 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             *off_out = off;
             return true;
         };
+        auto issue_b = [&](uint32_t slot2, uint32_t off, const CUtensorMap* bm2, const TaskDesc& dd, int stage,
+                           uint64_t pol) {
+            uint8_t* bdst = arena + off + kAStageBytes;
+            const uint32_t atom = (uint32_t)dd.n * 128u;
+            const int kx = dd.k0 + stage * kTileK;
+            for (int rb = 0; rb < dd.n; rb += 16)
+#pragma unroll
+                for (int at = 0; at < 2; ++at)
+                    tma_load_2d(bdst + at * atom + rb * 128, bm2, &sc->full[slot2], kx + at * kAtomK, dd.b_row0 + rb, pol);
+        };
         auto issue_a = [&](uint32_t slot2, uint32_t off, const CUtensorMap* am2, const TaskDesc& dd, int stage,
                            uint32_t tx, uint64_t pol) {
             mbar_arrive_expect_tx(&sc->full[slot2], tx);
             ++armed[slot2];
             uint8_t* dst = arena + off;
             const int kx = dd.k0 + stage * kTileK;
-            tma_load_2d(dst, am2, &sc->full[slot2], kx, dd.a_row0, pol);
-            tma_load_2d(dst + 64 * 128, am2, &sc->full[slot2], kx, dd.a_row1, pol);
+#pragma unroll
+            for (int at = 0; at < 2; ++at) {
+                tma_load_2d(dst + at * kAAtomBytes, am2, &sc->full[slot2], kx + at * kAtomK, dd.a_row0, pol);
+                tma_load_2d(dst + at * kAAtomBytes + 64 * 128, am2, &sc->full[slot2], kx + at * kAtomK, dd.a_row1, pol);
+            }
         };
         for (uint32_t it = 0;; ++it) {
             const uint32_t slot = it % kRing;
@@ -335,7 +349,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             if (brk) break;
             if (r == 1 && d.valid && d.gemm) {
                 const CUtensorMap* am = W::a_map(p, d.a_map);
-                const uint32_t bbytes = (uint32_t)d.n * 128u;
+                const uint32_t bbytes = 2u * (uint32_t)d.n * 128u;  // both K atoms
                 bool ok = true;
                 if (!d.gather) {
                     if (lane == 0) {
@@ -361,18 +375,14 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         mbar_arrive(&sc->ring_full[slot]);
                         // 2. activation tiles of the prefetched stages
                         for (int i = 0; ok && i < npre; ++i)
-                            for (int rb = 0; rb < d.n; rb += 16)
-                                tma_load_2d(arena + poff[i] + kAStageBytes + rb * 128, bm, &sc->full[pslot[i]],
-                                            d.k0 + i * kTileK, d.b_row0 + rb, pol_a);
+                            issue_b(pslot[i], poff[i], bm, d, i, pol_a);
                         // 3. the remaining stages, weights and activations together
                         for (; ok && s < d.nk; ++s) {
                             uint32_t sl, of;
                             ok = reserve(d.n, &sl, &of);
                             if (!ok) break;
                             issue_a(sl, of, am, d, s, kAStageBytes + bbytes, pol_w);
-                            for (int rb = 0; rb < d.n; rb += 16)
-                                tma_load_2d(arena + of + kAStageBytes + rb * 128, bm, &sc->full[sl], d.k0 + s * kTileK,
-                                            d.b_row0 + rb, pol_a);
+                            issue_b(sl, of, bm, d, s, pol_a);
                         }
                         sc->pok = ok;
                     }
@@ -414,14 +424,15 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         if (!ok) break;
                         const int kx = d.k0 + s * kTileK;
                         uint8_t* bdst = arena + of + kAStageBytes;
+                        const uint32_t atom = (uint32_t)d.n * 128u;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int rr = lane + 32 * i;
                             if (rows[i]) {
                                 const uint16_t* src = rows[i] + kx;
 #pragma unroll
-                                for (int c = 0; c < 8; ++c)
-                                    cp_async16(bdst + rr * 128 + ((c ^ (rr & 7)) << 4), src + c * 8);
+                                for (int c = 0; c < 16; ++c)
+                                    cp_async16(bdst + (c >> 3) * atom + rr * 128 + (((c & 7) ^ (rr & 7)) << 4), src + c * 8);
                             }
                         }
                         cp_async_mbar_arrive(&sc->full[sl]);
@@ -478,11 +489,14 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     tc_fence_after();
                     fence_proxy_async_smem();  // rows copied by cp.async (generic proxy) -> tensor core
                     const uint32_t a0 = smem_u32(arena + off);
-                    const uint64_t ad = sdesc_k128(a0);
-                    const uint64_t bd = sdesc_k128(a0 + kAStageBytes);
 #pragma unroll
-                    for (int kk = 0; kk < kTileK / 16; ++kk)
-                        tc_mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, idesc, (s | kk) ? 1u : 0u);
+                    for (int at = 0; at < 2; ++at) {
+                        const uint64_t ad = sdesc_k128(a0 + at * kAAtomBytes);
+                        const uint64_t bd = sdesc_k128(a0 + kAStageBytes + at * (uint32_t)d.n * 128u);
+#pragma unroll
+                        for (int kk = 0; kk < kAtomK / 16; ++kk)
+                            tc_mma_bf16(dt, ad + 2 * kk, bd + 2 * kk, idesc, (s | at | kk) ? 1u : 0u);
+                    }
                     tc_commit(&sc->empty[ss]);
                     issued_any = true;
                 }

@@ -279,7 +279,7 @@ et_status build_mlp(et_graph* g) {
     if (d.rms_eps <= 0.f) d.rms_eps = 1e-5f;
     if (d.fetch_batch <= 0) d.fetch_batch = 1;
     if (d.max_T > kMaxN) return ET_ERR_UNSUPPORTED;  // one token tile
-    if (d.hidden % 128 || d.inter % 64) return ET_ERR_UNSUPPORTED;
+    if (d.hidden % 128 || d.inter % 128) return ET_ERR_UNSUPPORTED;
     MlpParams& p = g->mlp;
     memset(&p, 0, sizeof(p));
     p.hidden = d.hidden;
@@ -288,7 +288,7 @@ et_status build_mlp(et_graph* g) {
     p.eps = d.rms_eps;
     p.gu_tile = 64;
     p.down_tile = 128;
-    p.kchunk = d.inter % 1024 == 0 ? 1024 : (d.inter % 256 == 0 ? 256 : 64);
+    p.kchunk = d.inter % 1024 == 0 ? 1024 : (d.inter % 256 == 0 ? 256 : 128);
     p.n_gu = d.inter / p.gu_tile;
     p.n_m = d.hidden / p.down_tile;
     p.n_c = d.inter / p.kchunk;
@@ -349,7 +349,7 @@ et_status build_moe(et_graph* g) {
     if (d.top_k <= 0) d.top_k = 8;
     if (d.fetch_batch <= 0) d.fetch_batch = 1;
     if (d.n_experts > 128 || d.n_experts % 8 || d.top_k > 8 || d.top_k > d.n_experts) return ET_ERR_UNSUPPORTED;
-    if (d.hidden % 128 || d.inter % 64) return ET_ERR_UNSUPPORTED;
+    if (d.hidden % 128 || d.inter % 128) return ET_ERR_UNSUPPORTED;
     MoeParams& p = g->moe;
     memset(&p, 0, sizeof(p));
     p.hidden = d.hidden;

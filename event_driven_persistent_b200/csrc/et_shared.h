@@ -14,14 +14,16 @@ constexpr int kThreads = 192;
 constexpr int kExecThreads = 128;
 constexpr int kExecWarp0 = 2;
 constexpr int kRing = 2;           // task ring depth (warp 0 runs one task ahead)
-constexpr int kTileK = 64;         // K elements per stage (one 128-byte swizzle row)
+constexpr int kTileK = 128;        // K elements per stage: two 128-byte swizzle atoms along K
+constexpr int kAtomK = 64;         // K elements per swizzle atom (one 128-byte row)
 // Pipeline stages live in a circular smem arena: a stage holds the weight
 // tile (A, 16 KB) followed by the activation tile (B, N x 128 B rounded up to
 // 1 KB), so tasks with few token rows keep more weight bytes in flight
 // (11 stages at N = 16, 6 at N = 128).  kSlots mbarrier pairs track stages.
 constexpr int kSlots = 12;
 constexpr int kArenaBytes = 208 * 1024;
-constexpr int kAStageBytes = 128 * 128;  // 128 rows x 128 B
+constexpr int kAAtomBytes = 128 * 128;   // weight tile of one atom: 128 rows x 128 B
+constexpr int kAStageBytes = 2 * kAAtomBytes;
 constexpr int kBStageBytes = 128 * 128;  // up to 128 rows x 128 B
 constexpr int kMaxN = 128;         // largest MMA N (token rows per tile)
 constexpr int kTmemCols = 256;     // two accumulators of kMaxN fp32 columns
