@@ -60,6 +60,7 @@ _sigs = {
     "et_run_splitk": ([_P, _P, _I, _P, _P, _P], _I),
     "et_run_mlp": ([_P, _I, _P, _P, _P, _P, _P, _P], _I),
     "et_run_moe": ([_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], _I),
+    "et_run_splitk_noalloc": ([_P, _I, _P, _P, _P], _I),
     "et_sync_status": ([_P, _P], _I),
     "et_get_trace": ([_P, _P, ctypes.c_size_t, ctypes.POINTER(_I)], _I),
     "et_get_info": ([_P, ctypes.POINTER(et_graph_info)], _I),
@@ -111,6 +112,11 @@ def et_build_graph(kind, sched, max_T, **dims):
 
 def et_run_splitk(g, A, n_rows, Bpart, C, stream=None):
     _check(_lib.et_run_splitk(g, _ptr(A), n_rows, _ptr(Bpart), _ptr(C), _stream(stream)), "et_run_splitk")
+
+
+def et_run_splitk_noalloc(A, n_rows, Bpart, C, stream=None):
+    """Allocation-free split-K (synchronous); returns the status code."""
+    return _lib.et_run_splitk_noalloc(_ptr(A), n_rows, _ptr(Bpart), _ptr(C), _stream(stream))
 
 
 def et_run_mlp(g, B, X, gamma, Wgu, Wd, Y, stream=None):

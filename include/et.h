@@ -183,6 +183,33 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
                      const uint16_t* W1, const uint16_t* W2, uint16_t* Y, int32_t* topk,
                      float* topk_w, int32_t* indptr, int32_t* perm, float* logits, void* stream);
 
+/* Split-K reduction without any device allocation.  (No counterpart in the
+ * paper: this is an interface addition of this library.)
+ *
+ * Some callers cannot call cudaMalloc: a plugin running inside a host
+ * framework that owns every device allocation and gives the plugin no
+ * allocator, or a latency-critical path that cannot afford cudaMalloc's
+ * implicit device synchronisation.  They cannot build an et_graph (its
+ * workspace is allocated), so this entry point runs the same split-K
+ * megakernel with its whole workspace -- event counters, ready queue and
+ * control block -- in one file-scope device array of 108,032 bytes that
+ * every GPU loading libet.so holds until the process exits.  It calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *   - Same computation and arguments as et_run_splitk (A fp32 [n_rows, 128],
+ *     chunk 32, Bpart fp32 [n_rows, 4], C fp32 [n_rows]), dynamic schedule.
+ *   - 0 <= n_rows <= 65536; larger n_rows returns ET_ERR_INVALID before any
+ *     CUDA call.  Null or misaligned pointers: ET_ERR_INVALID.
+ *   - The first call on a device does a one-time set-up there (it resolves
+ *     the array's device address and clears it with cudaMemsetAsync on
+ *     `stream`); make that first call before any stream capture.
+ *   - Synchronous: it waits for `stream`, then returns the device status of
+ *     this call (ET_ERR_TIMEOUT if a wait gave up, after which the workspace
+ *     is cleared again).
+ *   - Every call on a device shares the one array, which keeps the last
+ *     call's contents; calls that overlap on the GPU (other streams, other
+ *     host threads) race on it and must not be issued. */
+et_status et_run_splitk_noalloc(const float* A, int n_rows, float* Bpart, float* C, void* stream);
+
 /* Synchronise `stream`, then read and clear the graph's sticky device
  * status.  Returns ET_OK, or ET_ERR_TIMEOUT if a wait of any run since the
  * last call gave up (every CTA then drained and exited; no trap).  After a

@@ -41,6 +41,9 @@ def test_status_strings_and_null_checks():
     assert lib.et_run_mlp(None, 1, None, None, None, None, None, None) == et.ET_ERR_INVALID
     assert lib.et_run_moe(None, 1, *([None] * 12)) == et.ET_ERR_INVALID
     assert lib.et_sync_status(None, None) == et.ET_ERR_INVALID
+    # the allocation-free split-K rejects sizes beyond its maximum before any CUDA call
+    assert lib.et_run_splitk_noalloc(None, 65537, None, None, None) == et.ET_ERR_INVALID
+    assert lib.et_run_splitk_noalloc(None, 16, None, None, None) == et.ET_ERR_INVALID
 
 
 def test_bad_descriptor_rejected():
