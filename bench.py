@@ -121,6 +121,21 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm --
+def combine_ranks(ms, e2e_ms, nbytes, world, device):
+    """Whole-job figures of a replicas run: the max over ranks of the step
+    times (device-timed) and the algorithmic bytes summed over ranks.  Every
+    rank calls it (two all-reduces, in the same order on every rank)."""
+    if world <= 1:
+        return float(ms), float(e2e_ms), float(nbytes)
+    import torch
+    vals = torch.tensor([ms, e2e_ms, float(nbytes)], dtype=torch.float64, device=device)
+    mx = vals.clone()
+    torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
+    sm = vals.clone()
+    torch.distributed.all_reduce(sm, op=torch.distributed.ReduceOp.SUM)
+    return float(mx[0]), float(mx[1]), float(sm[2])
+
+
 def gpu_arm(args, rank, world, local_rank):
     import torch
     import event_driven_persistent_b200 as et
@@ -191,16 +206,7 @@ def gpu_arm(args, rank, world, local_rank):
             e2e_ms.append(a.elapsed_time(b))
     e2e = sum(e2e_ms) / len(e2e_ms)
 
-    # max over ranks of the per-step time; bytes summed over ranks
-    vals = torch.tensor([ms, e2e, float(nbytes)], dtype=torch.float64, device=dev)
-    if world > 1:
-        mx = vals.clone()
-        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
-        sm = vals.clone()
-        torch.distributed.all_reduce(sm, op=torch.distributed.ReduceOp.SUM)
-        ms, e2e, tot_bytes = float(mx[0]), float(mx[1]), float(sm[2])
-    else:
-        tot_bytes = float(nbytes)
+    ms, e2e, tot_bytes = combine_ranks(ms, e2e, nbytes, world, dev)
     et.et_destroy_graph(g)
     if rank != 0:
         return None
