@@ -262,7 +262,7 @@ def cpu_oracle(args, budget_s=15.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--T", type=int, default=128)
     ap.add_argument("--max_T", type=int, default=4096)

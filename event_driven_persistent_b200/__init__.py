@@ -44,7 +44,7 @@ class et_graph_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "kind", "sched", "max_T", "n_ctas", "threads", "smem_bytes", "fetch_batch", "hidden", "inter",
         "n_experts", "top_k", "splitk_cols", "splitk_chunk", "splitk_tile_rows", "mlp_gu_tile", "mlp_down_tile",
-        "mlp_kchunk", "moe_tt", "moe_gt", "moe_tkt", "moe_bm", "moe_n1_tile", "moe_n2_tile", "moe_cb", "moe_router_kc")]
+        "mlp_kchunk", "moe_tt", "moe_gt", "moe_tkt", "moe_bm", "moe_n1_tile", "moe_n2_tile", "moe_cb")]
 
 
 class et_trace_record(ctypes.Structure):

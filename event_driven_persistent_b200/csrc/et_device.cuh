@@ -79,11 +79,16 @@ __device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gp
 
 // Spin back-off: 148 SMs polling a few counters must not flood the L2 slice
 // that holds them (which slows every other access to that slice).
+// Exponential back-off between polls, 32 ns up to `cap` ns: short enough
+// that a hop from one task to the next costs little, long enough that
+// 148 pollers do not crowd the L2 slice of one counter.
 struct Backoff {
     uint32_t ns = 32;
+    uint32_t cap = 512;
+    __device__ __forceinline__ explicit Backoff(uint32_t c = 512) : cap(c) {}
     __device__ __forceinline__ void pause() {
         __nanosleep(ns);
-        if (ns < 1024) ns <<= 1;
+        if (ns < cap) ns <<= 1;
     }
 };
 
@@ -386,7 +391,7 @@ __device__ __forceinline__ int q_resolve(const Queue& q, int idx, uint32_t* word
     if (idx >= q.cap) return 0;  // beyond any run's last task
     const unsigned long long* s = &q.slots[idx];
     uint64_t t0 = 0;
-    Backoff bo;
+    Backoff bo(256);
     for (uint32_t it = 0;; ++it) {
         unsigned long long v = ld_relaxed_u64(s);
         if ((uint32_t)(v >> 32) == q.epoch) {

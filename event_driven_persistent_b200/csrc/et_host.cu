@@ -324,18 +324,21 @@ et_status build_mlp(et_graph* g) {
 
 // ----------------------------------------------------------------- MoE ----
 struct MoeShape {
-    int n_tt, n_kc, n_tk, n_cb, f_max;
+    int n_tt, n_tk, cb, n_cb, f_max;
 };
+
+// Tokens per combine task: one while the layer is small (the combine is the
+// layer's tail, so it is spread over as many SMs as there are tokens), eight
+// beyond 256 tokens (fewer, larger tasks once there are more tokens than SMs).
+constexpr int kCbOneMaxT = 256;
+inline int moe_cb_for(int T) { return T <= kCbOneMaxT ? 1 : 8; }
 
 MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
     MoeShape m;
     m.n_tt = cdiv(T, p.tt);
-    // router K split: enough (token tile, chunk) tasks to cover the SMs
-    int kc = 1;
-    while (kc < 8 && m.n_tt * kc * 2 <= g->n_ctas && (p.hidden / (kc * 2)) % kTileK == 0) kc *= 2;
-    m.n_kc = kc;
-    m.n_cb = cdiv(T, p.cb);
     m.n_tk = cdiv(T, p.tkt);
+    m.cb = moe_cb_for(T);
+    m.n_cb = cdiv(T, m.cb);
     const int pairs = p.k * T;
     m.f_max = std::min(pairs, std::min(p.E, pairs) + cdiv(pairs, p.bm));
     return m;
@@ -364,7 +367,7 @@ et_status build_moe(et_graph* g) {
     p.n_n1 = p.inter / p.n1_tile;
     p.n2_tile = 128;
     p.n_n2 = p.hidden / p.n2_tile;
-    p.cb = 8;
+    p.cb = moe_cb_for(d.max_T);
     p.sched = d.sched;
     p.early_max = 2 * g->n_ctas;
     p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
@@ -374,23 +377,20 @@ et_status build_moe(et_graph* g) {
     p.ev_tk = ev++;
     p.ev_sc = ev++;
     p.ev_grp = ev++;
-    p.ev_rt_all = ev++;
     p.ev_s1_all = ev++;
     p.ev_s2_all = ev++;
-    p.ev_rt = ev;
-    ev += mx.n_tt;
     p.ev_exp = ev;
     ev += p.E;
     p.ev_s1 = ev;
     ev += mx.f_max;
     p.ev_cb = ev;
-    ev += mx.n_cb;
+    const int n_cb_max = std::max(mx.n_cb, std::min(d.max_T, kCbOneMaxT));  // over every size bucket
+    ev += n_cb_max;
     p.ev_gcnt = ev;
     ev += mx.n_tt * p.E;
     g->n_ctr = ev;
-    g->qcap = mx.n_tt * 8 + mx.n_tk + mx.n_tt + 1 + mx.f_max * (p.n_n1 + p.n_n2) + mx.n_cb + g->n_ctas * d.fetch_batch + 64;
+    g->qcap = mx.n_tk + mx.n_tt + 1 + mx.f_max * (p.n_n1 + p.n_n2) + n_cb_max + g->n_ctas * d.fetch_batch + 64;
     const size_t pairs = (size_t)p.maxT * p.k;
-    ET_TRY(galloc(g, &p.lacc, (size_t)p.maxT * p.E));
     ET_TRY(galloc(g, &p.topk, pairs));
     ET_TRY(galloc(g, &p.topw, pairs));
     ET_TRY(galloc(g, &p.goff, (size_t)mx.n_tt * p.E));
@@ -410,10 +410,8 @@ et_status build_moe(et_graph* g) {
     const float c_s1 = 2.f * p.n1_tile * p.hidden * 2 / 1024.f, c_s2 = (float)p.n2_tile * p.inter * 2 / 1024.f;
     return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
         MoeShape m = moe_shape(g, p, Tb);
-        const float c_rt = (float)p.E * p.hidden * 2 / m.n_kc / 1024.f;
-        for (int t = 0; t < m.n_tt; ++t)
-            for (int c = 0; c < m.n_kc; ++c) s.push_back({tw(ET_OP_MOE_ROUTER, t, c), c_rt});
-        for (int j = 0; j < m.n_tk; ++j) s.push_back({tw(ET_OP_MOE_TOPK, j, 0), 8.f});
+        const float c_rt = (float)p.E * p.hidden * 2 / 1024.f;
+        for (int j = 0; j < m.n_tk; ++j) s.push_back({tw(ET_OP_MOE_ROUTER, j, 0), c_rt});
         s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 8.f});
         if (m.n_tt > 1)
             for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_GROUP, t, 0), 8.f});
@@ -506,8 +504,7 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
         in.moe_bm = g->moe.bm;
         in.moe_n1_tile = g->moe.n1_tile;
         in.moe_n2_tile = g->moe.n2_tile;
-        in.moe_cb = g->moe.cb;
-        in.moe_router_kc = g->moe.n_kc;
+        in.moe_cb = moe_cb_for(g->d.max_T);
     }
     *out = g;
     return ET_OK;
@@ -595,13 +592,13 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
     const int b = g->bucket_of(T);
     const MoeShape mb = moe_shape(g, p, g->bucket_T[b]);
     const MoeShape mt = moe_shape(g, p, T);
-    p.n_kc = mb.n_kc;  // the bucket fixes the router split (static lists and dynamic alike)
     p.n_tt = mt.n_tt;
     p.n_tk = mt.n_tk;
-    p.n_cb = mt.n_cb;
+    p.cb = mb.cb;  // the size bucket fixes the combine block (static lists and dynamic alike)
+    p.n_cb = cdiv(T, p.cb);
     p.f_max = mb.f_max;
     ET_TRY(pre_run(g, s));
-    RunArgs ra = run_args(g, T, p.n_tt * p.n_kc, 0);
+    RunArgs ra = run_args(g, T, p.n_tk, 0);
     ET_CU(launch_moe(p, ra, g->n_ctas, s));
     return ET_OK;
 }
@@ -619,7 +616,6 @@ et_status et_sync_status(et_graph* g, void* stream) {
     ET_CU(cudaMemset(g->ctr[1], 0, g->n_ctr * sizeof(int)));
     if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc) {
         ET_CU(cudaMemset(g->moe.Yacc, 0, (size_t)g->moe.maxT * g->moe.hidden * sizeof(float)));
-        ET_CU(cudaMemset(g->moe.lacc, 0, (size_t)g->moe.maxT * g->moe.E * sizeof(float)));
     }
     ET_CU(cudaDeviceSynchronize());
     // keep the diagnostic words readable through et_get_diag

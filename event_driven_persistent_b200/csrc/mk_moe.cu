@@ -17,15 +17,15 @@
 //     weights stream while stage 1 computes.
 //
 // Task graph (counts in brackets; dynamic schedule; tiles of 128 tokens):
-//   RT(t, c)  router partial logits of token tile t, K chunk c   -> E_rt[t] [#chunks]
-//   TK(j)     16 tokens: sum partials + bias, top-k, softmax, tile counts -> E_tk [#top-k tasks]
+//   RT(j)     16 tokens: router GEMM (full K, tensor cores), + bias, top-k and
+//             softmax in the epilogue, pair counts per 128-token tile -> E_tk [#router tasks]
 //   SC        expert counts, CSR (indptr, m-tile indptr), tile offsets -> E_sc [1]
 //             (run by the task that completes E_tk; with T <= 128 it is also the
 //             grouping task -> E_exp[topk[i,:]])
 //   GR(t)     grouped row of every pair of token tile t          -> E_exp[topk[i,:]]
 //   S1(f, n)  m-tile f (expert e, <= 128 rows gathered from X) x 64 intermediate cols -> E_s1[f] [#n1]
 //   S2(f, n)  m-tile f x 128 output cols, weighted red.add into Yacc -> E_cb[t / cb]
-//   CB(b)     Y = bf16(Yacc) for a block of cb tokens, Yacc = 0
+//   CB(b)     Y = bf16(Yacc) for a block of cb tokens (1 up to 256 tokens, else 8), Yacc = 0
 #include <cuda_bf16.h>
 
 #include "et_engine.cuh"
@@ -39,8 +39,6 @@ __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 __device__ __forceinline__ void red_add(float* p, float v) {
     asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
-// (value desc, index asc) total order
-__device__ __forceinline__ bool better(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
 
 // Exclusive prefix sum over the 128 exec threads (value v of thread tid);
 // returns the prefix, *total gets the sum.  `tmp` holds 4 ints of smem.
@@ -72,9 +70,7 @@ struct Moe {
 
     __device__ static bool is_unfused(const Params& p) { return p.sched == ET_SCHED_UNFUSED; }
 
-    __device__ static uint32_t fetch_init(const Params& p, int idx) {
-        return task_word(ET_OP_MOE_ROUTER, idx / p.n_kc, idx % p.n_kc);
-    }
+    __device__ static uint32_t fetch_init(const Params& p, int idx) { return task_word(ET_OP_MOE_ROUTER, idx, 0); }
 
     // m-tile f -> (expert, first grouped row, rows); needs the scan's outputs
     __device__ static void mtile(const Params& p, int f, int& e, int& row0, int& cnt) {
@@ -89,19 +85,17 @@ struct Moe {
         d.valid = 1;
         d.gemm = 0;
         if (op == ET_OP_MOE_ROUTER) {
-            d.valid = a < p.n_tt;
-            const int cnt = min(p.tt, p.T - a * p.tt);
+            // rows = the E experts of Wr, columns = the task's 16 tokens
+            d.valid = a < p.n_tk;
             d.gemm = 1;
             d.a_map = MOE_MAP_WR;
             d.a_row0 = 0;
             d.a_row1 = 64;
             d.b_map = MOE_MAP_X;
-            d.b_row0 = a * p.tt;
-            d.n = (cnt + 15) & ~15;
-            d.nk = p.hidden / p.n_kc / kTileK;
-            d.k0 = b * (p.hidden / p.n_kc);
-        } else if (op == ET_OP_MOE_TOPK) {
-            d.valid = a < p.n_tk;
+            d.b_row0 = a * p.tkt;
+            d.n = 16;
+            d.nk = p.hidden / kTileK;
+            d.k0 = 0;
         } else if (op == ET_OP_MOE_GROUP) {
             d.valid = p.n_tt > 1 && a < p.n_tt;  // one tile: the scan task groups
         } else if (op == ET_OP_MOE_COMBINE) {
@@ -184,27 +178,25 @@ struct Moe {
         const int q = (w + kExecWarp0) & 3;
         const int r = q * 32 + lane;
         if (op == ET_OP_MOE_ROUTER) {
-            // rows = experts, columns = tokens of tile a: add K chunk b's partial
-            // logits into lacc (the L2 performs the reduction over the chunks)
-            const int t0 = a * p.tt;
-            const int cnt = min(p.tt, p.T - t0);
-            for (int c0 = 0; c0 < d.n; c0 += 16) {
-                float v[16];
-                acc_load16(taddr, c0, v);
-                if (c0 + 16 >= d.n) acc_release(acc_empty);
-                if (r < p.E) {
+            // logits of the task's 16 tokens (+ bias), transposed through
+            // smem: L[token][expert], rows padded to 132 floats
+            const int t0 = a * p.tkt;
+            const int ntok = min(p.tkt, p.T - t0);
+            float* L = x.epi;
+            float v[16];
+            acc_load16(taddr, 0, v);
+            acc_release(acc_empty);
+            if (r < p.E) {
+                const float bb = p.bias[r];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c0 + i < cnt) red_add(p.lacc + (size_t)(t0 + c0 + i) * p.E + r, v[i]);
+                for (int c = 0; c < 16; ++c) {
+                    const float lg = v[c] + bb;
+                    L[c * 132 + r] = lg;
+                    if (p.out_logits && c < ntok) p.out_logits[(size_t)(t0 + c) * p.E + r] = lg;
                 }
             }
-            int* ev = x.ctr + (is_unfused(p) ? p.ev_rt_all : p.ev_rt + a);
-            const int tgt = is_unfused(p) ? p.n_tt * p.n_kc : p.n_kc;
-            const bool fired = group_finish_notify(x, d, ev, 1, tgt);
-            if (fired && x.dynamic) {
-                const int j0 = a * (p.tt / p.tkt), nj = min(p.tt / p.tkt, p.n_tk - j0);
-                group_push(x, nj, [&](int i) { return task_word(ET_OP_MOE_TOPK, j0 + i, 0); });
-            }
+            exec_bar();
+            return route_topk(p, x, d, a, L);
         } else if (op == ET_OP_MOE_S1) {
             const int row0 = d.p[1], cnt = d.p[2];
             const bool is_up = q >= 2;
@@ -265,7 +257,12 @@ struct Moe {
                 group_finish_notify(x, d, x.ctr + p.ev_s2_all, 1, -1);
             } else {
                 group_finish_notify(x, d, nullptr, 0, 0);
-                // one notify per run of rows in the same combine block
+                // One notify per run of rows in the same combine block.  Under
+                // the dynamic schedule the first block this task completes is
+                // converted here and the others are queued.
+                int* fired = reinterpret_cast<int*>(s_w + 128);  // [128] completed blocks
+                if (x.tid == 0) x.sc->bcast[7] = 0;
+                exec_bar();
                 if (x.tid < cnt) {
                     const int c = x.tid;
                     const int blk = s_tok[c] / p.cb;
@@ -276,8 +273,21 @@ struct Moe {
                         const int ntok = min(p.cb, p.T - blk * p.cb);
                         const int tgt = p.k * p.n_n2 * ntok;
                         if (notify(x.ctr + p.ev_cb + blk, len) == tgt && x.dynamic)
-                            thread_push(x, 1, [&](int) { return task_word(ET_OP_MOE_COMBINE, blk, 0); });
+                            fired[atomicAdd(&x.sc->bcast[7], 1)] = blk;
                     }
+                }
+                exec_bar();
+                const int nf = x.sc->bcast[7];
+                if (nf > 0) {
+                    // the run's task total counts every combine block, so the
+                    // block converted here is queued as an empty placeholder
+                    // (block index n_cb, which derive marks invalid)
+                    group_push(x, nf, [&](int i) { return task_word(ET_OP_MOE_COMBINE, i == 0 ? p.n_cb : fired[i], 0); });
+                    TaskDesc cd = d;
+                    cd.word = task_word(ET_OP_MOE_COMBINE, fired[0], 0);
+                    cd.t_fetch = cd.t_acc = 0;
+                    if (x.debug & ET_DEBUG_TRACE) cd.t_fetch = globaltimer();
+                    if (!combine_task(p, x, cd)) return false;
                 }
                 exec_bar();  // s_tok is reused by the next task
             }
@@ -287,7 +297,6 @@ struct Moe {
 
     __device__ static bool simt(const Params& p, Ctx& x, TaskDesc& d) {
         const int op = task_op(d.word), a = task_a(d.word);
-        if (op == ET_OP_MOE_TOPK) return topk_task(p, x, d, a);
         if (op == ET_OP_MOE_SCAN) return scan_task(p, x, d);
         if (op == ET_OP_MOE_GROUP) return group_task(p, x, d, a);
         return combine_task(p, x, d);
@@ -335,17 +344,14 @@ struct Moe {
     }
 
     // Exec-group scratch of the routing tasks (x.epi and x.simt, which are
-    // contiguous and free while the exec group runs a CUDA-core task):
-    //   L     [16][132] fp32  logits of 16 tokens; expert e of token t at
-    //                         t*132 + (e/32)*33 + e%32 (bank-conflict free);
-    //                         reused for the per-quarter top-8 lists
+    // contiguous and free while the exec group runs a routing task), after
+    // the router's logits L [16][132] fp32 at x.epi:
     //   tk    [128 * k] int   selected experts of a 128-token tile, pair order
     //   emask [128][4]  u32   per expert: bit t = token t of the tile picked it
     //   base  [128] int       first grouped row per expert (placement)
     //   hist  [128] int       pairs per expert of a top-k task
     //   misc  [8] int
     struct RouteSmem {
-        float* L;
         int* tk;
         uint32_t* emask;
         int* base;
@@ -354,8 +360,7 @@ struct Moe {
     };
     __device__ static RouteSmem route_smem(Ctx& x) {
         RouteSmem s;
-        s.L = x.epi;
-        s.tk = reinterpret_cast<int*>(x.epi + 16 * 132);
+        s.tk = reinterpret_cast<int*>(x.epi + 16 * 132);  // after the router's logits L
         s.emask = reinterpret_cast<uint32_t*>(s.tk + 128 * 8);
         s.base = reinterpret_cast<int*>(s.emask + 128 * 4);
         s.hist = s.base + 128;
@@ -363,113 +368,85 @@ struct Moe {
         return s;
     }
 
-    // Insert candidate (v, i) into a descending top-8 list (order: logit
-    // desc, index asc).  The list keeps the 8 best candidates seen so far.
-    __device__ static void ins8(float (&tv)[8], int (&ti)[8], float v, int i) {
-        if (!better(v, i, tv[7], ti[7])) return;
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            const bool c = better(v, i, tv[s], ti[s]);
-            const float ov = tv[s];
-            const int oi = ti[s];
-            tv[s] = c ? v : ov;
-            ti[s] = c ? i : oi;
-            v = c ? ov : v;
-            i = c ? oi : i;
-        }
+    // Top-k of router task j (tokens [16j, 16j+16)) from its logits L
+    // [16][132] in smem: top-k by (logit desc, index asc), softmax of the
+    // selected logits, pair counts per expert of the token's 128-token tile.
+    // Thread (g, q) = (tid / 8, tid % 8) holds experts 16q .. 16q+15 of token
+    // g as 64-bit keys (order-preserving logit bits, then the complemented
+    // index, so a larger key is a better candidate); the eight threads of a
+    // token take the k best keys in k arg-max rounds, and thread q owns
+    // slot q of the token's top-k.  The task that completes E_tk runs the
+    // scan itself (dynamic schedule), with no trip through the queue.
+    __device__ static uint64_t tk_key(float v, int e) {
+        uint32_t b = __float_as_uint(v + 0.0f);  // -0 -> +0: equal logits tie on the index
+        b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+        return ((uint64_t)b << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)e);
     }
+    __device__ static float tk_val(uint64_t k) {
+        const uint32_t h = (uint32_t)(k >> 32);
+        return __uint_as_float((h & 0x80000000u) ? (h & 0x7FFFFFFFu) : ~h);
+    }
+    __device__ static int tk_idx(uint64_t k) { return (int)(0xFFFFFFFFu - (uint32_t)k); }
 
-    // TK(j): tokens [16j, 16j+16).  logits = (sum of the K-chunk partials) +
-    // bias; top-k by (logit desc, index asc); softmax of the selected logits;
-    // pair counts per expert of the token's 128-token tile.  Thread (g, q)
-    // takes token g and experts 32q .. 32q+31, keeps a top-8 list of its
-    // quarter, and the q = 0 thread merges the four lists.  Loops stay
-    // rolled: this code runs once per task and must stay small in the
-    // instruction cache.  The task that completes E_tk runs the scan itself
-    // (dynamic schedule), with no trip through the queue.
-    __device__ static bool topk_task(const Params& p, Ctx& x, TaskDesc& d, int j) {
-        const int tile = j * p.tkt / p.tt;
-        const int* ev = x.ctr + (is_unfused(p) ? p.ev_rt_all : p.ev_rt + tile);
-        const int tgt = (is_unfused(p) ? p.n_tt * p.n_kc : p.n_kc) + p.bad_count;
-        if (!group_wait(x, d, ev, tgt, 220)) return false;
+    __device__ static bool route_topk(const Params& p, Ctx& x, TaskDesc& d, int j, const float* L) {
         RouteSmem sm = route_smem(x);
-        const int tg = x.tid >> 2, q = x.tid & 3;
+        const int tile = j * p.tkt / p.tt;
+        const int g = x.tid >> 3, q = x.tid & 7;
         const int t0 = j * p.tkt;
         const int ntok = min(p.tkt, p.T - t0);
-        const bool valid = tg < ntok;
-        const int t = t0 + tg;
+        const int t = t0 + g;
+        const int e0 = q * 16;
+        // experts of this thread: 16, 8 (the last group when E % 16 == 8) or none
+        const int ne = g < ntok ? max(0, min(16, p.E - e0)) : 0;
+        float l[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) l[i] = i < ne ? L[g * 132 + e0 + i] : 0.f;
         if (x.tid < 128) sm.hist[x.tid] = 0;
-        float* row = sm.L + tg * 132 + q * 33;
-        // logits of this thread's token quarter (and re-zero the accumulator)
+        uint64_t key[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) key[i] = i < ne ? tk_key(l[i], e0 + i) : 0ull;
+        // k rounds of an arg-max over the token's 8 threads: each thread's best
+        // key not taken yet, then the max over the eight by xor shuffles; the
+        // owner marks it taken (keys are unique: they hold the index).  Thread
+        // q keeps the key of round q.  A rolled loop: this code runs once per
+        // task and must stay small in the instruction cache.
+        uint32_t taken = 0;
+        uint64_t kq = 0, k0 = 0;
 #pragma unroll 1
-        for (int sub = 0; sub < 4; ++sub) {
-            const int e0 = q * 32 + sub * 8;
-            if (!valid || e0 >= p.E) break;
-            float4* src = reinterpret_cast<float4*>(p.lacc + (size_t)t * p.E + e0);
-            const float4 a0 = __ldcg(src), a1 = __ldcg(src + 1);
-            const float4 b0 = *reinterpret_cast<const float4*>(p.bias + e0);
-            const float4 b1 = *reinterpret_cast<const float4*>(p.bias + e0 + 4);
-            __stcg(src, make_float4(0.f, 0.f, 0.f, 0.f));
-            __stcg(src + 1, make_float4(0.f, 0.f, 0.f, 0.f));
-            const float4 l0 = make_float4(a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w);
-            const float4 l1 = make_float4(a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w);
-            float* r8 = row + sub * 8;
-            r8[0] = l0.x;
-            r8[1] = l0.y;
-            r8[2] = l0.z;
-            r8[3] = l0.w;
-            r8[4] = l1.x;
-            r8[5] = l1.y;
-            r8[6] = l1.z;
-            r8[7] = l1.w;
-            if (p.out_logits) {
-                float4* o = reinterpret_cast<float4*>(p.out_logits + (size_t)t * p.E + e0);
-                o[0] = l0;
-                o[1] = l1;
+        for (int s = 0; s < p.k; ++s) {
+            uint64_t best = 0;
+            int bi = 16;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const bool ok = !((taken >> i) & 1u) && key[i] > best;
+                best = ok ? key[i] : best;
+                bi = ok ? i : bi;
             }
+            uint64_t w = best;
+#pragma unroll
+            for (int m = 1; m < 8; m <<= 1) {
+                const uint64_t o = __shfl_xor_sync(0xffffffffu, w, m);
+                w = o > w ? o : w;
+            }
+            if (bi < 16 && best == w) taken |= 1u << bi;
+            k0 = s == 0 ? w : k0;
+            kq = q == s ? w : kq;
         }
-        float tv[8];
-        int ti[8];
+        const bool mine = g < ntok && q < p.k;
+        float ex = mine ? expf(tk_val(kq) - tk_val(k0)) : 0.f;
+        float z = ex;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            tv[s] = -INFINITY;
-            ti[s] = 0x7fffffff;
-        }
-        const int ne = valid ? max(0, min(32, p.E - q * 32)) : 0;
-#pragma unroll 1
-        for (int i = 0; i < ne; ++i) ins8(tv, ti, row[i], q * 32 + i);
-        exec_bar();  // every thread is done with L: reuse it for the lists
-        float* lst = sm.L + x.tid * 16;
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            lst[s] = tv[s];
-            reinterpret_cast<int*>(lst)[8 + s] = ti[s];
-        }
-        exec_bar();
-        if (q == 0 && valid) {
-#pragma unroll 1
-            for (int qq = 1; qq < 4; ++qq) {
-                const float* o = sm.L + (tg * 4 + qq) * 16;
-#pragma unroll 1
-                for (int s = 0; s < 8; ++s) ins8(tv, ti, o[s], reinterpret_cast<const int*>(o)[8 + s]);
-            }
-            float ex[8], z = 0.f;
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                ex[s] = s < p.k ? expf(tv[s] - tv[0]) : 0.f;
-                z += ex[s];
-            }
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                if (s >= p.k) break;
-                const size_t pi = (size_t)t * p.k + s;
-                const float wt = ex[s] / z;
-                p.topk[pi] = ti[s];
-                p.topw[pi] = wt;
-                if (p.out_topk) p.out_topk[pi] = ti[s];
-                if (p.out_w) p.out_w[pi] = wt;
-                atomicAdd(&sm.hist[ti[s]], 1);
-            }
+        for (int m = 1; m < 8; m <<= 1) z += __shfl_xor_sync(0xffffffffu, z, m);
+        exec_bar();  // hist zeroed
+        if (mine) {
+            const int e = tk_idx(kq);
+            const size_t pi = (size_t)t * p.k + q;
+            const float wt = ex / z;
+            p.topk[pi] = e;
+            p.topw[pi] = wt;
+            if (p.out_topk) p.out_topk[pi] = e;
+            if (p.out_w) p.out_w[pi] = wt;
+            atomicAdd(&sm.hist[e], 1);
         }
         exec_bar();
         if (x.tid < p.E && sm.hist[x.tid] > 0) atomicAdd(x.ctr + p.ev_gcnt + tile * p.E + x.tid, sm.hist[x.tid]);
@@ -514,10 +491,9 @@ struct Moe {
             const bool early = x.dynamic && n_stage_tasks(p, ttot, false) <= p.early_max;
             p.scal[1] = early;
             if (x.dynamic) {
-                // queued tasks of the run: router, top-k, group (several tiles),
-                // stage 1 and 2, combine (the scan runs inline)
-                const int total = p.n_tt * p.n_kc + p.n_tk + (p.n_tt > 1 ? p.n_tt : 0) +
-                                  ttot * (p.n_n1 + p.n_n2) + p.n_cb;
+                // queued tasks of the run: router (+ top-k), group (several
+                // tiles), stage 1 and 2, combine (the scan runs inline)
+                const int total = p.n_tk + (p.n_tt > 1 ? p.n_tt : 0) + ttot * (p.n_n1 + p.n_n2) + p.n_cb;
                 __threadfence();
                 atomicExch(x.ctr + kCtrTotal, total + 1);
             }
@@ -534,11 +510,18 @@ struct Moe {
     __device__ static void load_tile_picks(const Params& p, Ctx& x, RouteSmem& sm, int t0, int ntok) {
         for (int i = x.tid; i < 128 * 4; i += kExecThreads) sm.emask[i] = 0;
         exec_bar();
-        for (int i = x.tid; i < ntok * p.k; i += kExecThreads) {
-            const int ee = __ldcg(p.topk + (size_t)t0 * p.k + i);
-            const int tl = i / p.k;
-            sm.tk[i] = ee;
-            atomicOr(&sm.emask[ee * 4 + (tl >> 5)], 1u << (tl & 31));
+        const int tl = x.tid;  // token of the tile; its k picks are loaded together
+        if (tl < ntok) {
+            int ee[8];
+#pragma unroll
+            for (int s = 0; s < 8; ++s) ee[s] = s < p.k ? __ldcg(p.topk + (size_t)(t0 + tl) * p.k + s) : 0;
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                if (s < p.k) {
+                    sm.tk[tl * p.k + s] = ee[s];
+                    atomicOr(&sm.emask[ee[s] * 4 + (tl >> 5)], 1u << (tl & 31));
+                }
+            }
         }
         exec_bar();
     }
@@ -567,12 +550,20 @@ struct Moe {
     // tile's first grouped row per expert.  With one 128-token tile it is
     // also the grouping task (placement, then the stage tasks / E_grp).
     __device__ static bool scan_task(const Params& p, Ctx& x, TaskDesc& d) {
-        if (!group_wait(x, d, x.ctr + p.ev_tk, p.n_tk, 230)) return false;
+        if (!group_wait(x, d, x.ctr + p.ev_tk, p.n_tk + p.bad_count, 230)) return false;
         RouteSmem sm = route_smem(x);
         const int e = x.tid;
         int cnt = 0;
-        if (e < p.E)
-            for (int g = 0; g < p.n_tt; ++g) cnt += ld_relaxed(x.ctr + p.ev_gcnt + g * p.E + e);
+        // (plain L2 loads after the acquiring wait, sixteen tiles at a time)
+#pragma unroll 1
+        for (int g0 = 0; g0 < p.n_tt; g0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                v[i] = (e < p.E && g0 + i < p.n_tt) ? __ldcg(x.ctr + p.ev_gcnt + (g0 + i) * p.E + e) : 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) cnt += v[i];
+        }
         int ex;
         const int ttot = build_csr(p, x, sm, cnt, &ex);
         if (p.n_tt == 1) {
@@ -590,9 +581,16 @@ struct Moe {
         }
         if (e < p.E) {
             int run = ex;
-            for (int g = 0; g < p.n_tt; ++g) {
-                p.goff[(size_t)g * p.E + e] = run;
-                run += ld_relaxed(x.ctr + p.ev_gcnt + g * p.E + e);
+#pragma unroll 1
+            for (int g0 = 0; g0 < p.n_tt; g0 += 16) {
+                int v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = g0 + i < p.n_tt ? __ldcg(x.ctr + p.ev_gcnt + (g0 + i) * p.E + e) : 0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    if (g0 + i < p.n_tt) p.goff[(size_t)(g0 + i) * p.E + e] = run;
+                    run += v[i];
+                }
             }
         }
         const bool fired = group_finish_notify(x, d, x.ctr + p.ev_sc, 1, 1);

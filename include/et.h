@@ -97,14 +97,14 @@ typedef struct {
     int mlp_gu_tile;     /* intermediate columns per gate/up task */
     int mlp_down_tile;   /* output columns per down task */
     int mlp_kchunk;      /* K (intermediate) columns per down task */
-    int moe_tt;          /* tokens per router/top-k tile */
+    int moe_tt;          /* tokens per grouping tile (pair counts are kept per tile) */
     int moe_gt;          /* tokens per grouping task (= moe_tt) */
-    int moe_tkt;         /* tokens per top-k task */
+    int moe_tkt;         /* tokens per router task (router GEMM + top-k + softmax) */
     int moe_bm;          /* rows (token, slot pairs) per expert m-tile */
     int moe_n1_tile;     /* intermediate columns per stage-1 task */
     int moe_n2_tile;     /* output columns per stage-2 task */
-    int moe_cb;          /* tokens per combine task */
-    int moe_router_kc;   /* router K-chunks at this graph's max_T bucket */
+    int moe_cb;          /* tokens per combine task at this graph's max_T; a run whose size
+                            bucket (the power of two >= T, capped at max_T) is <= 256 uses 1 */
 } et_graph_info;
 
 /* Trace record (ET_DEBUG_TRACE): one per executed task. */
@@ -114,8 +114,7 @@ typedef struct {
     uint32_t end;     /* ticket taken after its outputs were written, before its notify */
     uint64_t t_fetch; /* %globaltimer (ns): task taken from the static list / ready queue */
     uint64_t t_ready; /* %globaltimer: input event complete */
-    uint64_t t_acc;   /* %globaltimer: tensor-core accumulator ready (GEMM tasks), end of the
-                         first phase (top-k task), else 0 */
+    uint64_t t_acc;   /* %globaltimer: tensor-core accumulator ready (GEMM tasks), else 0 */
     uint64_t t_end;   /* %globaltimer: outputs written */
 } et_trace_record;
 
@@ -126,8 +125,7 @@ typedef struct {
 #define ET_OP_MLP_GATEUP 11
 #define ET_OP_MLP_DOWN 12
 #define ET_OP_MLP_REDUCE 13
-#define ET_OP_MOE_ROUTER 20
-#define ET_OP_MOE_TOPK 21
+#define ET_OP_MOE_ROUTER 20 /* router GEMM of 16 tokens, then their top-k and softmax */
 #define ET_OP_MOE_SCAN 22
 #define ET_OP_MOE_GROUP 23
 #define ET_OP_MOE_S1 24

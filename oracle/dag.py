@@ -25,8 +25,8 @@ import numpy as np
 # include/et.h, where the record format is defined)
 OP_SK_PARTIAL, OP_SK_FINAL = 1, 2
 OP_MLP_NORM, OP_MLP_GATEUP, OP_MLP_DOWN, OP_MLP_REDUCE = 10, 11, 12, 13
-OP_MOE_ROUTER, OP_MOE_TOPK, OP_MOE_SCAN, OP_MOE_GROUP, OP_MOE_S1, OP_MOE_S2, OP_MOE_COMBINE = (
-    20, 21, 22, 23, 24, 25, 26)
+OP_MOE_ROUTER, OP_MOE_SCAN, OP_MOE_GROUP, OP_MOE_S1, OP_MOE_S2, OP_MOE_COMBINE = (
+    20, 22, 23, 24, 25, 26)
 
 
 def _cdiv(a, b):
@@ -120,15 +120,15 @@ def mlp_graph(B, hidden, inter, gu_tile, down_tile, kchunk, sched):
     return g.finish()
 
 
-def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
+def moe_graph(topk, E, tt, tkt, gt, bm, n_n1, n_n2, cb, sched):
     """MoE layer, expanded with the runtime routing `topk` [T, k]:
-      router (t, c)   --"tc->t"-->           E_rt[t]         (count = #K chunks; tt tokens)
-      E_rt[t]         -->                    topk j for the tkt-token tiles j inside tile t
-      topk j          --"j->"-->             E_tk            (count = #top-k tasks)
+      router j        --"j->"-->             E_tk            (count = #router tasks; each
+                                                             routes tkt tokens: logits,
+                                                             top-k, softmax)
       E_tk            -->                    scan
-      one router tile (T <= tt): the scan is the grouping task:
+      one grouping tile (T <= tt): the scan is the grouping task:
       scan            --> E_exp[topk[i,:]] for every token i
-      several router tiles:
+      several grouping tiles:
       scan            -->                    E_sc            (count 1)
       E_sc            --"->g"-->             group g         (gt tokens)
       group g         --> E_exp[topk[i,:]] for every token i of group g
@@ -160,15 +160,9 @@ def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
         r = rows_of[e]
         for m in range(_cdiv(len(r), bm)):
             mtiles.append((e, m, r[m * bm:(m + 1) * bm]))
-    for t in range(n_tt):
-        for c in range(n_kc):
-            task = (OP_MOE_ROUTER, t, c)
-            g.add_task(task)
-            g.produce(task, ("E_rt_all",) if unf else ("E_rt", t))
     for j in range(n_tk):
-        task = (OP_MOE_TOPK, j, 0)
+        task = (OP_MOE_ROUTER, j, 0)
         g.add_task(task)
-        g.consume(task, ("E_rt_all",) if unf else ("E_rt", (j * tkt) // tt))
         g.produce(task, ("E_tk",))
     scan = (OP_MOE_SCAN, 0, 0)
     g.add_task(scan)
