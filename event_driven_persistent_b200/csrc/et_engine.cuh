@@ -101,28 +101,44 @@ __device__ __forceinline__ void thread_push(Ctx& x, int n, Gen gen) {
     for (int i = 0; i < n; ++i) q_publish_after_fence(x.q, base + i, gen(i));
 }
 
+// Trace record of a finished task (debug; out of line, off the hot path).
+static __device__ __noinline__ void trace_task(Ctl* ctl, TraceRec* buf, int cap, uint32_t word, uint32_t start,
+                                               uint64_t t_fetch, uint64_t t_ready, uint64_t t_acc,
+                                               uint32_t end_ticket, uint64_t t_end) {
+    TraceRec r;
+    r.end = end_ticket;
+    r.t_end = t_end;
+    r.op = task_op(word);
+    r.a = task_a(word);
+    r.b = task_b(word);
+    r.sm = (int)smid();
+    r.start = start;
+    r.t_fetch = t_fetch;
+    r.t_ready = t_ready;
+    r.t_acc = t_acc;
+    trace_write(ctl, buf, cap, r);
+}
+
 // End of a task in the exec group: every thread has written its outputs.
 // Thread 0 records the trace and adds `n` to one event counter; returns (to
 // all threads) whether this notify completed the event (counter == target).
-__device__ __forceinline__ bool group_finish_notify(Ctx& x, const TaskDesc& d, int* ctr, int n, int target) {
+// With trace_if_fired false, a notify that completes the event writes no
+// trace record (the task goes on with more work and records at its end).
+__device__ __forceinline__ bool group_finish_notify(Ctx& x, const TaskDesc& d, int* ctr, int n, int target,
+                                                    bool trace_if_fired = true) {
     exec_bar();
     if (x.tid == 0) {
         int fired = 0;
-        if (x.debug & ET_DEBUG_TRACE) {
-            TraceRec r;
-            r.end = take_ticket(x.ctl);
-            r.t_end = globaltimer();
-            r.op = task_op(d.word);
-            r.a = task_a(d.word);
-            r.b = task_b(d.word);
-            r.sm = (int)smid();
-            r.start = d.start;
-            r.t_fetch = d.t_fetch;
-            r.t_ready = d.t_ready;
-            r.t_acc = d.t_acc;
-            trace_write(x.ctl, x.trace, x.trace_cap, r);
+        const bool tr = (x.debug & ET_DEBUG_TRACE) != 0;
+        uint32_t tk = 0;
+        uint64_t te = 0;
+        if (tr) {
+            tk = take_ticket(x.ctl);
+            te = globaltimer();
         }
         if (ctr) fired = notify(ctr, n) == target;
+        if (tr && (trace_if_fired || !fired))
+            trace_task(x.ctl, x.trace, x.trace_cap, d.word, d.start, d.t_fetch, d.t_ready, d.t_acc, tk, te);
         x.sc->bcast[1] = fired;
     }
     exec_bar();

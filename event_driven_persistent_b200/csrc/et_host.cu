@@ -324,7 +324,7 @@ et_status build_mlp(et_graph* g) {
 
 // ----------------------------------------------------------------- MoE ----
 struct MoeShape {
-    int n_tt, n_tk, cb, n_cb, f_max;
+    int n_tt, n_tk, n_kc, cb, n_cb, f_max;
 };
 
 // Tokens per combine task: one while the layer is small (the combine is the
@@ -337,6 +337,11 @@ MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
     MoeShape m;
     m.n_tt = cdiv(T, p.tt);
     m.n_tk = cdiv(T, p.tkt);
+    // router K split: up to 8 chunks while the (token block, chunk) tasks fit
+    // in a quarter of the SMs, so that a small batch streams Wr on many SMs
+    int kc = 1;
+    while (kc < 8 && m.n_tk * kc * 2 * 4 <= g->n_ctas && (p.hidden / (kc * 2)) % kTileK == 0) kc *= 2;
+    m.n_kc = kc;
     m.cb = moe_cb_for(T);
     m.n_cb = cdiv(T, m.cb);
     const int pairs = p.k * T;
@@ -375,6 +380,8 @@ et_status build_moe(et_graph* g) {
     if (mx.f_max > 0xFFFF || mx.n_tt > 0xFFFF || p.n_n1 > 0x3FF || p.n_n2 > 0x3FF) return ET_ERR_UNSUPPORTED;
     int ev = kCtrFirstEvent;
     p.ev_tk = ev++;
+    p.ev_rt = ev;
+    ev += mx.n_tk;
     p.ev_sc = ev++;
     p.ev_grp = ev++;
     p.ev_s1_all = ev++;
@@ -389,8 +396,9 @@ et_status build_moe(et_graph* g) {
     p.ev_gcnt = ev;
     ev += mx.n_tt * p.E;
     g->n_ctr = ev;
-    g->qcap = mx.n_tk + mx.n_tt + 1 + mx.f_max * (p.n_n1 + p.n_n2) + n_cb_max + g->n_ctas * d.fetch_batch + 64;
+    g->qcap = mx.n_tk * 8 + mx.n_tt + 1 + mx.f_max * (p.n_n1 + p.n_n2) + n_cb_max + g->n_ctas * d.fetch_batch + 64;
     const size_t pairs = (size_t)p.maxT * p.k;
+    ET_TRY(galloc(g, &p.lacc, (size_t)p.maxT * p.E));
     ET_TRY(galloc(g, &p.topk, pairs));
     ET_TRY(galloc(g, &p.topw, pairs));
     ET_TRY(galloc(g, &p.goff, (size_t)mx.n_tt * p.E));
@@ -410,8 +418,9 @@ et_status build_moe(et_graph* g) {
     const float c_s1 = 2.f * p.n1_tile * p.hidden * 2 / 1024.f, c_s2 = (float)p.n2_tile * p.inter * 2 / 1024.f;
     return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
         MoeShape m = moe_shape(g, p, Tb);
-        const float c_rt = (float)p.E * p.hidden * 2 / 1024.f;
-        for (int j = 0; j < m.n_tk; ++j) s.push_back({tw(ET_OP_MOE_ROUTER, j, 0), c_rt});
+        const float c_rt = (float)p.E * p.hidden * 2 / m.n_kc / 1024.f;
+        for (int j = 0; j < m.n_tk; ++j)
+            for (int c = 0; c < m.n_kc; ++c) s.push_back({tw(ET_OP_MOE_ROUTER, j, c), c_rt});
         s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 8.f});
         if (m.n_tt > 1)
             for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_GROUP, t, 0), 8.f});
@@ -594,11 +603,12 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
     const MoeShape mt = moe_shape(g, p, T);
     p.n_tt = mt.n_tt;
     p.n_tk = mt.n_tk;
-    p.cb = mb.cb;  // the size bucket fixes the combine block (static lists and dynamic alike)
+    p.n_kc = mb.n_kc;  // the size bucket fixes the router split and the combine block
+    p.cb = mb.cb;      // (static lists and dynamic alike)
     p.n_cb = cdiv(T, p.cb);
     p.f_max = mb.f_max;
     ET_TRY(pre_run(g, s));
-    RunArgs ra = run_args(g, T, p.n_tk, 0);
+    RunArgs ra = run_args(g, T, p.n_tk * p.n_kc, 0);
     ET_CU(launch_moe(p, ra, g->n_ctas, s));
     return ET_OK;
 }
@@ -616,6 +626,7 @@ et_status et_sync_status(et_graph* g, void* stream) {
     ET_CU(cudaMemset(g->ctr[1], 0, g->n_ctr * sizeof(int)));
     if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc) {
         ET_CU(cudaMemset(g->moe.Yacc, 0, (size_t)g->moe.maxT * g->moe.hidden * sizeof(float)));
+        ET_CU(cudaMemset(g->moe.lacc, 0, (size_t)g->moe.maxT * g->moe.E * sizeof(float)));
     }
     ET_CU(cudaDeviceSynchronize());
     // keep the diagnostic words readable through et_get_diag

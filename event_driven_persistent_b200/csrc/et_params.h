@@ -68,6 +68,9 @@ struct MoeParams {
     int32_t* out_perm;
     float* out_logits;
     // workspace
+    float* lacc;        // [maxT, E] router logits without bias when the router's K is split:
+                        // the chunk tasks add their partials (fp32 red.add), the last one
+                        // reads and re-zeroes them, so it is zero between runs
     int32_t* topk;      // [maxT, k]
     float* topw;        // [maxT, k]
     int32_t* goff;      // [n_tt, E] first grouped row of tile g's pairs of expert e
@@ -81,11 +84,11 @@ struct MoeParams {
     uint16_t* Hm;       // [maxT*k, I] stage-1 output, grouped order
     float* Yacc;        // [maxT, H] fp32 combine accumulator (kept zero between runs)
     int T, hidden, inter, E, k, maxT;
-    int tt, n_tt, tkt, n_tk, bm, n1_tile, n_n1, n2_tile, n_n2, cb, n_cb;
+    int tt, n_tt, n_kc, tkt, n_tk, bm, n1_tile, n_n1, n2_tile, n_n2, cb, n_cb;
     int f_max;          // static: m-tile slots of this bucket
     int early_max;      // dynamic: push stage-2 tasks with stage 1 when #stage-1 tasks <= this
     // events
-    int ev_tk, ev_sc, ev_grp, ev_exp, ev_s1, ev_cb, ev_s1_all, ev_s2_all;
+    int ev_rt, ev_tk, ev_sc, ev_grp, ev_exp, ev_s1, ev_cb, ev_s1_all, ev_s2_all;
     int ev_gcnt;        // counter-set block [n_tt, E]: pairs of 128-token tile g per expert
     int sched;          // et_sched
     int bad_count;

@@ -17,8 +17,10 @@
 //     weights stream while stage 1 computes.
 //
 // Task graph (counts in brackets; dynamic schedule; tiles of 128 tokens):
-//   RT(j)     16 tokens: router GEMM (full K, tensor cores), + bias, top-k and
-//             softmax in the epilogue, pair counts per 128-token tile -> E_tk [#router tasks]
+//   RT(j, c)  16 tokens, K chunk c of n_kc: router GEMM (tensor cores); with n_kc > 1
+//             the chunk partials are added at L2 (fp32 red.add) -> E_rt[j] [n_kc];
+//             the task that completes E_rt[j] (or the only one) adds the bias and
+//             takes top-k and softmax, pair counts per 128-token tile -> E_tk [#blocks]
 //   SC        expert counts, CSR (indptr, m-tile indptr), tile offsets -> E_sc [1]
 //             (run by the task that completes E_tk; with T <= 128 it is also the
 //             grouping task -> E_exp[topk[i,:]])
@@ -70,7 +72,9 @@ struct Moe {
 
     __device__ static bool is_unfused(const Params& p) { return p.sched == ET_SCHED_UNFUSED; }
 
-    __device__ static uint32_t fetch_init(const Params& p, int idx) { return task_word(ET_OP_MOE_ROUTER, idx, 0); }
+    __device__ static uint32_t fetch_init(const Params& p, int idx) {
+        return task_word(ET_OP_MOE_ROUTER, idx / p.n_kc, idx % p.n_kc);
+    }
 
     // m-tile f -> (expert, first grouped row, rows); needs the scan's outputs
     __device__ static void mtile(const Params& p, int f, int& e, int& row0, int& cnt) {
@@ -94,8 +98,8 @@ struct Moe {
             d.b_map = MOE_MAP_X;
             d.b_row0 = a * p.tkt;
             d.n = 16;
-            d.nk = p.hidden / kTileK;
-            d.k0 = 0;
+            d.nk = p.hidden / p.n_kc / kTileK;
+            d.k0 = b * (p.hidden / p.n_kc);
         } else if (op == ET_OP_MOE_GROUP) {
             d.valid = p.n_tt > 1 && a < p.n_tt;  // one tile: the scan task groups
         } else if (op == ET_OP_MOE_COMBINE) {
@@ -186,6 +190,24 @@ struct Moe {
             float v[16];
             acc_load16(taddr, 0, v);
             acc_release(acc_empty);
+            if (p.n_kc > 1) {
+                // K split: add this chunk's partials into lacc at L2; the chunk
+                // task that completes E_rt[a] reads the sums and re-zeroes lacc
+                float* acc = p.lacc + (size_t)t0 * p.E + r;
+                if (r < p.E) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (c < ntok) red_add(acc + (size_t)c * p.E, v[c]);
+                }
+                if (!group_finish_notify(x, d, x.ctr + p.ev_rt + a, 1, p.n_kc, false)) return true;
+                if (r < p.E) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) v[c] = c < ntok ? __ldcg(acc + (size_t)c * p.E) : 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        if (c < ntok) __stcg(acc + (size_t)c * p.E, 0.f);
+                }
+            }
             if (r < p.E) {
                 const float bb = p.bias[r];
 #pragma unroll
@@ -491,9 +513,9 @@ struct Moe {
             const bool early = x.dynamic && n_stage_tasks(p, ttot, false) <= p.early_max;
             p.scal[1] = early;
             if (x.dynamic) {
-                // queued tasks of the run: router (+ top-k), group (several
+                // queued tasks of the run: router chunks, group (several
                 // tiles), stage 1 and 2, combine (the scan runs inline)
-                const int total = p.n_tk + (p.n_tt > 1 ? p.n_tt : 0) + ttot * (p.n_n1 + p.n_n2) + p.n_cb;
+                const int total = p.n_tk * p.n_kc + (p.n_tt > 1 ? p.n_tt : 0) + ttot * (p.n_n1 + p.n_n2) + p.n_cb;
                 __threadfence();
                 atomicExch(x.ctr + kCtrTotal, total + 1);
             }

@@ -120,11 +120,13 @@ def mlp_graph(B, hidden, inter, gu_tile, down_tile, kchunk, sched):
     return g.finish()
 
 
-def moe_graph(topk, E, tt, tkt, gt, bm, n_n1, n_n2, cb, sched):
+def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
     """MoE layer, expanded with the runtime routing `topk` [T, k]:
-      router j        --"j->"-->             E_tk            (count = #router tasks; each
-                                                             routes tkt tokens: logits,
-                                                             top-k, softmax)
+      router (j, c)   --"jc->j"-->           E_rt[j]         (count = #K chunks n_kc; tkt
+                                                             tokens per block j)
+      the chunk task completing E_rt[j] routes block j (logits, top-k,
+      softmax), so every router (j, c) precedes:
+      router (j, *)   --"j->"-->             E_tk            (count = #token blocks)
       E_tk            -->                    scan
       one grouping tile (T <= tt): the scan is the grouping task:
       scan            --> E_exp[topk[i,:]] for every token i
@@ -161,9 +163,10 @@ def moe_graph(topk, E, tt, tkt, gt, bm, n_n1, n_n2, cb, sched):
         for m in range(_cdiv(len(r), bm)):
             mtiles.append((e, m, r[m * bm:(m + 1) * bm]))
     for j in range(n_tk):
-        task = (OP_MOE_ROUTER, j, 0)
-        g.add_task(task)
-        g.produce(task, ("E_tk",))
+        for c in range(n_kc):
+            task = (OP_MOE_ROUTER, j, c)
+            g.add_task(task)
+            g.produce(task, ("E_tk",))
     scan = (OP_MOE_SCAN, 0, 0)
     g.add_task(scan)
     g.consume(scan, ("E_tk",))

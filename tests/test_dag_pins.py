@@ -30,7 +30,7 @@ def test_splitk_unfused_is_a_barrier():
 def test_moe_tiny_by_hand():
     # T=2 tokens, k=2, E=3 experts, one token tile, one router task per token, one group, bm=1
     topk = np.array([[2, 0], [0, 1]])
-    g, mtiles = dag.moe_graph(topk, E=3, tt=2, tkt=1, gt=2, bm=1, n_n1=1, n_n2=1, cb=1, sched="dynamic")
+    g, mtiles = dag.moe_graph(topk, E=3, tt=2, n_kc=1, tkt=1, gt=2, bm=1, n_n1=1, n_n2=1, cb=1, sched="dynamic")
     # grouping: expert 0 <- (0,1),(1,0); expert 1 <- (1,1); expert 2 <- (0,0); bm=1 -> 4 m-tiles
     assert [(e, m, rows) for (e, m, rows) in mtiles] == [
         (0, 0, [(0, 1)]), (0, 1, [(1, 0)]), (1, 0, [(1, 1)]), (2, 0, [(0, 0)])]
@@ -88,12 +88,13 @@ def test_checker_accepts_valid_and_catches_planted_mistakes():
 def test_moe_two_tiles_by_hand():
     # T=3 tokens in tiles of 2: router -> scan -> group per tile; top-1 of 2 experts
     topk = np.array([[1], [0], [1]])
-    g, mtiles = dag.moe_graph(topk, E=2, tt=2, tkt=2, gt=2, bm=2, n_n1=1, n_n2=1, cb=2, sched="dynamic")
+    g, mtiles = dag.moe_graph(topk, E=2, tt=2, n_kc=2, tkt=2, gt=2, bm=2, n_n1=1, n_n2=1, cb=2, sched="dynamic")
     R, SC, GR, S1, S2, CB = (dag.OP_MOE_ROUTER, dag.OP_MOE_SCAN, dag.OP_MOE_GROUP,
                              dag.OP_MOE_S1, dag.OP_MOE_S2, dag.OP_MOE_COMBINE)
     # expert 0 <- token 1 (m-tile 0); expert 1 <- tokens 0, 2 (m-tile 1)
     assert [(e, rows) for (e, m, rows) in mtiles] == [(0, [(1, 0)]), (1, [(0, 0), (2, 0)])]
-    want = {((R, j, 0), (SC, 0, 0)) for j in range(2)}
+    # two K chunks per router block: every chunk task precedes the scan
+    want = {((R, j, c), (SC, 0, 0)) for j in range(2) for c in range(2)}
     want |= {((SC, 0, 0), (GR, q, 0)) for q in range(2)}
     # group 0 (tokens 0,1) touches experts 1 and 0; group 1 (token 2) touches expert 1
     want |= {((GR, 0, 0), (S1, 0, 0)), ((GR, 0, 0), (S1, 1, 0)), ((GR, 1, 0), (S1, 1, 0))}

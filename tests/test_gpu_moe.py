@@ -114,23 +114,6 @@ def test_moe_e24_top8(sched, T):
         et.et_destroy_graph(g)
 
 
-def test_moe_logits_deterministic(small_inputs):
-    """The router sums in a fixed order: logits, top-k and weights are
-    identical bit for bit from run to run."""
-    d = small_inputs
-    g = et.et_build_graph(et.ET_GRAPH_MOE, "dynamic", 512, **SMALL)
-    try:
-        st, a = run_moe(g, d, 300, 4, 16)
-        assert st == 0
-        st, b = run_moe(g, d, 300, 4, 16)
-        assert st == 0
-        assert np.array_equal(a["logits"].view(np.uint32), b["logits"].view(np.uint32))
-        assert np.array_equal(a["topk"], b["topk"])
-        assert np.array_equal(a["w"].view(np.uint32), b["w"].view(np.uint32))
-    finally:
-        et.et_destroy_graph(g)
-
-
 @pytest.mark.parametrize("sched", ["static", "dynamic"])
 def test_moe_symbolic_T_repeated_runs(small_inputs, sched):
     """One graph, one binary, T changing from run to run (no rebuild)."""
@@ -157,7 +140,10 @@ def test_moe_dependency_order(small_inputs, sched, T):
         st, out = run_moe(g, d, T, 4, 16)
         assert st == 0
         info = et.et_get_info(g)
-        graph, _ = dag.moe_graph(out["topk"], 16, info["moe_tt"], info["moe_tkt"], info["moe_gt"], info["moe_bm"],
+        # the router split of a run is fixed by its size bucket; read it from the trace
+        rt = [r for r in et.et_get_trace(g) if r[0] == dag.OP_MOE_ROUTER]
+        n_kc = max(r[2] for r in rt) + 1
+        graph, _ = dag.moe_graph(out["topk"], 16, info["moe_tt"], n_kc, info["moe_tkt"], info["moe_gt"], info["moe_bm"],
                                  128 // info["moe_n1_tile"], 256 // info["moe_n2_tile"], info["moe_cb"], sched)
         errs = dag.check_trace(graph, et.et_get_trace(g))
         assert errs == [], errs[:5]
