@@ -405,7 +405,7 @@ et_status build_moe(et_graph* g) {
     ET_TRY(galloc(g, &p.counts, (size_t)p.E));
     ET_TRY(galloc(g, &p.indptr, (size_t)p.E + 1));
     ET_TRY(galloc(g, &p.tindptr, (size_t)p.E + 1));
-    ET_TRY(galloc(g, &p.mt_expert, (size_t)mx.f_max));
+    ET_TRY(galloc(g, &p.mt_desc, (size_t)mx.f_max));
     ET_TRY(galloc(g, &p.perm, pairs));
     ET_TRY(galloc(g, &p.pos, pairs));
     ET_TRY(galloc(g, &p.scal, 8));

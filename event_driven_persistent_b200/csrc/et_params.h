@@ -77,7 +77,7 @@ struct MoeParams {
     int32_t* counts;    // [E]
     int32_t* indptr;    // [E+1]
     int32_t* tindptr;   // [E+1] m-tile CSR
-    int32_t* mt_expert; // [F_max] expert of flat m-tile f
+    int4* mt_desc;      // [F_max] flat m-tile f: (expert, first grouped row, rows, 0)
     int32_t* perm;      // [maxT*k]
     int32_t* pos;       // [maxT*k]
     int32_t* scal;      // [8]: 0 = total m-tiles, 1 = stage-2 tasks were pushed early

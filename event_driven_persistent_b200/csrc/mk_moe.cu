@@ -76,12 +76,13 @@ struct Moe {
         return task_word(ET_OP_MOE_ROUTER, idx / p.n_kc, idx % p.n_kc);
     }
 
-    // m-tile f -> (expert, first grouped row, rows); needs the scan's outputs
+    // m-tile f -> (expert, first grouped row, rows): one 16-byte load of the
+    // descriptor the scan wrote
     __device__ static void mtile(const Params& p, int f, int& e, int& row0, int& cnt) {
-        e = p.mt_expert[f];
-        const int mt = f - p.tindptr[e];
-        row0 = p.indptr[e] + mt * p.bm;
-        cnt = min(p.bm, p.counts[e] - mt * p.bm);
+        const int4 m = p.mt_desc[f];
+        e = m.x;
+        row0 = m.y;
+        cnt = m.z;
     }
 
     __device__ static bool derive(const Params& p, Ctx& x, TaskDesc& d) {
@@ -484,6 +485,13 @@ struct Moe {
         return true;
     }
 
+    // Dynamic schedule: the run's queued-task total (CTAs whose next queue
+    // slot lies past it stop).  Published after the scan's own pushes, so it
+    // stays off the path to the first stage tasks.
+    __device__ static void publish_total(Ctx& x, const RouteSmem& sm) {
+        if (x.tid == 0) atomicExch(x.ctr + kCtrTotal, sm.misc[6] + 1);
+    }
+
     __device__ static int tile_count(const RouteSmem& sm, int e) {
         return __popc(sm.emask[e * 4]) + __popc(sm.emask[e * 4 + 1]) + __popc(sm.emask[e * 4 + 2]) +
                __popc(sm.emask[e * 4 + 3]);
@@ -503,7 +511,7 @@ struct Moe {
             p.indptr[e] = ex;
             p.tindptr[e] = tex;
             if (p.out_indptr) p.out_indptr[e] = ex;
-            for (int f = tex; f < tex + nt; ++f) p.mt_expert[f] = e;
+            for (int m = 0; m < nt; ++m) p.mt_desc[tex + m] = make_int4(e, ex + m * p.bm, min(p.bm, cnt - m * p.bm), 0);
         }
         if (x.tid == 0) {
             p.indptr[p.E] = tot;
@@ -512,13 +520,10 @@ struct Moe {
             p.scal[0] = ttot;
             const bool early = x.dynamic && n_stage_tasks(p, ttot, false) <= p.early_max;
             p.scal[1] = early;
-            if (x.dynamic) {
-                // queued tasks of the run: router chunks, group (several
-                // tiles), stage 1 and 2, combine (the scan runs inline)
-                const int total = p.n_tk * p.n_kc + (p.n_tt > 1 ? p.n_tt : 0) + ttot * (p.n_n1 + p.n_n2) + p.n_cb;
-                __threadfence();
-                atomicExch(x.ctr + kCtrTotal, total + 1);
-            }
+            // queued tasks of the run: router chunks, group (several tiles),
+            // stage 1 and 2, combine (the scan runs inline); published once
+            // the scan has queued its successors (publish_total)
+            sm.misc[6] = p.n_tk * p.n_kc + (p.n_tt > 1 ? p.n_tt : 0) + ttot * (p.n_n1 + p.n_n2) + p.n_cb;
             sm.misc[4] = ttot;
             sm.misc[5] = early;
         }
@@ -599,6 +604,7 @@ struct Moe {
             group_finish_notify(x, d, nullptr, 0, 0);
             const bool early = sm.misc[5] != 0;
             group_push(x, n_stage_tasks(p, ttot, early), [&](int i) { return stage_task(p, 0, ttot, i); });
+            publish_total(x, sm);
             return true;
         }
         if (e < p.E) {
@@ -616,7 +622,10 @@ struct Moe {
             }
         }
         const bool fired = group_finish_notify(x, d, x.ctr + p.ev_sc, 1, 1);
-        if (fired && x.dynamic) group_push(x, p.n_tt, [&](int g) { return task_word(ET_OP_MOE_GROUP, g, 0); });
+        if (fired && x.dynamic) {
+            group_push(x, p.n_tt, [&](int g) { return task_word(ET_OP_MOE_GROUP, g, 0); });
+            publish_total(x, sm);
+        }
         return true;
     }
 
