@@ -518,7 +518,11 @@ struct Moe {
             p.tindptr[p.E] = ttot;
             if (p.out_indptr) p.out_indptr[p.E] = tot;
             p.scal[0] = ttot;
-            const bool early = x.dynamic && n_stage_tasks(p, ttot, false) <= p.early_max;
+            // early push: with one grouping tile the scan queues every stage-1
+            // task before any stage-2 task, so a stage-2 task never holds an
+            // SM while stage-1 work waits behind it; with several tiles the
+            // experts' batches interleave and it only pays when stage 1 is small
+            const bool early = x.dynamic && (p.n_tt == 1 || n_stage_tasks(p, ttot, false) <= p.early_max);
             p.scal[1] = early;
             // queued tasks of the run: router chunks, group (several tiles),
             // stage 1 and 2, combine (the scan runs inline); published once

@@ -99,7 +99,7 @@ typedef struct {
     int mlp_kchunk;      /* K (intermediate) columns per down task */
     int moe_tt;          /* tokens per grouping tile (pair counts are kept per tile) */
     int moe_gt;          /* tokens per grouping task (= moe_tt) */
-    int moe_tkt;         /* tokens per router task (router GEMM + top-k + softmax) */
+    int moe_tkt;         /* tokens per router block (router GEMM, then top-k + softmax) */
     int moe_bm;          /* rows (token, slot pairs) per expert m-tile */
     int moe_n1_tile;     /* intermediate columns per stage-1 task */
     int moe_n2_tile;     /* output columns per stage-2 task */
@@ -125,7 +125,8 @@ typedef struct {
 #define ET_OP_MLP_GATEUP 11
 #define ET_OP_MLP_DOWN 12
 #define ET_OP_MLP_REDUCE 13
-#define ET_OP_MOE_ROUTER 20 /* router GEMM of 16 tokens, then their top-k and softmax */
+#define ET_OP_MOE_ROUTER 20 /* a = 16-token block, b = K chunk (up to 8 at small T); the chunk
+                               that completes the block also takes its top-k and softmax */
 #define ET_OP_MOE_SCAN 22
 #define ET_OP_MOE_GROUP 23
 #define ET_OP_MOE_S1 24
