@@ -143,7 +143,7 @@ def gpu_arm(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     T, H, E, k = args.T, 2048, 128, 8
-    d = W.moe_inputs(T, zipf_s=args.zipf)
+    d = _layer_inputs(T, args.zipf)
 
     def to_dev(a):
         a = np.ascontiguousarray(a)
@@ -236,13 +236,24 @@ def gpu_arm(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------ CPU oracle --
+_INPUTS = {}
+
+
+def _layer_inputs(T, zipf):
+    """The seeded layer inputs, generated once per process (generation is
+    not part of any timed region)."""
+    if (T, zipf) not in _INPUTS:
+        _INPUTS[(T, zipf)] = W.moe_inputs(T, zipf_s=zipf)
+    return _INPUTS[(T, zipf)]
+
+
 def cpu_oracle(args, budget_s=15.0):
     """The oracle as it stands (single thread) on a bounded token sample of
     the same layer: per-token evaluation (router, top-8, eight experts,
     combine).  The layer time is the per-token time x T."""
     import oracle
     T = args.T
-    d = W.moe_inputs(T, zipf_s=args.zipf)
+    d = _layer_inputs(T, args.zipf)
     ntok, el = 0, 0.0
     t0 = time.perf_counter()
     while ntok < T and time.perf_counter() - t0 < budget_s:
