@@ -235,6 +235,65 @@ def gpu_arm(args, rank, world, local_rank):
     }
 
 
+# ------------------------------------------- other workloads (one GPU) --
+MLP_BYTES = 2 * (2 * 14336 * 4096 + 4096 * 14336)  # Wgu + Wd, bf16
+
+
+def other_arm(args):
+    """--workload mlp (decode MLP, static schedule, batch --B) or splitk
+    (2048 x 128 fp32, static): device time of one megakernel launch with
+    the L2 flushed before it, and the achieved algorithmic HBM GB/s."""
+    import torch
+    import event_driven_persistent_b200 as et
+    dev = torch.device("cuda", 0)
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+
+    if args.workload == "mlp":
+        B = args.B
+        d = W.mlp_inputs(B)
+        t = {n: to_dev(d[n]) for n in ("X", "gamma", "Wgu", "Wd")}
+        Y = torch.empty((B, 4096), dtype=torch.int16, device=dev)
+        g = et.et_build_graph(et.ET_GRAPH_MLP, args.sched, 64)
+        run = lambda: et.et_run_mlp(g, B, t["X"], t["gamma"], t["Wgu"], t["Wd"], Y)
+        nbytes = MLP_BYTES + 8192 + 16384 * B
+        workload = "decode MLP B=%d, hidden 4096, SwiGLU 14336, %s schedule" % (B, args.sched)
+    else:
+        A = to_dev(W.splitk_inputs(2048))
+        Bp = torch.zeros((2048, 4), device=dev)
+        C = torch.zeros((2048,), device=dev)
+        g = et.et_build_graph(et.ET_GRAPH_SPLITK, args.sched, 2048)
+        run = lambda: et.et_run_splitk(g, A, 2048, Bp, C)
+        nbytes = 2048 * 128 * 4 + 2048 * 5 * 4
+        workload = "split-K 2048 x 128 fp32, chunks of 32, %s schedule" % args.sched
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        run()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    if et.et_sync_status(g) != 0:
+        raise RuntimeError("run reported a device error")
+    et.et_destroy_graph(g)
+    ms = sum(times) / len(times)
+    hbm, _, src = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": workload, "latency_us": round(ms * 1e3, 2), "value": round(gbs, 1), "unit": "GB/s",
+            "steps": args.steps, "warmup": args.warmup, "bytes_per_launch": nbytes,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_source": src}}
+
+
 # ------------------------------------------------------------ CPU oracle --
 _INPUTS = {}
 
@@ -281,6 +340,9 @@ def main():
     ap.add_argument("--zipf", type=float, default=1.2)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="moe", choices=["moe", "mlp", "splitk"],
+                    help="moe (the benchmark line); mlp or splitk print a kernel timing line")
+    ap.add_argument("--B", type=int, default=1, help="decode MLP batch (--workload mlp)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -288,6 +350,12 @@ def main():
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.workload != "moe":
+        if args.sched == "dynamic" and "--sched" not in sys.argv:
+            args.sched = "static"
+        print(json.dumps(other_arm(args)))
+        return
 
     if args.impl == "reference":
         if rank != 0:
