@@ -13,8 +13,13 @@ the device time of a step (CUDA events on the launch stream, max over
 ranks).  The L2 is flushed before every step, outside the timed events.
 Several GPUs run independent replicas (the layer does not shard here).
 
---impl reference times the CPU oracle (plain C, fp64) on this host, on a
-bounded sample of the same workload, and prints the same line with
+The line also carries a driver-timed `sweep` (T in {1, 16, 128, 1024, 4096}
+x static / dynamic / unfused schedules, Zipf 1.2, same graph and binary) and
+the CPU oracle timed on this host's cores (`cpu_baseline`: the whole layer,
+single thread and all threads, median of 3).
+
+--impl reference times the CPU oracle (plain C, fp64, all host threads) on
+the whole layer, one layer per step, and prints the same line with
 "impl": "reference".
 """
 import argparse
@@ -165,6 +170,7 @@ def gpu_arm(args, rank, world, local_rank):
         raise RuntimeError("MoE run reported a device error")
     nbytes, touched = algorithmic_bytes(topk.cpu().numpy(), T)
 
+    clk = ClockSampler(local_rank).__enter__()  # sampled over the timed region, the sweep and e2e
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -172,21 +178,21 @@ def gpu_arm(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    with ClockSampler(local_rank) as clk:
-        torch.cuda.synchronize(dev)
-        for i in range(args.steps):
-            flush.zero_()
-            evs[i][0].record(stream)
-            step()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     st = et.et_sync_status(g, stream)
     if st != 0:
         raise RuntimeError("MoE run reported a device error: %s" % et.et_status_str(st))
     times = [a.elapsed_time(b) for a, b in evs]  # ms
-    ms = sum(times) / len(times)
+    ms = statistics.median(times)
+    sweep = run_sweep(args, et, g, t, dev, stream, flush) if (args.sweep and world == 1) else None
 
     # end to end through the C ABI with host buffers: H2D of X, the layer, D2H of Y
     Xh = torch.from_numpy(np.ascontiguousarray(d["X"]).view(np.int16)).pin_memory()
@@ -204,7 +210,8 @@ def gpu_arm(args, rank, world, local_rank):
         b.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e = sum(e2e_ms) / len(e2e_ms)
+    e2e = statistics.median(e2e_ms)
+    clk.__exit__()
 
     ms, e2e, tot_bytes = combine_ranks(ms, e2e, nbytes, world, dev)
     et.et_destroy_graph(g)
@@ -217,6 +224,7 @@ def gpu_arm(args, rank, world, local_rank):
         "metric": METRIC, "value": round(tot_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
         "latency_us": round(ms * 1e3, 2), "latency_us_p10_p90": [round(float(np.percentile(times, 10)) * 1e3, 2),
                                                                  round(float(np.percentile(times, 90)) * 1e3, 2)],
+        "latency_us_mean": round(float(np.mean(times)) * 1e3, 2), "timing": "median of the timed steps",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "MoE layer T=%d, hidden 2048, 128 experts top-8, SwiGLU 768, Zipf s=%g bias, "
@@ -232,7 +240,55 @@ def gpu_arm(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2)},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
+        "sweep": sweep,
     }
+
+
+def run_sweep(args, et, g_dyn, t, dev, stream, flush):
+    """Device time of the layer over the token range and the three schedules
+    (same binary; one graph per schedule, max_T 4096), Zipf s = 1.2: median
+    of `sweep_steps` launches, L2 flushed before each."""
+    import torch
+    hbm, tc, _ = load_peaks()
+    graphs = {"dynamic": g_dyn}
+    for s in ("static", "unfused"):
+        graphs[s] = et.et_build_graph(et.ET_GRAPH_MOE, s, max(4096, args.max_T), device=dev.index)
+    out = []
+    try:
+        for T in (1, 16, 128, 1024, 4096):
+            x = W.moe_inputs(T, weights=False)["X"]   # the weights and bias are the benchmark's own
+            X = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(dev)
+            Y = torch.empty((T, 2048), dtype=torch.int16, device=dev)
+            topk = torch.empty((T, 8), dtype=torch.int32, device=dev)
+            row = {"T": T}
+            for s, g in graphs.items():
+                et.et_run_moe(g, T, X, t["Wr"], t["bias"], t["W1"], t["W2"], Y, topk, stream=stream)
+                if et.et_sync_status(g, stream) != 0:
+                    raise RuntimeError("sweep run reported a device error")
+                nbytes, touched = algorithmic_bytes(topk.cpu().numpy(), T)
+                ts = []
+                for i in range(3 + args.sweep_steps):
+                    flush.zero_()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    et.et_run_moe(g, T, X, t["Wr"], t["bias"], t["W1"], t["W2"], Y, stream=stream)
+                    b.record(stream)
+                    b.synchronize()
+                    if i >= 3:
+                        ts.append(a.elapsed_time(b))
+                if et.et_sync_status(g, stream) != 0:
+                    raise RuntimeError("sweep run reported a device error")
+                ms = statistics.median(ts)
+                row[s] = {"us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                          "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4),
+                          "tensor_frac": round(moe_flops(T) / (ms * 1e-3) / (tc * 1e12), 4) if tc else None}
+                row["experts_touched"] = touched
+            out.append(row)
+    finally:
+        for s in ("static", "unfused"):
+            et.et_destroy_graph(graphs[s])
+    return {"zipf_s": args.zipf, "steps_per_point": args.sweep_steps, "timing": "median, L2 flushed before each launch",
+            "points": out}
 
 
 # ------------------------------------------- other workloads (one GPU) --
@@ -306,27 +362,80 @@ def _layer_inputs(T, zipf):
     return _INPUTS[(T, zipf)]
 
 
-def cpu_oracle(args, budget_s=15.0):
-    """The oracle as it stands (single thread) on a bounded token sample of
-    the same layer: per-token evaluation (router, top-8, eight experts,
-    combine).  The layer time is the per-token time x T."""
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def oracle_layer_seconds(T, zipf, threads):
+    """One whole MoE layer through the oracle (router logits, top-8 +
+    softmax, grouping, both grouped GEMMs per routed pair, combine) on
+    `threads` host threads; returns (seconds, algorithmic bytes)."""
     import oracle
-    T = args.T
-    d = _layer_inputs(T, args.zipf)
-    ntok, el = 0, 0.0
+    d = _layer_inputs(T, zipf)
+    oracle.set_threads(threads)
     t0 = time.perf_counter()
-    while ntok < T and time.perf_counter() - t0 < budget_s:
-        oracle.moe_per_token(d["X"], d["Wr"], d["bias"], d["W1"], d["W2"], [ntok], 8)
-        ntok += 1
+    out = oracle.moe(d["X"], d["Wr"], d["bias"], d["W1"], d["W2"], 8)
     el = time.perf_counter() - t0
-    logits = oracle.router_logits(d["X"], d["Wr"], d["bias"])
-    tk, _ = oracle.topk_softmax(logits, 8)
-    nbytes, _ = algorithmic_bytes(tk, T)
-    layer_s = el / ntok * T
-    return {"value": round(nbytes / layer_s / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "%d of %d tokens evaluated per token (router, top-8, 8 experts, combine) in %.1f s; "
-                      "layer time = per-token time x T" % (ntok, T, el),
-            "latency_us": round(layer_s * 1e6, 1)}
+    nbytes, _ = algorithmic_bytes(out["topk"], T)
+    return el, nbytes
+
+
+def cpu_oracle(args, reps=3):
+    """The oracle as it stands, timed on this host: the whole layer at the
+    benchmark's T, median of `reps` runs on one thread and on every thread."""
+    import oracle
+    n_all = oracle.max_threads()
+    res = {}
+    for threads in (1, n_all):
+        ts = []
+        for _ in range(reps):
+            el, nbytes = oracle_layer_seconds(args.T, args.zipf, threads)
+            ts.append(el)
+        res[threads] = (statistics.median(ts), nbytes)
+    (s_all, nbytes), (s_one, _) = res[n_all], res[1]
+    return {"value": round(nbytes / s_all / 1e9, 4), "unit": "GB/s", "cores": n_all, "kind": "oracle",
+            "sample": "whole layer T=%d (router, top-8, grouping, both grouped GEMMs, combine), median of %d runs "
+                      "on %d threads (OpenMP over tokens / routed pairs)" % (args.T, reps, n_all),
+            "latency_us": round(s_all * 1e6, 1), "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+            "single_thread": {"value": round(nbytes / s_one / 1e9, 4), "latency_us": round(s_one * 1e6, 1),
+                              "cores": 1, "sample": "same layer, median of %d runs on one thread" % reps}}
+
+
+def reference_arm(args, budget_s=180.0):
+    """The oracle as it stands on this host's threads, one whole layer per
+    step.  Steps beyond what fits in `budget_s` (after the first timed step)
+    are not run; `steps` reports how many were."""
+    import oracle
+    n_all = oracle.max_threads()
+    for _ in range(args.warmup):
+        oracle_layer_seconds(args.T, args.zipf, n_all)
+    ts, nbytes = [], 0
+    t_start = time.perf_counter()
+    for i in range(args.steps):
+        el, nbytes = oracle_layer_seconds(args.T, args.zipf, n_all)
+        ts.append(el)
+        if time.perf_counter() - t_start + el > budget_s:
+            break
+    sec = statistics.median(ts)
+    v = round(nbytes / sec / 1e9, 4)
+    sample = ("whole layer T=%d per step (router, top-8, grouping, both grouped GEMMs, combine) on %d threads; "
+              "%d of %d requested steps run within %.0f s" % (args.T, n_all, len(ts), args.steps, budget_s))
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "latency_us": round(sec * 1e6, 1),
+            "n_gpus": args.gpus, "steps": len(ts), "steps_requested": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "MoE layer T=%d, hidden 2048, 128 experts top-8, SwiGLU 768, Zipf s=%g bias, "
+                                   "%s schedule" % (args.T, args.zipf, args.sched),
+                       "T": args.T, "sched": args.sched, "zipf_s": args.zipf},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": n_all, "kind": "oracle", "sample": sample,
+                             "nproc": os.cpu_count(), "cpu_model": cpu_model()},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def main():
@@ -343,6 +452,8 @@ def main():
     ap.add_argument("--workload", default="moe", choices=["moe", "mlp", "splitk"],
                     help="moe (the benchmark line); mlp or splitk print a kernel timing line")
     ap.add_argument("--B", type=int, default=1, help="decode MLP batch (--workload mlp)")
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false", help="skip the T x schedule sweep")
+    ap.add_argument("--sweep-steps", type=int, default=50)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -360,23 +471,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        times = []
-        for i in range(args.warmup + args.steps):
-            r = cpu_oracle(args, budget_s=max(2.0, 60.0 / (args.warmup + args.steps)))
-            if i >= args.warmup:
-                times.append(r)
-        v = statistics.median(x["value"] for x in times)
-        lat = statistics.median(x["latency_us"] for x in times)
-        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "latency_us": lat,
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": round(lat / 1e3, 3), "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "MoE layer T=%d, hidden 2048, 128 experts top-8, SwiGLU 768, Zipf s=%g bias"
-                                       % (args.T, args.zipf), "T": args.T, "zipf_s": args.zipf},
-                "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                 "sample": times[-1]["sample"]},
-                "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line))
+        print(json.dumps(reference_arm(args)))
         return
 
     if world > 1:
@@ -388,7 +483,7 @@ def main():
         import torch
         torch.distributed.destroy_process_group()
     if rank == 0:
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_oracle(args)
         print(json.dumps(line))
 

@@ -19,7 +19,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 # ------------------------------------------------------------ constants --
-ET_OK, ET_ERR_INVALID, ET_ERR_CUDA, ET_ERR_TIMEOUT, ET_ERR_OOM, ET_ERR_UNSUPPORTED, ET_ERR_PENDING = range(7)
+ET_OK, ET_ERR_INVALID, ET_ERR_CUDA, ET_ERR_TIMEOUT, ET_ERR_OOM, ET_ERR_UNSUPPORTED, ET_ERR_PENDING, ET_ERR_INTERNAL = range(8)
 ET_SCHED_STATIC, ET_SCHED_DYNAMIC, ET_SCHED_UNFUSED = 0, 1, 2
 ET_GRAPH_SPLITK, ET_GRAPH_MLP, ET_GRAPH_MOE = 0, 1, 2
 ET_DEBUG_TRACE, ET_DEBUG_DELAY, ET_DEBUG_BAD_COUNT = 1, 2, 4
@@ -53,6 +53,10 @@ class et_trace_record(ctypes.Structure):
                 ("t_ready", ctypes.c_uint64), ("t_acc", ctypes.c_uint64), ("t_end", ctypes.c_uint64)]
 
 
+class et_event_count(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("index", ctypes.c_int32), ("count", ctypes.c_int32)]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _sigs = {
@@ -65,6 +69,7 @@ _sigs = {
     "et_get_trace": ([_P, _P, ctypes.c_size_t, ctypes.POINTER(_I)], _I),
     "et_get_info": ([_P, ctypes.POINTER(et_graph_info)], _I),
     "et_get_diag": ([_P, ctypes.POINTER(ctypes.c_int32)], _I),
+    "et_get_event_counts": ([_P, _P, _I, ctypes.POINTER(_I)], _I),
     "et_destroy_graph": ([_P], None),
     "et_status_str": ([_I], ctypes.c_char_p),
 }
@@ -143,6 +148,16 @@ def et_get_trace(g):
     buf = (et_trace_record * max(n.value, 1))()
     _check(_lib.et_get_trace(g, ctypes.cast(buf, _P), ctypes.sizeof(buf), ctypes.byref(n)), "et_get_trace")
     return [(r.op, r.a, r.b, r.sm, r.start, r.end, r.t_fetch, r.t_ready, r.t_acc, r.t_end) for r in buf[:n.value]]
+
+
+def et_get_event_counts(g):
+    """List of (kind, index, count): notifications each event of the last
+    run received (kind = ET_EV_* code of include/et.h)."""
+    n = _I(0)
+    _check(_lib.et_get_event_counts(g, None, 0, ctypes.byref(n)), "et_get_event_counts")
+    buf = (et_event_count * max(n.value, 1))()
+    _check(_lib.et_get_event_counts(g, ctypes.cast(buf, _P), n.value, ctypes.byref(n)), "et_get_event_counts")
+    return [(r.kind, r.index, r.count) for r in buf[:n.value]]
 
 
 def et_get_info(g):

@@ -257,6 +257,10 @@ __device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
 
 
 
+// Record the first device error of a run: the sticky status word and the
+// diagnostic words in device memory, a copy of the status in mapped host
+// memory (so the host sees it without a synchronisation), and the grid-wide
+// abort flag every spin checks.
 __device__ __forceinline__ void fail(Ctl* ctl, int code, int where, int a, int b, int c) {
     if (atomicCAS(&ctl->status, 0, code) == 0) {
         ctl->diag[0] = where;
@@ -265,6 +269,10 @@ __device__ __forceinline__ void fail(Ctl* ctl, int code, int where, int a, int b
         ctl->diag[3] = c;
         ctl->diag[4] = (int)blockIdx.x;
         ctl->diag[5] = (int)threadIdx.x;
+        if (ctl->host_status) {
+            *reinterpret_cast<volatile int*>(ctl->host_status) = code;
+            __threadfence_system();
+        }
     }
     __threadfence();
     atomicExch(&ctl->abort, 1);
@@ -354,6 +362,7 @@ __device__ __forceinline__ int task_b(uint32_t w) { return (int)(w & 0x3FF); }
 struct Queue {
     unsigned long long* slots;  // capacity entries, (epoch << 32) | task word
     int cap;
+    Ctl* ctl;                   // error reporting (a push past the capacity)
     int* head;                  // next slot to claim
     int* tail;                  // next slot to fill
     int* total;                 // total tasks this run + 1 (0 = not known yet)
@@ -367,9 +376,14 @@ __device__ __forceinline__ int q_reserve(const Queue& q, int n) { return q.n_ini
 
 // The ring never wraps within a run: its capacity covers every task of the
 // largest run plus one over-claimed batch per CTA, so a slot index is never
-// shared by two tasks of one run.
+// shared by two tasks of one run.  A push past the capacity would lose its
+// task: it is recorded as ET_ERR_INTERNAL (and the run aborts) instead.
+static __device__ __noinline__ void q_overflow(const Queue& q, int idx) {
+    fail(q.ctl, ET_ERR_INTERNAL, 903, idx, q.cap, (int)q.epoch);
+}
 __device__ __forceinline__ void q_publish(const Queue& q, int idx, uint32_t word) {
     if (idx < q.cap) st_release_u64(&q.slots[idx], ((unsigned long long)q.epoch << 32) | word);
+    else q_overflow(q, idx);
 }
 // Publish after the caller issued one release fence for the whole batch.
 __device__ __forceinline__ void q_publish_after_fence(const Queue& q, int idx, uint32_t word) {
@@ -377,6 +391,8 @@ __device__ __forceinline__ void q_publish_after_fence(const Queue& q, int idx, u
         asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(&q.slots[idx]),
                      "l"(((unsigned long long)q.epoch << 32) | word)
                      : "memory");
+    else
+        q_overflow(q, idx);
 }
 
 // Resolve slot `idx`: 1 = task in *word, 0 = no more tasks (idx beyond the

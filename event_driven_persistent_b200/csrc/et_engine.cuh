@@ -243,6 +243,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     x.ctr = ra.ctr;
     x.q.slots = ra.qslots;
     x.q.cap = ra.qcap;
+    x.q.ctl = ctl;
     x.q.head = ra.ctr + 0;
     x.q.tail = ra.ctr + 1;
     x.q.total = ra.ctr + 2;
@@ -409,10 +410,8 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     // B rows gathered through an index list: every lane copies
                     // up to 4 rows per stage with cp.async into the 128-byte
                     // swizzled layout; lane 0 adds the weight tile by TMA.
+                    // (the start ticket is taken before the index list is read)
                     any_gather = true;
-                    const uint16_t* rows[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) rows[i] = W::gather_row(p, d, lane + 32 * i);
                     if (lane == 0) {
                         ok = W::gemm_wait(p, x, d);
                         if (ok && (x.debug & ET_DEBUG_TRACE)) {
@@ -426,6 +425,9 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     __syncwarp();
                     ok = sc->pok;
                     __syncwarp();
+                    const uint16_t* rows[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) rows[i] = ok ? W::gather_row(p, d, lane + 32 * i) : nullptr;
                     for (int s = 0; s < d.nk && ok; ++s) {
                         if (lane == 0) {
                             uint32_t sl = 0, of = 0;

@@ -121,6 +121,8 @@ struct et_graph {
     et_graph_info info;
     int dev = 0, n_sm = 0, n_ctas = 0;
     Ctl* ctl = nullptr;
+    int* host_status = nullptr;      // mapped host word the kernel mirrors its error status into
+    int* host_status_dev = nullptr;  // its device address
     int* ctr[2] = {nullptr, nullptr};
     int n_ctr = 0;
     unsigned long long* qslots = nullptr;
@@ -134,6 +136,11 @@ struct et_graph {
     int* lists_off = nullptr;
     uint32_t* lists_words = nullptr;
     std::vector<void*> allocs;
+    // the last launched run (event-count introspection)
+    int last_T = 0;
+    SplitKParams last_sk;
+    MlpParams last_mlp;
+    MoeParams last_moe;
     // workload state
     SplitKParams sk;
     MlpParams mlp;
@@ -205,17 +212,21 @@ et_status build_lists(et_graph* g, const std::function<void(int, std::vector<Slo
     return ET_OK;
 }
 
+// Arguments of the graph's next run.  The run number (epoch) selects the
+// counter set and tags the queue slots; it is committed by commit_run only
+// once the launch succeeded, so a launch that failed leaves the counter sets
+// as they were (the set the next run uses is still the zeroed one).
 RunArgs run_args(et_graph* g, int T, int n_init, int total_static) {
     RunArgs ra;
     memset(&ra, 0, sizeof(ra));
-    ++g->epoch;
+    const uint32_t ep = g->epoch + 1;
     ra.ctl = g->ctl;
-    ra.ctr = g->ctr[g->epoch & 1];
-    ra.ctr_next = g->ctr[(g->epoch + 1) & 1];
+    ra.ctr = g->ctr[ep & 1];
+    ra.ctr_next = g->ctr[(ep + 1) & 1];
     ra.n_ctr = g->n_ctr;
     ra.qslots = g->qslots;
     ra.qcap = g->qcap;
-    ra.epoch = g->epoch;
+    ra.epoch = ep;
     ra.n_init = n_init;
     ra.total_static = total_static;
     ra.dynamic = g->d.sched == ET_SCHED_DYNAMIC;
@@ -230,7 +241,29 @@ RunArgs run_args(et_graph* g, int T, int n_init, int total_static) {
     return ra;
 }
 
+et_status launched(et_graph* g, cudaError_t e) {
+    if (e != cudaSuccess) return cuda_fail(e);
+    ++g->epoch;
+    return ET_OK;
+}
+
+// A device error of an earlier run that the host can already see (the
+// failing kernel mirrored it into mapped host memory) and that
+// et_sync_status has not collected yet.
+bool pending(const et_graph* g) { return *reinterpret_cast<volatile const int*>(g->host_status) != 0; }
+
+// Upload a clean control block (status 0, the host mirror's device address).
+et_status reset_ctl(et_graph* g) {
+    Ctl h;
+    memset(&h, 0, sizeof(h));
+    h.host_status = g->host_status_dev;
+    ET_CU(cudaMemcpy(g->ctl, &h, sizeof(Ctl), cudaMemcpyHostToDevice));
+    *reinterpret_cast<volatile int*>(g->host_status) = 0;
+    return ET_OK;
+}
+
 et_status pre_run(et_graph* g, cudaStream_t s) {
+    if (pending(g)) return ET_ERR_PENDING;
     if (g->d.debug_flags & ET_DEBUG_TRACE) {
         // the trace of one run: clear the record counter and tickets
         ET_CU(cudaMemsetAsync(&g->ctl->ticket, 0, 2 * sizeof(int), s));
@@ -445,7 +478,8 @@ const char* et_status_str(et_status s) {
         case ET_ERR_TIMEOUT: return "device wait timed out";
         case ET_ERR_OOM: return "out of device memory";
         case ET_ERR_UNSUPPORTED: return "unsupported device or dims";
-        case ET_ERR_PENDING: return "an earlier run failed";
+        case ET_ERR_PENDING: return "an earlier run failed and its error was not collected";
+        case ET_ERR_INTERNAL: return "device-side capacity check failed";
     }
     return "unknown status";
 }
@@ -478,6 +512,15 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     if (st != ET_OK) return fail(st);
     // common workspace
     if ((st = galloc(g, &g->ctl, 1)) != ET_OK) return fail(st);
+    {
+        void* hp = nullptr;
+        if (cudaHostAlloc(&hp, sizeof(int), cudaHostAllocMapped) != cudaSuccess) return fail(ET_ERR_OOM);
+        g->host_status = static_cast<int*>(hp);
+        void* dp = nullptr;
+        if (cudaHostGetDevicePointer(&dp, hp, 0) != cudaSuccess) return fail(ET_ERR_CUDA);
+        g->host_status_dev = static_cast<int*>(dp);
+        if ((st = reset_ctl(g)) != ET_OK) return fail(st);
+    }
     if ((st = galloc(g, &g->ctr[0], g->n_ctr)) != ET_OK) return fail(st);
     if ((st = galloc(g, &g->ctr[1], g->n_ctr)) != ET_OK) return fail(st);
     if ((st = galloc(g, &g->qslots, g->qcap)) != ET_OK) return fail(st);
@@ -524,6 +567,7 @@ void et_destroy_graph(et_graph* g) {
     cudaSetDevice(g->dev);
     cudaDeviceSynchronize();
     for (void* p : g->allocs) cudaFree(p);
+    if (g->host_status) cudaFreeHost(g->host_status);
     delete g;
 }
 
@@ -549,7 +593,9 @@ et_status et_run_splitk(et_graph* g, const float* A, int n_rows, float* Bpart, f
     ET_TRY(pre_run(g, s));
     const int n_init = p.n_tiles * p.n_chunks;
     RunArgs ra = run_args(g, n_rows, n_init, n_init + p.n_tiles);
-    ET_CU(launch_splitk(p, ra, g->n_ctas, s));
+    ET_TRY(launched(g, launch_splitk(p, ra, g->n_ctas, s)));
+    g->last_T = n_rows;
+    g->last_sk = p;
     return ET_OK;
 }
 
@@ -571,7 +617,9 @@ et_status et_run_mlp(et_graph* g, int B, const uint16_t* X, const uint16_t* gamm
     ET_TRY(pre_run(g, s));
     const int total = B + p.n_gu + p.n_m * p.n_c + p.n_m;
     RunArgs ra = run_args(g, B, B, total);
-    ET_CU(launch_mlp(p, ra, g->n_ctas, s));
+    ET_TRY(launched(g, launch_mlp(p, ra, g->n_ctas, s)));
+    g->last_T = B;
+    g->last_mlp = p;
     return ET_OK;
 }
 
@@ -609,7 +657,9 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
     p.f_max = mb.f_max;
     ET_TRY(pre_run(g, s));
     RunArgs ra = run_args(g, T, p.n_tk * p.n_kc, 0);
-    ET_CU(launch_moe(p, ra, g->n_ctas, s));
+    ET_TRY(launched(g, launch_moe(p, ra, g->n_ctas, s)));
+    g->last_T = T;
+    g->last_moe = p;
     return ET_OK;
 }
 
@@ -620,8 +670,9 @@ et_status et_sync_status(et_graph* g, void* stream) {
     Ctl h;
     ET_CU(cudaMemcpy(&h, g->ctl, sizeof(Ctl), cudaMemcpyDeviceToHost));
     if (h.status == 0) return ET_OK;
-    // reset: status, abort flag, counters, scratch that must start at zero
-    ET_CU(cudaMemset(g->ctl, 0, sizeof(Ctl)));
+    // reset: status, abort flag, host mirror, counters, scratch that must start at zero
+    ET_CU(cudaDeviceSynchronize());
+    ET_TRY(reset_ctl(g));
     ET_CU(cudaMemset(g->ctr[0], 0, g->n_ctr * sizeof(int)));
     ET_CU(cudaMemset(g->ctr[1], 0, g->n_ctr * sizeof(int)));
     if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc) {
@@ -644,6 +695,43 @@ et_status et_get_trace(et_graph* g, void* host_buf, size_t bytes, int* n_records
     *n_records = n;
     size_t want = std::min((size_t)n * sizeof(TraceRec), bytes);
     if (host_buf && want) ET_CU(cudaMemcpy(host_buf, g->trace, want, cudaMemcpyDeviceToHost));
+    return ET_OK;
+}
+
+et_status et_get_event_counts(et_graph* g, et_event_count* buf, int cap, int* n_events) {
+    if (!g || !n_events || cap < 0 || (cap > 0 && !buf)) return ET_ERR_INVALID;
+    if (g->last_T == 0) return ET_ERR_INVALID;
+    ET_CU(cudaSetDevice(g->dev));
+    ET_CU(cudaDeviceSynchronize());
+    std::vector<int> c(g->n_ctr);
+    ET_CU(cudaMemcpy(c.data(), g->ctr[g->epoch & 1], g->n_ctr * sizeof(int), cudaMemcpyDeviceToHost));
+    std::vector<et_event_count> v;
+    auto add = [&](int kind, int idx, int ctr_index) { v.push_back({kind, idx, c[ctr_index]}); };
+    if (g->d.kind == ET_GRAPH_SPLITK) {
+        const SplitKParams& p = g->last_sk;
+        for (int i = 0; i < p.n_tiles; ++i) add(ET_EV_SK_TILE, i, p.ev_base + i);
+        add(ET_EV_SK_ALL, 0, p.ev_all);
+    } else if (g->d.kind == ET_GRAPH_MLP) {
+        const MlpParams& p = g->last_mlp;
+        add(ET_EV_MLP_NORM, 0, p.ev_norm);
+        for (int i = 0; i < p.n_c; ++i) add(ET_EV_MLP_H, i, p.ev_h + i);
+        for (int i = 0; i < p.n_m; ++i) add(ET_EV_MLP_Y, i, p.ev_y + i);
+        add(ET_EV_MLP_GU_ALL, 0, p.ev_gu_all);
+        add(ET_EV_MLP_DOWN_ALL, 0, p.ev_down_all);
+    } else {
+        const MoeParams& p = g->last_moe;
+        for (int j = 0; j < p.n_tk; ++j) add(ET_EV_MOE_RT, j, p.ev_rt + j);
+        add(ET_EV_MOE_TK, 0, p.ev_tk);
+        add(ET_EV_MOE_SC, 0, p.ev_sc);
+        add(ET_EV_MOE_GRP, 0, p.ev_grp);
+        for (int e = 0; e < p.E; ++e) add(ET_EV_MOE_EXP, e, p.ev_exp + e);
+        for (int f = 0; f < p.f_max; ++f) add(ET_EV_MOE_S1, f, p.ev_s1 + f);
+        for (int b = 0; b < p.n_cb; ++b) add(ET_EV_MOE_CB, b, p.ev_cb + b);
+        add(ET_EV_MOE_S1_ALL, 0, p.ev_s1_all);
+        add(ET_EV_MOE_S2_ALL, 0, p.ev_s2_all);
+    }
+    *n_events = (int)v.size();
+    for (int i = 0; i < cap && i < (int)v.size(); ++i) buf[i] = v[i];
     return ET_OK;
 }
 

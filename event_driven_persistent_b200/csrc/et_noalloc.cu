@@ -93,16 +93,19 @@ extern "C" et_status et_run_splitk_noalloc(const float* A, int n_rows, float* Bp
     p.ev_all = kCtrFirstEvent + kNaMaxTiles;
     RunArgs ra;
     memset(&ra, 0, sizeof(ra));
-    ++nd.epoch;
+    // The call number selects the counter set; it is committed only after a
+    // successful launch, so a launch that failed leaves the next call on the
+    // set the previous call cleared.
+    const uint32_t ep = nd.epoch + 1;
     int* ctr0 = reinterpret_cast<int*>(nd.base + kOffCtr0);
     int* ctr1 = reinterpret_cast<int*>(nd.base + kOffCtr1);
     ra.ctl = reinterpret_cast<Ctl*>(nd.base + kOffCtl);
-    ra.ctr = (nd.epoch & 1) ? ctr1 : ctr0;       // zero at entry (cleared by the previous call)
-    ra.ctr_next = (nd.epoch & 1) ? ctr0 : ctr1;  // cleared during this call
+    ra.ctr = (ep & 1) ? ctr1 : ctr0;       // zero at entry (cleared by the previous call)
+    ra.ctr_next = (ep & 1) ? ctr0 : ctr1;  // cleared during this call
     ra.n_ctr = kNaCtr;
     ra.qslots = reinterpret_cast<unsigned long long*>(nd.base + kOffQueue);
     ra.qcap = kNaQueue;
-    ra.epoch = nd.epoch;
+    ra.epoch = ep;
     ra.n_init = p.n_tiles * p.n_chunks;
     ra.total_static = ra.n_init + p.n_tiles;
     ra.dynamic = 1;
@@ -110,7 +113,8 @@ extern "C" et_status et_run_splitk_noalloc(const float* A, int n_rows, float* Bp
     ra.trace = reinterpret_cast<TraceRec*>(nd.base + kOffTrace);
     ra.trace_cap = 1;
     ra.timeout_ns = 1000000000ull;
-    if (launch_splitk(p, ra, nd.n_ctas, s) != cudaSuccess) return ET_ERR_CUDA;
+    if (launch_splitk(p, ra, nd.n_ctas, s) != cudaSuccess) return ET_ERR_CUDA;  // nothing was enqueued
+    nd.epoch = ep;
     // Synchronous: read the device status of this call, and after a device
     // error clear the workspace so the next call starts clean.
     Ctl h;

@@ -46,7 +46,8 @@ struct Ctl {
     int diag[8];      // where the first error happened
     unsigned ticket;  // trace ticket counter
     int n_trace;      // trace records written
-    int pad[4];
+    int* host_status; // device address of a mapped host word that mirrors status (or null)
+    int pad[2];
 };
 
 // Per-run arguments common to every megakernel.

@@ -671,8 +671,9 @@ cudaError_t moe_setup(int* max_blocks_per_sm) {
 }
 
 cudaError_t launch_moe(const MoeParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s) {
-    moe_kernel<<<n_ctas, kThreads, kSmemBytes, s>>>(p, ra);
-    return cudaGetLastError();
+    // the launch's own status (not an unrelated error left pending earlier)
+    void* args[] = {const_cast<MoeParams*>(&p), const_cast<RunArgs*>(&ra)};
+    return cudaLaunchKernel(reinterpret_cast<const void*>(moe_kernel), dim3(n_ctas), dim3(kThreads), args, kSmemBytes, s);
 }
 
 }  // namespace et

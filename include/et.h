@@ -20,6 +20,13 @@
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Runs are
  *    asynchronous: et_run_* returns after the launch; device-side errors
  *    (a wait that timed out) are reported by et_sync_status.
+ *  - A device error is sticky per graph until et_sync_status collects it.
+ *    The failing kernel also mirrors its status into a word of mapped
+ *    host memory, so once the error has happened every et_run_* on the
+ *    graph returns ET_ERR_PENDING without launching.  A run that was
+ *    already launched (or issued before the error happened) finds the error
+ *    when it starts, does no work and leaves its outputs untouched; its
+ *    et_run_* returned ET_OK, and et_sync_status reports the error.
  *  - The token / batch count T (or B, or the split-K row count) is a plain
  *    run-time int: the same graph and binary serve every value up to
  *    max_T with no recompile and no graph capture ([ETN] §Shape dynamism).
@@ -46,7 +53,10 @@ typedef enum {
     ET_ERR_TIMEOUT = 3,     /* a device-side wait exceeded its time limit (see et_sync_status) */
     ET_ERR_OOM = 4,         /* workspace allocation failed */
     ET_ERR_UNSUPPORTED = 5, /* device is not sm_100, or dims outside what the kernels tile */
-    ET_ERR_PENDING = 6      /* an earlier run failed and its error was not yet collected by et_sync_status */
+    ET_ERR_PENDING = 6,     /* an earlier run of this graph failed on the device and the error was
+                               not yet collected by et_sync_status: nothing was launched */
+    ET_ERR_INTERNAL = 7     /* a device-side capacity check failed (a ready-queue push past its
+                               capacity); the run aborted instead of losing the task */
 } et_status;
 
 /* How tasks are ordered on the SMs ([ETN] §静态调度, §动态调度, §静态与动态调度的消融). */
@@ -133,6 +143,32 @@ typedef struct {
 #define ET_OP_MOE_S2 25
 #define ET_OP_MOE_COMBINE 26
 
+/* Event kinds of et_event_count records; index = the event's coordinate. */
+#define ET_EV_SK_TILE 1       /* split-K E[i]: partial tasks of row tile i done (count = #chunks) */
+#define ET_EV_SK_ALL 2        /* split-K, unfused control: every partial task done */
+#define ET_EV_MLP_NORM 10     /* E_norm: normalised rows (count = B) */
+#define ET_EV_MLP_H 11        /* E_h[c]: gate/up tiles of down K-chunk c */
+#define ET_EV_MLP_Y 12        /* E_y[m]: down partials of output tile m (count = #K chunks) */
+#define ET_EV_MLP_GU_ALL 13   /* unfused control: every gate/up tile */
+#define ET_EV_MLP_DOWN_ALL 14 /* unfused control: every down tile */
+#define ET_EV_MOE_RT 20       /* E_rt[j]: K chunks of router block j (kept only when the K is split) */
+#define ET_EV_MOE_TK 21       /* E_tk: router blocks routed (top-k taken) */
+#define ET_EV_MOE_SC 22       /* E_sc: the scan (runs with several grouping tiles) */
+#define ET_EV_MOE_GRP 23      /* E_grp: the coarse grouping event (static and unfused schedules) */
+#define ET_EV_MOE_EXP 24      /* E_exp[e]: pairs of expert e placed (dynamic, several grouping tiles;
+                                 one tile is grouped by the scan, which then triggers directly) */
+#define ET_EV_MOE_S1 25       /* E_s1[f]: stage-1 tiles of m-tile f */
+#define ET_EV_MOE_CB 26       /* E_cb[b]: stage-2 row contributions to combine block b */
+#define ET_EV_MOE_S1_ALL 27   /* unfused control: every stage-1 tile */
+#define ET_EV_MOE_S2_ALL 28   /* unfused control: every stage-2 tile */
+
+/* Notifications one event received in the last run (debug introspection). */
+typedef struct {
+    int32_t kind;   /* ET_EV_* */
+    int32_t index;  /* coordinate of the event in its event tensor */
+    int32_t count;  /* notifications received (the pages' wait count minus the remaining count) */
+} et_event_count;
+
 /* Build a graph: validate dims, allocate its workspace for max_T, build the
  * static per-SM task lists for every power-of-two bucket up to max_T
  * ([ETN] §静态调度: "per-SM task queue" materialised at build time; an
@@ -210,16 +246,27 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
 et_status et_run_splitk_noalloc(const float* A, int n_rows, float* Bpart, float* C, void* stream);
 
 /* Synchronise `stream`, then read and clear the graph's sticky device
- * status.  Returns ET_OK, or ET_ERR_TIMEOUT if a wait of any run since the
- * last call gave up (every CTA then drained and exited; no trap).  After a
- * device error the workspace (counters, scratch) is reset here, so the next
- * run starts clean; until then et_run_* refuses with ET_ERR_PENDING. */
+ * status.  Returns ET_OK, or the device error of a run since the last call:
+ * ET_ERR_TIMEOUT if a wait gave up, ET_ERR_INTERNAL if a capacity check
+ * failed (every CTA then drained and exited; no trap).  After a device
+ * error the workspace (counters, scratch, the host mirror of the status)
+ * is reset here, so the next run starts clean; until then et_run_* returns
+ * ET_ERR_PENDING. */
 et_status et_sync_status(et_graph* g, void* stream);
 
 /* Copy the trace of the last run (ET_DEBUG_TRACE) to host memory.
  * Synchronises the device.  *n_records receives the record count; at most
  * bytes / sizeof(et_trace_record) records are copied. */
 et_status et_get_trace(et_graph* g, void* host_buf, size_t bytes, int* n_records);
+
+/* Every event of the last run's graph (for that run's T) with the number of
+ * notifications it received ("Event Tensor：用“事件张量”编译动态 Megakernel",
+ * §Event Tensor: a consumer runs once its event received its wait count).
+ * Synchronises the device; call it after the run and before the next run of
+ * the graph (which clears these counters).  At most `cap` records are
+ * written to `buf` (host memory); *n_events receives the total number.
+ * ET_ERR_INVALID if the graph has not run yet. */
+et_status et_get_event_counts(et_graph* g, et_event_count* buf, int cap, int* n_events);
 
 /* Tile parameters of a built graph. */
 et_status et_get_info(const et_graph* g, et_graph_info* info);

@@ -20,7 +20,7 @@ _lib = None
 def build(force=False):
     """Compile liboracle.so next to its source (gcc, -O2, strict IEEE)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fopenmp",
                "-o", _LIB, _SRC, "-lm"]
         subprocess.check_call(cmd)
     return _LIB
@@ -31,7 +31,26 @@ def _load():
     if _lib is None:
         build()
         _lib = ctypes.CDLL(_LIB)
+        _lib.orc_moe_grouped.restype = ctypes.c_int
+        for f in ("orc_get_threads", "orc_max_threads"):
+            getattr(_lib, f).restype = ctypes.c_int
+        _lib.orc_set_threads(ctypes.c_int(int(os.environ.get("ORACLE_THREADS", "1"))))
     return _lib
+
+
+def set_threads(n):
+    """OpenMP threads for the oracle's parallel loops (tokens, rows, pairs);
+    results are bit-identical for every thread count."""
+    _load().orc_set_threads(ctypes.c_int(int(n)))
+
+
+def get_threads():
+    return _load().orc_get_threads()
+
+
+def max_threads():
+    """Processors available to this process."""
+    return _load().orc_max_threads()
 
 
 def _p(a):
@@ -151,10 +170,16 @@ def moe_grouped(X, W1, W2, topk, w, indptr, perm, want_h=False):
     k = topk.shape[1]
     Y = np.zeros((T, hidden), np.uint16)
     h = np.zeros((T * k, inter), np.uint16) if want_h else None
-    lib.orc_moe_grouped(_p(X), _p(_c(W1, np.uint16)), _p(_c(W2, np.uint16)), _p(_c(topk, np.int32)),
-                        _p(_c(w, np.float32)), _p(_c(indptr, np.int32)), _p(_c(perm, np.int32)),
-                        ctypes.c_int(T), ctypes.c_int(hidden), ctypes.c_int(inter), ctypes.c_int(E),
-                        ctypes.c_int(k), _p(Y), _p(h))
+    indptr = _c(indptr, np.int32)
+    perm = _c(perm, np.int32)
+    if indptr.shape != (E + 1,) or perm.shape != (T * k,):
+        raise ValueError("malformed grouping: indptr must have E+1 entries and perm T*k")
+    rc = lib.orc_moe_grouped(_p(X), _p(_c(W1, np.uint16)), _p(_c(W2, np.uint16)), _p(_c(topk, np.int32)),
+                             _p(_c(w, np.float32)), _p(indptr), _p(perm),
+                             ctypes.c_int(T), ctypes.c_int(hidden), ctypes.c_int(inter), ctypes.c_int(E),
+                             ctypes.c_int(k), _p(Y), _p(h))
+    if rc != 0:
+        raise ValueError("malformed grouping: indptr/perm do not group the pairs of topk by expert")
     return (Y, h) if want_h else Y
 
 
@@ -193,6 +218,46 @@ def moe_rows_given_routing(X, W1, W2, tokens, topk_rows, w_rows):
     return Y
 
 
+def rope(x, pos, base=500000.0):
+    """Rotary embedding of one bf16 head vector at position pos (bf16 out)."""
+    lib = _load()
+    x = _c(x, np.uint16)
+    out = np.zeros_like(x)
+    lib.orc_rope_bf16(_p(x), ctypes.c_int(x.shape[0]), ctypes.c_int(int(pos)), ctypes.c_double(base), _p(out))
+    return out
+
+
+def decode_layer(X, pos, w, Kc, Vc, n_q, n_kv, eps=1e-5, rope_base=500000.0):
+    """One decode step of the layer for B requests (see orc_decode_layer).
+    w: dict(g1, Wqkv, gq, gk, Wo, g2, Wgu, Wd) of bf16 bits.  Kc, Vc:
+    [B, n_kv, max_ctx, hd] caches; copies are updated and returned.
+    Returns dict(y, q, k, a, h1, Kc, Vc)."""
+    lib = _load()
+    X = _c(X, np.uint16)
+    pos = _c(pos, np.int32)
+    B, hidden = X.shape
+    Kc = np.array(Kc, dtype=np.uint16, copy=True)
+    Vc = np.array(Vc, dtype=np.uint16, copy=True)
+    _, nkv2, max_ctx, hd = Kc.shape
+    assert nkv2 == n_kv and Vc.shape == Kc.shape and Kc.shape[0] == B
+    inter = w["Wgu"].shape[0] // 2
+    Y = np.zeros((B, hidden), np.uint16)
+    q = np.zeros((B, n_q * hd), np.uint16)
+    k = np.zeros((B, n_kv * hd), np.uint16)
+    a = np.zeros((B, n_q * hd), np.uint16)
+    h1 = np.zeros((B, hidden), np.uint16)
+    rc = lib.orc_decode_layer(_p(X), _p(pos), ctypes.c_int(B), ctypes.c_int(hidden), ctypes.c_int(n_q),
+                              ctypes.c_int(n_kv), ctypes.c_int(hd), ctypes.c_int(inter),
+                              _p(_c(w["g1"], np.uint16)), _p(_c(w["Wqkv"], np.uint16)), _p(_c(w["gq"], np.uint16)),
+                              _p(_c(w["gk"], np.uint16)), _p(_c(w["Wo"], np.uint16)), _p(_c(w["g2"], np.uint16)),
+                              _p(_c(w["Wgu"], np.uint16)), _p(_c(w["Wd"], np.uint16)), _p(Kc), _p(Vc),
+                              ctypes.c_int(max_ctx), ctypes.c_double(eps), ctypes.c_double(rope_base),
+                              _p(Y), _p(q), _p(k), _p(a), _p(h1))
+    if rc != 0:
+        raise ValueError("decode layer: a position lies outside the cache")
+    return dict(y=Y, q=q, k=k, a=a, h1=h1, Kc=Kc, Vc=Vc)
+
+
 def moe(X, Wr, bias, W1, W2, k, bm=128):
     """Whole MoE layer through the grouped path; returns a dict of every
     intermediate the method defines (logits, topk, w, grouping, h, y)."""
@@ -205,5 +270,5 @@ def moe(X, Wr, bias, W1, W2, k, bm=128):
     return out
 
 
-__all__ = ["build", "bf16_round_bits", "splitk", "rmsnorm", "mlp", "mlp_rows", "router_logits",
-           "topk_softmax", "group", "moe_grouped", "moe_per_token", "moe_rows_given_routing", "moe"]
+__all__ = ["build", "set_threads", "get_threads", "max_threads", "bf16_round_bits", "splitk", "rmsnorm", "mlp", "mlp_rows", "router_logits",
+           "topk_softmax", "group", "moe_grouped", "moe_per_token", "moe_rows_given_routing", "moe", "rope", "decode_layer"]

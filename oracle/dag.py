@@ -12,10 +12,24 @@ that a device execution trace can be checked against it:
 * every task of the graph ran exactly once, and nothing else ran;
 * for every edge p -> c, p finished before c started (tickets from one
   global counter, taken by c after its wait and by p before its notify);
-* every event received exactly its wait count of notifications.
+* every event received exactly its wait count of notifications
+  (``check_wait_counts`` on the expansion itself, ``check_event_counts``
+  against the counts the device reports after a run).
+
+The event graph restates which events the device library uses.  A second,
+independent check does not look at events at all: ``*_dataflow`` derives
+from what each operator computes the data every task reads and writes
+(router logits of a token, the grouped row of a routed pair, a column tile
+of the stage-1 output, the combine accumulator of a token, ...), and
+``check_dataflow`` requires every writer of an item to finish before any
+task that reads it starts.  A dependency missing from the device's event
+design (and so from the event graph) is still caught there.
 
 Tasks are tuples ``(op, a, b)``; the op names and coordinates follow the
-trace record format of the device library (see ``include/et.h``).
+trace record format of the device library (see ``include/et.h``).  An
+"inline" task is work the device runs inside another task (the top-k of a
+router block, run by the router task that completes the block); it has no
+trace record, and edges through it are contracted.
 """
 from collections import defaultdict
 
@@ -33,31 +47,69 @@ def _cdiv(a, b):
     return (a + b - 1) // b
 
 
+# event kinds of the device's event-count records (an interface: the same
+# numbers are declared in include/et.h) -> event names used below
+EVENT_KIND = {1: "E", 2: "Eall", 10: "E_norm", 11: "E_h", 12: "E_y", 13: "E_h_all", 14: "E_y_all",
+              20: "E_rt", 21: "E_tk", 22: "E_sc", 23: "E_grp", 24: "E_exp", 25: "E_s1", 26: "E_cb",
+              27: "E_s1_all", 28: "E_s2_all"}
+_SCALAR_EVENTS = {"Eall", "E_norm", "E_h_all", "E_y_all", "E_tk", "E_sc", "E_grp", "E_s1_all", "E_s2_all"}
+
+
+def event_key(kind, index):
+    name = EVENT_KIND[kind]
+    return (name,) if name in _SCALAR_EVENTS else (name, index)
+
+
 class Graph:
-    """Explicit DAG: tasks, edges, and per-event producer lists."""
+    """Explicit DAG: tasks, edges, per-event producer lists (one entry per
+    notification, so a task that notifies an event n times is listed n
+    times) and the declared wait count of every event a counter realises."""
 
     def __init__(self):
         self.tasks = []
+        self.inline = set()
         self.edges = set()
-        self.event_producers = defaultdict(list)   # event -> producer tasks
+        self.event_producers = defaultdict(list)   # event -> producer tasks (with multiplicity)
         self.event_consumers = defaultdict(list)   # event -> consumer tasks
-        self.wait_count = {}                        # event -> declared wait count
+        self.wait_count = {}                        # counted event -> declared wait count
 
-    def add_task(self, t):
+    def add_task(self, t, inline=False):
         self.tasks.append(t)
+        if inline:
+            self.inline.add(t)
 
-    def produce(self, task, event):
-        self.event_producers[event].append(task)
+    def produce(self, task, event, n=1):
+        self.event_producers[event].extend([task] * n)
 
     def consume(self, task, event):
         self.event_consumers[event].append(task)
 
+    def counted(self, event, wait_count):
+        """`event` is a device counter that fires at `wait_count` notifications."""
+        self.wait_count[event] = int(wait_count)
+
     def finish(self):
-        """Edges = every producer of an event -> every consumer of it."""
+        """Edges = every producer of an event -> every consumer of it, with
+        inline tasks contracted (pred -> inline -> succ becomes pred -> succ)."""
+        raw = set()
         for ev, cons in self.event_consumers.items():
-            for p in self.event_producers.get(ev, []):
+            for p in set(self.event_producers.get(ev, [])):
                 for c in cons:
-                    self.edges.add((p, c))
+                    raw.add((p, c))
+        if self.inline:
+            pred, succ = defaultdict(set), defaultdict(set)
+            for p, c in raw:
+                pred[c].add(p)
+                succ[p].add(c)
+            for t in self.inline:
+                for p in pred[t]:
+                    for c in succ[t]:
+                        raw.add((p, c))
+                        pred[c].add(p)
+                        succ[p].add(c)
+            raw = {(p, c) for (p, c) in raw if p not in self.inline and c not in self.inline}
+        self.edges = raw
+        self.tasks = [t for t in self.tasks if t not in self.inline]
         return self
 
 
@@ -77,9 +129,12 @@ def splitk_graph(rows, cols, chunk, tile_rows, sched):
         t = (OP_SK_FINAL, i, 0)
         g.add_task(t)
         g.consume(t, ("E", i) if sched != "unfused" else ("Eall",))
-    for i in range(n):
-        g.wait_count[("E", i)] = J
-    g.wait_count[("Eall",)] = n * J
+    # E = ETensor((n,), wait_count=#chunks): each row tile's final waits for its partials
+    if sched != "unfused":
+        for i in range(n):
+            g.counted(("E", i), J)
+    else:
+        g.counted(("Eall",), n * J)
     return g.finish()
 
 
@@ -116,19 +171,30 @@ def mlp_graph(B, hidden, inter, gu_tile, down_tile, kchunk, sched):
         t = (OP_MLP_REDUCE, m, 0)
         g.add_task(t)
         g.consume(t, ("E_y_all",) if unf else ("E_y", m))
-    g.wait_count[("E_norm",)] = B
+    # wait counts: every row normalised (a symbolic count B); a K chunk of h
+    # holds kchunk / gu_tile gate/up tiles; an output tile sums every chunk
+    g.counted(("E_norm",), B)
+    if unf:
+        g.counted(("E_h_all",), n_gu)
+        g.counted(("E_y_all",), n_m * n_c)
+    else:
+        for c in range(n_c):
+            g.counted(("E_h", c), sum(1 for n in range(n_gu) if (n * gu_tile) // kchunk == c))
+        for m in range(n_m):
+            g.counted(("E_y", m), n_c)
     return g.finish()
 
 
 def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
     """MoE layer, expanded with the runtime routing `topk` [T, k]:
       router (j, c)   --"jc->j"-->           E_rt[j]         (count = #K chunks n_kc; tkt
-                                                             tokens per block j)
-      the chunk task completing E_rt[j] routes block j (logits, top-k,
-      softmax), so every router (j, c) precedes:
-      router (j, *)   --"j->"-->             E_tk            (count = #token blocks)
+                                                             tokens per block j; only with n_kc > 1)
+      E_rt[j]         -->                    route j         (inline: top-k + softmax of block j,
+                                                             run by the chunk task completing E_rt[j])
+      route j         --"j->"-->             E_tk            (count = #token blocks)
       E_tk            -->                    scan
-      one grouping tile (T <= tt): the scan is the grouping task:
+      one grouping tile (T <= tt): the scan is the grouping task and
+      triggers the stage-1 tasks itself (E_exp has no counter then):
       scan            --> E_exp[topk[i,:]] for every token i
       several grouping tiles:
       scan            -->                    E_sc            (count 1)
@@ -162,23 +228,38 @@ def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
         r = rows_of[e]
         for m in range(_cdiv(len(r), bm)):
             mtiles.append((e, m, r[m * bm:(m + 1) * bm]))
+    counts = [len(r) for r in rows_of]
     for j in range(n_tk):
+        route = ("route", j)
+        g.add_task(route, inline=True)
         for c in range(n_kc):
             task = (OP_MOE_ROUTER, j, c)
             g.add_task(task)
-            g.produce(task, ("E_tk",))
+            if n_kc > 1:
+                g.produce(task, ("E_rt", j))
+            else:
+                g.produce(task, ("E_rt1", j))   # one chunk: the router task routes its own block
+        if n_kc > 1:
+            g.consume(route, ("E_rt", j))
+            g.counted(("E_rt", j), n_kc)
+        else:
+            g.consume(route, ("E_rt1", j))
+        g.produce(route, ("E_tk",))
+    g.counted(("E_tk",), n_tk)
     scan = (OP_MOE_SCAN, 0, 0)
     g.add_task(scan)
     g.consume(scan, ("E_tk",))
     if n_tt == 1:
         if unf or static:
             g.produce(scan, ("E_grp",))
+            g.counted(("E_grp",), 1)
         else:
             for i in range(T):
                 for s in range(k):
                     g.produce(scan, ("E_exp", int(topk[i, s])))
     else:
         g.produce(scan, ("E_sc",))
+        g.counted(("E_sc",), 1)
         for q in range(n_g):
             task = (OP_MOE_GROUP, q, 0)
             g.add_task(task)
@@ -189,12 +270,23 @@ def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
                 for i in range(q * gt, min(T, (q + 1) * gt)):
                     for s in range(k):
                         g.produce(task, ("E_exp", int(topk[i, s])))
+        if unf or static:
+            g.counted(("E_grp",), n_g)
+        else:
+            # data-dependent initial count: the number of pairs routed to e
+            for e in range(E):
+                if counts[e]:
+                    g.counted(("E_exp", e), counts[e])
     for f, (e, m, rows) in enumerate(mtiles):
         for n in range(n_n1):
             task = (OP_MOE_S1, f, n)
             g.add_task(task)
             g.consume(task, ("E_grp",) if (unf or static) else ("E_exp", e))
             g.produce(task, ("E_s1_all",) if unf else ("E_s1", f))
+        if not unf:
+            g.counted(("E_s1", f), n_n1)
+    if unf:
+        g.counted(("E_s1_all",), len(mtiles) * n_n1)
     for f, (e, m, rows) in enumerate(mtiles):
         for n in range(n_n2):
             task = (OP_MOE_S2, f, n)
@@ -208,7 +300,16 @@ def moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched):
     for b in range(n_cb):
         task = (OP_MOE_COMBINE, b, 0)
         g.add_task(task)
-        g.consume(task, ("E_s2_all",) if unf else ("E_cb", b))
+        if unf:
+            g.consume(task, ("E_grp",))
+            g.consume(task, ("E_s2_all",))
+        else:
+            g.consume(task, ("E_cb", b))
+            # every stage-2 column tile of every routed pair of the block's tokens
+            ntok = min(cb, T - b * cb)
+            g.counted(("E_cb", b), k * n_n2 * ntok)
+    if unf:
+        g.counted(("E_s2_all",), len(mtiles) * n_n2)
     return g.finish(), mtiles
 
 
@@ -233,4 +334,153 @@ def check_trace(graph, records):
     for (p, c) in graph.edges:
         if p in seen and c in seen and not seen[p][1] < seen[c][0]:
             errs.append("edge violated: %r (end %d) -> %r (start %d)" % (p, seen[p][1], c, seen[c][0]))
+    return errs
+
+
+# ------------------------------------------------------------ wait counts --
+
+def check_wait_counts(graph):
+    """Every counted event has exactly its wait count of producer
+    notifications in the expansion.  Returns violation strings."""
+    errs = []
+    for ev, want in sorted(graph.wait_count.items(), key=repr):
+        got = len(graph.event_producers.get(ev, []))
+        if got != want:
+            errs.append("event %r: %d producer notifications, wait count %d" % (ev, got, want))
+    return errs
+
+
+def check_event_counts(graph, device_counts):
+    """device_counts: (kind, index, count) records of the device's events
+    after a run.  Every event the expansion counts received exactly its wait
+    count of notifications; every other event of the device received none.
+    Returns violation strings."""
+    errs = []
+    seen = set()
+    for kind, index, count in device_counts:
+        key = event_key(int(kind), int(index))
+        seen.add(key)
+        want = graph.wait_count.get(key, 0)
+        if int(count) != want:
+            errs.append("event %r received %d notifications, wait count %d" % (key, int(count), want))
+    for key in graph.wait_count:
+        if key not in seen:
+            errs.append("event %r has no device counter" % (key,))
+    return errs
+
+
+# --------------------------------------------------------------- dataflow --
+# Read and write sets of each task, from what its operator computes.  Items:
+#   ("logit", t, c)   K chunk c of token t's router logits
+#   ("route", t)      top-k experts and weights of token t (a function of all
+#                     of t's logit chunks; the router tasks of t's block write it)
+#   ("csr",)          expert counts, pair CSR, m-tile CSR (needs every token's route)
+#   ("row", r)        the routed pair placed at grouped row r
+#   ("h", r, n)       stage-1 output of grouped row r, column tile n
+#   ("acc", t, n)     token t's combine accumulator, column tile n (summed by stage 2)
+#   ("y", t)          token t's output
+
+def moe_dataflow(topk, n_kc, tkt, tt, bm, n_n1, n_n2, cb, E):
+    """{task: (reads, writes)} of every task of the MoE layer given the
+    runtime routing; the task split (tkt, n_kc, tt, bm, n-tiles, cb) is the
+    device's tiling, the items each task touches follow from the operators."""
+    topk = np.asarray(topk)
+    T, k = topk.shape
+    rw = {}
+    # stable grouping by brute force: expert-major, ascending token
+    order = [(t, s) for e in range(E) for t in range(T) for s in range(k) if int(topk[t, s]) == e]
+    row_of = {pair: r for r, pair in enumerate(order)}
+    all_route = {("route", t) for t in range(T)}
+    for j in range(_cdiv(T, tkt)):
+        toks = range(j * tkt, min(T, (j + 1) * tkt))
+        for c in range(n_kc):
+            w = {("logit", t, c) for t in toks} | {("route", t) for t in toks}
+            rw[(OP_MOE_ROUTER, j, c)] = (set(), w)
+    n_tt = _cdiv(T, tt)
+    sc_w = {("csr",)}
+    if n_tt == 1:
+        sc_w |= {("row", r) for r in range(len(order))}
+    rw[(OP_MOE_SCAN, 0, 0)] = (set(all_route), sc_w)
+    if n_tt > 1:
+        for g in range(n_tt):
+            toks = range(g * tt, min(T, (g + 1) * tt))
+            rows = {("row", row_of[(t, s)]) for t in toks for s in range(k)}
+            rw[(OP_MOE_GROUP, g, 0)] = ({("csr",)} | all_route, rows)
+    f = 0
+    for e in range(E):
+        rows_e = [r for r, (t, s) in enumerate(order) if int(topk[t, s]) == e]
+        for m in range(_cdiv(len(rows_e), bm)):
+            rows = rows_e[m * bm:(m + 1) * bm]
+            toks = {order[r][0] for r in rows}
+            base = {("csr",)} | {("row", r) for r in rows}
+            for n in range(n_n1):
+                rw[(OP_MOE_S1, f, n)] = (set(base), {("h", r, n) for r in rows})
+            h_all = {("h", r, n) for r in rows for n in range(n_n1)}
+            for n in range(n_n2):
+                rw[(OP_MOE_S2, f, n)] = (base | h_all | {("route", t) for t in toks},
+                                         {("acc", t, n) for t in toks})
+            f += 1
+    for b in range(_cdiv(T, cb)):
+        toks = range(b * cb, min(T, (b + 1) * cb))
+        rw[(OP_MOE_COMBINE, b, 0)] = ({("acc", t, n) for t in toks for n in range(n_n2)},
+                                      {("y", t) for t in toks})
+    return rw
+
+
+def mlp_dataflow(B, hidden, inter, gu_tile, down_tile, kchunk):
+    """Decode MLP: norm b writes xn row b; gate/up tile n reads every xn row
+    and writes h columns of tile n; down (m, c) reads the h columns of K
+    chunk c and writes partial (m, c); reduce m reads every partial of m."""
+    rw = {}
+    n_gu, n_m, n_c = _cdiv(inter, gu_tile), _cdiv(hidden, down_tile), _cdiv(inter, kchunk)
+    for b in range(B):
+        rw[(OP_MLP_NORM, b, 0)] = (set(), {("xn", b)})
+    for n in range(n_gu):
+        rw[(OP_MLP_GATEUP, n, 0)] = ({("xn", b) for b in range(B)}, {("h", n)})
+    for m in range(n_m):
+        for c in range(n_c):
+            cols = {("h", n) for n in range(n_gu) if c * kchunk <= n * gu_tile < (c + 1) * kchunk}
+            rw[(OP_MLP_DOWN, m, c)] = (cols, {("part", m, c)})
+        rw[(OP_MLP_REDUCE, m, 0)] = ({("part", m, c) for c in range(n_c)}, {("y", m)})
+    return rw
+
+
+def splitk_dataflow(rows, cols, chunk, tile_rows):
+    """Split-K: partial (i, j) writes B[rows of tile i, j]; final i reads
+    B[rows of tile i, every j]."""
+    rw = {}
+    n, J = _cdiv(rows, tile_rows), _cdiv(cols, chunk)
+    for i in range(n):
+        for j in range(J):
+            rw[(OP_SK_PARTIAL, i, j)] = (set(), {("B", i, j)})
+        rw[(OP_SK_FINAL, i, 0)] = ({("B", i, j) for j in range(J)}, {("C", i)})
+    return rw
+
+
+def check_dataflow(rw, records):
+    """Every task that reads an item starts after every task that writes it
+    has finished (read-after-write by ticket).  records as in check_trace.
+    Returns violation strings."""
+    start, end = {}, {}
+    for r in records:
+        key = (int(r[0]), int(r[1]), int(r[2]))
+        start[key], end[key] = int(r[4]), int(r[5])
+    writers = defaultdict(list)
+    for task, (_, writes) in rw.items():
+        for it in writes:
+            writers[it].append(task)
+    errs = []
+    for task, (reads, _) in rw.items():
+        if task not in start:
+            errs.append("task never ran: %r" % (task,))
+            continue
+        for it in reads:
+            for w in writers.get(it, []):
+                if w == task:
+                    continue
+                if w not in end:
+                    errs.append("writer of %r never ran: %r" % (it, w))
+                elif not end[w] < start[task]:
+                    errs.append("read before write: %r reads %r, written by %r (end %d, start %d)"
+                                % (task, it, w, end[w], start[task]))
     return errs

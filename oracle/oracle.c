@@ -17,9 +17,15 @@
  * and routing weights are fp32 tensors).  bf16 rounding is round-to-nearest-
  * even, written out below from the IEEE definition.
  *
+ * Threads: loops whose iterations compute disjoint outputs (tokens, rows,
+ * routed pairs) may run on several OpenMP threads (orc_set_threads).  Each
+ * output is still computed by one thread with the same sums in the same
+ * order, so every result is bit-identical for any thread count.
+ *
  * Parity status of each entry point is stated in its comment.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -49,6 +55,12 @@ static float orc_bf16_to_f32(uint16_t h) {
 static uint16_t orc_d_to_bf16(double d) { return orc_f32_to_bf16((float)d); }
 
 uint16_t orc_bf16_round_bits(float f) { return orc_f32_to_bf16(f); }
+
+/* Number of OpenMP threads used by the parallel loops below (default 1). */
+static int orc_threads = 1;
+void orc_set_threads(int n) { orc_threads = n > 0 ? n : 1; }
+int orc_get_threads(void) { return orc_threads; }
+int orc_max_threads(void) { return omp_get_num_procs(); }
 float orc_bf16_value(uint16_t h) { return orc_bf16_to_f32(h); }
 
 /* ------------------------------------------------------------- split-K -- */
@@ -157,6 +169,7 @@ void orc_mlp(const uint16_t* X, const uint16_t* gamma, const uint16_t* Wgu, cons
  * accumulation, rounded to fp32 (the logits tensor is fp32). */
 void orc_router_logits(const uint16_t* X, const uint16_t* Wr, const float* bias, int T, int hidden,
                        int E, float* logits) {
+#pragma omp parallel for num_threads(orc_threads) schedule(dynamic, 1) if (T > 1)
     for (int t = 0; t < T; ++t)
         for (int e = 0; e < E; ++e) {
             double acc = 0.0;
@@ -245,22 +258,51 @@ static void orc_expert(const uint16_t* x, const uint16_t* W1, const uint16_t* W2
  * pairs (perm order), then the weighted combine per token in slot order:
  *   y[t] = bf16( sum_{s<k} w[t,s] * o[t,s] )  (double sum, slots 0..k-1).
  * topk/w/indptr/perm come from orc_topk_softmax and orc_group.
- * h_out [T*k, inter] in grouped (perm) order is optional. */
-void orc_moe_grouped(const uint16_t* X, const uint16_t* W1, const uint16_t* W2,
-                     const int32_t* topk, const float* w, const int32_t* indptr,
-                     const int32_t* perm, int T, int hidden, int inter, int E, int k,
-                     uint16_t* Y, uint16_t* h_out) {
-    double* o_all = (double*)malloc((size_t)T * k * hidden * sizeof(double));
-    uint16_t* h = (uint16_t*)malloc((size_t)inter * 2);
-    for (int e = 0; e < E; ++e)
-        for (int r = indptr[e]; r < indptr[e + 1]; ++r) {
+ * h_out [T*k, inter] in grouped (perm) order is optional.
+ * Returns 0, or -1 (and computes nothing) when the grouping is malformed:
+ * indptr not a non-decreasing CSR over T*k pairs, a perm entry out of
+ * range or listed twice, or a pair listed under an expert its topk entry
+ * does not name. */
+int orc_moe_grouped(const uint16_t* X, const uint16_t* W1, const uint16_t* W2,
+                    const int32_t* topk, const float* w, const int32_t* indptr,
+                    const int32_t* perm, int T, int hidden, int inter, int E, int k,
+                    uint16_t* Y, uint16_t* h_out) {
+    const int P = T * k;
+    if (indptr[0] != 0 || indptr[E] != P) return -1;
+    int32_t* row_expert = (int32_t*)malloc((size_t)(P > 0 ? P : 1) * sizeof(int32_t));
+    char* seen = (char*)calloc((size_t)(P > 0 ? P : 1), 1);
+    int bad = 0;
+    for (int e = 0; e < E && !bad; ++e) {
+        if (indptr[e + 1] < indptr[e]) bad = 1;
+        for (int r = indptr[e]; r < indptr[e + 1] && !bad; ++r) {
+            int p = perm[r];
+            if (p < 0 || p >= P || seen[p] || topk[p] != e) bad = 1;
+            else {
+                seen[p] = 1;
+                row_expert[r] = e;
+            }
+        }
+    }
+    free(seen);
+    if (bad) {
+        free(row_expert);
+        return -1;
+    }
+    double* o_all = (double*)malloc((size_t)(P > 0 ? P : 1) * hidden * sizeof(double));
+#pragma omp parallel num_threads(orc_threads) if (P > 1)
+    {
+        uint16_t* h = (uint16_t*)malloc((size_t)inter * 2);
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < P; ++r) {
             int p = perm[r];
             int t = p / k;
-            if (topk[p] != e) { free(o_all); free(h); return; } /* malformed grouping */
-            orc_expert(X + (size_t)t * hidden, W1, W2, hidden, inter, e, h,
+            orc_expert(X + (size_t)t * hidden, W1, W2, hidden, inter, row_expert[r], h,
                        o_all + (size_t)p * hidden);
             if (h_out) memcpy(h_out + (size_t)r * inter, h, (size_t)inter * 2);
         }
+        free(h);
+    }
+    free(row_expert);
     for (int t = 0; t < T; ++t)
         for (int n = 0; n < hidden; ++n) {
             double acc = 0.0;
@@ -269,7 +311,7 @@ void orc_moe_grouped(const uint16_t* X, const uint16_t* W1, const uint16_t* W2,
             Y[(size_t)t * hidden + n] = orc_d_to_bf16(acc);
         }
     free(o_all);
-    free(h);
+    return 0;
 }
 
 /* MoE layer, per-token evaluation of the same definition: for each token,
@@ -282,11 +324,14 @@ void orc_moe_per_token(const uint16_t* X, const uint16_t* Wr, const float* bias,
                        const uint16_t* W1, const uint16_t* W2, const int32_t* tokens,
                        int n_tokens, int hidden, int inter, int E, int k, uint16_t* Y_rows,
                        int32_t* topk_rows, float* w_rows) {
+#pragma omp parallel num_threads(orc_threads) if (n_tokens > 1)
+    {
     float* l = (float*)malloc((size_t)E * sizeof(float));
     int32_t* idx = (int32_t*)malloc((size_t)k * sizeof(int32_t));
     float* wt = (float*)malloc((size_t)k * sizeof(float));
     uint16_t* h = (uint16_t*)malloc((size_t)inter * 2);
     double* o = (double*)malloc((size_t)k * hidden * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
     for (int i = 0; i < n_tokens; ++i) {
         const uint16_t* x = X + (size_t)tokens[i] * hidden;
         orc_router_logits(x, Wr, bias, 1, hidden, E, l);
@@ -305,6 +350,7 @@ void orc_moe_per_token(const uint16_t* X, const uint16_t* Wr, const float* bias,
     free(wt);
     free(h);
     free(o);
+    }
 }
 
 /* Same per-token evaluation, but with the routing given (topk, w for each
@@ -314,8 +360,11 @@ void orc_moe_rows_given_routing(const uint16_t* X, const uint16_t* W1, const uin
                                 const int32_t* tokens, const int32_t* topk_rows,
                                 const float* w_rows, int n_tokens, int hidden, int inter, int k,
                                 uint16_t* Y_rows) {
+#pragma omp parallel num_threads(orc_threads) if (n_tokens > 1)
+    {
     uint16_t* h = (uint16_t*)malloc((size_t)inter * 2);
     double* o = (double*)malloc((size_t)k * hidden * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
     for (int i = 0; i < n_tokens; ++i) {
         const uint16_t* x = X + (size_t)tokens[i] * hidden;
         for (int s = 0; s < k; ++s)
@@ -328,6 +377,7 @@ void orc_moe_rows_given_routing(const uint16_t* X, const uint16_t* W1, const uin
     }
     free(h);
     free(o);
+    }
 }
 
 /* MLP rows: the decode MLP evaluated for the listed rows only (sampled
@@ -335,10 +385,168 @@ void orc_moe_rows_given_routing(const uint16_t* X, const uint16_t* W1, const uin
 void orc_mlp_rows(const uint16_t* X, const uint16_t* gamma, const uint16_t* Wgu, const uint16_t* Wd,
                   const int32_t* rows, int n_rows, int hidden, int inter, double eps,
                   uint16_t* Y_rows) {
-    uint16_t* x1 = (uint16_t*)malloc((size_t)hidden * 2);
-    for (int i = 0; i < n_rows; ++i) {
-        memcpy(x1, X + (size_t)rows[i] * hidden, (size_t)hidden * 2);
-        orc_mlp(x1, gamma, Wgu, Wd, 1, hidden, inter, eps, Y_rows + (size_t)i * hidden, NULL, NULL);
+#pragma omp parallel num_threads(orc_threads) if (n_rows > 1)
+    {
+        uint16_t* x1 = (uint16_t*)malloc((size_t)hidden * 2);
+#pragma omp for schedule(dynamic, 1)
+        for (int i = 0; i < n_rows; ++i) {
+            memcpy(x1, X + (size_t)rows[i] * hidden, (size_t)hidden * 2);
+            orc_mlp(x1, gamma, Wgu, Wd, 1, hidden, inter, eps, Y_rows + (size_t)i * hidden, NULL, NULL);
+        }
+        free(x1);
     }
-    free(x1);
+}
+
+/* --------------------------------------------------------- decode layer -- */
+
+/* Rotary position embedding of one head vector at position `pos`
+ * (rotate-half pairing: element i is rotated with element i + dim/2 by the
+ * angle pos * base^(-2i/dim), i < dim/2).  In place, double precision. */
+static void orc_rope(double* v, int dim, int pos, double base) {
+    int half = dim / 2;
+    for (int i = 0; i < half; ++i) {
+        double ang = (double)pos * pow(base, -2.0 * (double)i / (double)dim);
+        double c = cos(ang), s = sin(ang);
+        double a = v[i], b = v[i + half];
+        v[i] = a * c - b * s;
+        v[i + half] = b * c + a * s;
+    }
+}
+
+void orc_rope_bf16(const uint16_t* x, int dim, int pos, double base, uint16_t* out) {
+    double* v = (double*)malloc((size_t)dim * sizeof(double));
+    for (int i = 0; i < dim; ++i) v[i] = orc_bf16_to_f32(x[i]);
+    orc_rope(v, dim, pos, base);
+    for (int i = 0; i < dim; ++i) out[i] = orc_d_to_bf16(v[i]);
+    free(v);
+}
+
+/* One decode step of a transformer layer for B requests, each adding one
+ * token ([ETN] §端到端低 batch serving: the decoding pipeline fuses
+ * Attention, RoPE, KV-cache, Norm and MLP; the Q branch runs Norm + RoPE,
+ * the K branch Norm + RoPE + cache append).  Per request b, at position
+ * p = pos[b] (the number of tokens already in its cache):
+ *   xn  = bf16(rmsnorm(x) * g1)
+ *   qkv = bf16(xn . Wqkv^T)                 rows: n_q query heads, then
+ *                                           n_kv key heads, then n_kv value heads
+ *   q_h = bf16(rope(rmsnorm(q_h) * gq, p))  every query head (per-head norm)
+ *   k_g = bf16(rope(rmsnorm(k_g) * gk, p))  every key head
+ *   cache: K[b,g,p] = k_g, V[b,g,p] = v_g   (written in place)
+ *   o_h = sum_{j<=p} softmax_j(q_h . K[b,g,j] / sqrt(hd)) V[b,g,j],  g = h / (n_q / n_kv)
+ *   a   = bf16(o)                            heads concatenated [n_q * hd]
+ *   h1  = bf16(x + a . Wo^T)                 residual, one rounding
+ *   y   = bf16(h1 + mlp(h1))                 mlp = the decode MLP above
+ *                                           (rmsnorm with g2, SwiGLU, down)
+ * Caches are [B, n_kv, max_ctx, hd] bf16.  All sums in double, in index
+ * order; softmax max-subtracted.  Optional outputs (NULL to skip): q_out
+ * [B, n_q*hd], k_out [B, n_kv*hd], a_out [B, n_q*hd], h1_out [B, hidden].
+ * Returns 0, or -1 when a position is outside the cache. */
+int orc_decode_layer(const uint16_t* X, const int32_t* pos, int B, int hidden, int n_q, int n_kv,
+                     int hd, int inter, const uint16_t* g1, const uint16_t* Wqkv, const uint16_t* gq,
+                     const uint16_t* gk, const uint16_t* Wo, const uint16_t* g2,
+                     const uint16_t* Wgu, const uint16_t* Wd, uint16_t* Kc, uint16_t* Vc,
+                     int max_ctx, double eps, double rope_base, uint16_t* Y, uint16_t* q_out,
+                     uint16_t* k_out, uint16_t* a_out, uint16_t* h1_out) {
+    for (int b = 0; b < B; ++b)
+        if (pos[b] < 0 || pos[b] >= max_ctx) return -1;
+    const int nqkv = (n_q + 2 * n_kv) * hd;
+    const int group = n_q / n_kv;
+    const double scale = 1.0 / sqrt((double)hd);
+#pragma omp parallel num_threads(orc_threads) if (B > 1)
+    {
+        uint16_t* xn = (uint16_t*)malloc((size_t)hidden * 2);
+        uint16_t* qkv = (uint16_t*)malloc((size_t)nqkv * 2);
+        uint16_t* q = (uint16_t*)malloc((size_t)n_q * hd * 2);
+        uint16_t* a = (uint16_t*)malloc((size_t)n_q * hd * 2);
+        uint16_t* h1 = (uint16_t*)malloc((size_t)hidden * 2);
+        double* o = (double*)malloc((size_t)(hidden > nqkv ? hidden : nqkv) * sizeof(double));
+        double* v = (double*)malloc((size_t)hd * sizeof(double));
+        double* s = (double*)malloc((size_t)max_ctx * sizeof(double));
+        double* acc = (double*)malloc((size_t)hd * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b) {
+            const uint16_t* x = X + (size_t)b * hidden;
+            const int p = pos[b];
+            orc_rmsnorm(x, g1, 1, hidden, eps, xn);
+            orc_linear_row(xn, Wqkv, hidden, nqkv, o);
+            for (int i = 0; i < nqkv; ++i) qkv[i] = orc_d_to_bf16(o[i]);
+            /* Q branch: per-head norm + rope */
+            for (int h = 0; h < n_q; ++h) {
+                const uint16_t* qh = qkv + (size_t)h * hd;
+                double ss = 0.0;
+                for (int i = 0; i < hd; ++i) {
+                    double t = orc_bf16_to_f32(qh[i]);
+                    ss += t * t;
+                }
+                double inv = 1.0 / sqrt(ss / (double)hd + eps);
+                for (int i = 0; i < hd; ++i) v[i] = orc_bf16_to_f32(qh[i]) * inv * orc_bf16_to_f32(gq[i]);
+                orc_rope(v, hd, p, rope_base);
+                for (int i = 0; i < hd; ++i) q[(size_t)h * hd + i] = orc_d_to_bf16(v[i]);
+            }
+            /* K branch: per-head norm + rope + cache append; V appended as is */
+            for (int g = 0; g < n_kv; ++g) {
+                const uint16_t* kh = qkv + (size_t)(n_q + g) * hd;
+                const uint16_t* vh = qkv + (size_t)(n_q + n_kv + g) * hd;
+                double ss = 0.0;
+                for (int i = 0; i < hd; ++i) {
+                    double t = orc_bf16_to_f32(kh[i]);
+                    ss += t * t;
+                }
+                double inv = 1.0 / sqrt(ss / (double)hd + eps);
+                for (int i = 0; i < hd; ++i) v[i] = orc_bf16_to_f32(kh[i]) * inv * orc_bf16_to_f32(gk[i]);
+                orc_rope(v, hd, p, rope_base);
+                uint16_t* kd = Kc + (((size_t)b * n_kv + g) * max_ctx + p) * hd;
+                uint16_t* vd = Vc + (((size_t)b * n_kv + g) * max_ctx + p) * hd;
+                for (int i = 0; i < hd; ++i) {
+                    kd[i] = orc_d_to_bf16(v[i]);
+                    vd[i] = vh[i];
+                }
+                if (k_out) memcpy(k_out + ((size_t)b * n_kv + g) * hd, kd, (size_t)hd * 2);
+            }
+            /* attention over positions 0..p (the appended token included) */
+            for (int h = 0; h < n_q; ++h) {
+                const int g = h / group;
+                const uint16_t* K = Kc + ((size_t)b * n_kv + g) * max_ctx * hd;
+                const uint16_t* V = Vc + ((size_t)b * n_kv + g) * max_ctx * hd;
+                const uint16_t* qh = q + (size_t)h * hd;
+                double m = -INFINITY;
+                for (int j = 0; j <= p; ++j) {
+                    double d = 0.0;
+                    for (int i = 0; i < hd; ++i)
+                        d += (double)orc_bf16_to_f32(qh[i]) * (double)orc_bf16_to_f32(K[(size_t)j * hd + i]);
+                    s[j] = d * scale;
+                    if (s[j] > m) m = s[j];
+                }
+                double z = 0.0;
+                for (int j = 0; j <= p; ++j) {
+                    s[j] = exp(s[j] - m);
+                    z += s[j];
+                }
+                for (int i = 0; i < hd; ++i) acc[i] = 0.0;
+                for (int j = 0; j <= p; ++j)
+                    for (int i = 0; i < hd; ++i) acc[i] += s[j] * (double)orc_bf16_to_f32(V[(size_t)j * hd + i]);
+                for (int i = 0; i < hd; ++i) a[(size_t)h * hd + i] = orc_d_to_bf16(acc[i] / z);
+            }
+            /* o-proj + residual */
+            orc_linear_row(a, Wo, n_q * hd, hidden, o);
+            for (int n = 0; n < hidden; ++n) h1[n] = orc_d_to_bf16((double)orc_bf16_to_f32(x[n]) + o[n]);
+            /* MLP + residual: y = bf16(h1 + down(silu(gate(xn2)) * up(xn2))), one rounding */
+            {
+                uint16_t* xn2 = (uint16_t*)malloc((size_t)hidden * 2);
+                uint16_t* hm = (uint16_t*)malloc((size_t)inter * 2);
+                orc_rmsnorm(h1, g2, 1, hidden, eps, xn2);
+                orc_swiglu_row(xn2, Wgu, hidden, inter, hm);
+                orc_linear_row(hm, Wd, inter, hidden, o);
+                for (int n = 0; n < hidden; ++n)
+                    Y[(size_t)b * hidden + n] = orc_d_to_bf16((double)orc_bf16_to_f32(h1[n]) + o[n]);
+                free(xn2);
+                free(hm);
+            }
+            if (q_out) memcpy(q_out + (size_t)b * n_q * hd, q, (size_t)n_q * hd * 2);
+            if (a_out) memcpy(a_out + (size_t)b * n_q * hd, a, (size_t)n_q * hd * 2);
+            if (h1_out) memcpy(h1_out + (size_t)b * hidden, h1, (size_t)hidden * 2);
+        }
+        free(xn); free(qkv); free(q); free(a); free(h1); free(o); free(v); free(s); free(acc);
+    }
+    return 0;
 }

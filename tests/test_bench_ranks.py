@@ -96,3 +96,6 @@ def test_reference_arm_line():
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["T"] == 2
+    # one whole layer per step, and the steps reported are the steps run
+    assert d["steps"] == 1 and d["ms_per_step"] > 0
+    assert "whole layer" in d["cpu_baseline"]["sample"]

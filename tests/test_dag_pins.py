@@ -101,3 +101,116 @@ def test_moe_two_tiles_by_hand():
     want |= {((S1, f, 0), (S2, f, 0)) for f in range(2)}
     want |= {((S2, 0, 0), (CB, 0, 0)), ((S2, 1, 0), (CB, 0, 0)), ((S2, 1, 0), (CB, 1, 0))}
     assert g.edges == want
+
+
+# ------------------------------------------- wait counts and data-level order --
+# §Event Tensor 的本质 (an event's wait count = the producer notifications it
+# needs), §Data-dependent event update (E_exp[e] starts at the number of
+# pairs routed to e).
+
+import heapq
+
+
+def _trace_priority(graph, first, last=frozenset()):
+    """A valid trace of `graph` (tasks one after another, in a topological
+    order) that runs the tasks in `first` as early and those in `last` as
+    late as the graph allows."""
+    indeg = {t: 0 for t in graph.tasks}
+    succ = {t: [] for t in graph.tasks}
+    for p, c in graph.edges:
+        indeg[c] += 1
+        succ[p].append(c)
+    prio = lambda t: 0 if t in first else (2 if t in last else 1)  # noqa: E731
+    heap = [(prio(t), i, t) for i, t in enumerate(graph.tasks) if indeg[t] == 0]
+    heapq.heapify(heap)
+    order_ix = {t: i for i, t in enumerate(graph.tasks)}
+    recs, tick = [], 0
+    while heap:
+        _, _, t = heapq.heappop(heap)
+        recs.append((t[0], t[1], t[2], 0, tick, tick + 1))
+        tick += 2
+        for c in succ[t]:
+            indeg[c] -= 1
+            if indeg[c] == 0:
+                heapq.heappush(heap, (prio(c), order_ix[c], c))
+    return recs
+
+
+def _moe_case(T, sched, n_kc=2, tt=4, cb=2, seed=0):
+    rng = np.random.default_rng(seed)
+    E, k = 5, 2
+    topk = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    kw = dict(E=E, tt=tt, n_kc=n_kc, tkt=2, gt=tt, bm=3, n_n1=2, n_n2=2, cb=cb)
+    g, mt = dag.moe_graph(topk, sched=sched, **kw)
+    rw = dag.moe_dataflow(topk, n_kc=n_kc, tkt=2, tt=tt, bm=3, n_n1=2, n_n2=2, cb=cb, E=E)
+    return topk, g, mt, rw
+
+
+def test_wait_counts_of_every_graph():
+    for sched in ("static", "dynamic", "unfused"):
+        assert dag.check_wait_counts(dag.splitk_graph(100, 128, 32, 32, sched)) == []
+        assert dag.check_wait_counts(dag.mlp_graph(3, 256, 512, 64, 128, 256, sched)) == []
+        for T in (3, 9):
+            for n_kc in (1, 2):
+                _, g, _, _ = _moe_case(T, sched, n_kc=n_kc)
+                assert dag.check_wait_counts(g) == [], (T, sched, n_kc)
+
+
+def test_expert_event_count_is_pairs_routed():
+    topk, g, _, _ = _moe_case(9, "dynamic")
+    for e in range(5):
+        n = int(np.sum(topk == e))
+        if n:
+            assert g.wait_count[("E_exp", e)] == n
+
+
+def test_event_counts_check_against_device_records():
+    _, g, _, _ = _moe_case(9, "dynamic")
+    names = {v: k for k, v in dag.EVENT_KIND.items()}
+    recs = [(names[ev[0]], ev[1] if len(ev) > 1 else 0, n) for ev, n in g.wait_count.items()]
+    recs.append((names["E_grp"], 0, 0))   # an event this schedule does not use: no notification
+    assert dag.check_event_counts(g, recs) == []
+    short = [r if i else (r[0], r[1], r[2] - 1) for i, r in enumerate(recs)]
+    assert any("received" in e for e in dag.check_event_counts(g, short))
+    stray = recs[:-1] + [(names["E_grp"], 0, 1)]   # a notification of an event the graph does not use
+    assert any("E_grp" in e for e in dag.check_event_counts(g, stray))
+
+
+def test_dataflow_accepts_every_event_order():
+    for sched in ("static", "dynamic", "unfused"):
+        for T, n_kc in ((3, 1), (9, 2)):
+            _, g, _, rw = _moe_case(T, sched, n_kc=n_kc)
+            for first in (set(), {t for t in g.tasks if t[0] == dag.OP_MOE_COMBINE}):
+                assert dag.check_dataflow(rw, _trace_priority(g, first)) == []
+    g = dag.mlp_graph(3, 256, 512, 64, 128, 256, "dynamic")
+    assert dag.check_dataflow(dag.mlp_dataflow(3, 256, 512, 64, 128, 256), _trace_priority(g, set())) == []
+    g = dag.splitk_graph(100, 128, 32, 32, "dynamic")
+    assert dag.check_dataflow(dag.splitk_dataflow(100, 128, 32, 32), _trace_priority(g, set())) == []
+
+
+def _drop(g, pred):
+    g.edges = {(p, c) for (p, c) in g.edges if not pred(p, c)}
+    return g
+
+
+def test_dataflow_catches_a_dependency_missing_from_the_event_design():
+    """Plant a missing true dependency in the event graph (as a kernel with a
+    wrong event map would have it); a trace that follows the mutilated graph
+    passes the event-level check but not the data-level one."""
+    S1, S2, CB, R, SC = dag.OP_MOE_S1, dag.OP_MOE_S2, dag.OP_MOE_COMBINE, dag.OP_MOE_ROUTER, dag.OP_MOE_SCAN
+    plants = [
+        # stage 2 of m-tile 0 no longer waits for stage-1 column tile 1
+        (lambda p, c: p == (S1, 0, 1) and c[0] == S2 and c[1] == 0, {(S2, 0, 0), (S2, 0, 1)}, {(S1, 0, 1)}),
+        # combine block 0 no longer waits for the stage-2 tasks of m-tile 0
+        (lambda p, c: p[0] == S2 and p[1] == 0 and c == (CB, 0, 0), {(CB, 0, 0)}, {(S2, 0, 0), (S2, 0, 1)}),
+        # the scan no longer waits for router K chunk 1 of block 0
+        (lambda p, c: p == (R, 0, 1) and c == (SC, 0, 0), {(SC, 0, 0)}, {(R, 0, 1)}),
+    ]
+    for pred, first, last in plants:
+        topk, g, mt, rw = _moe_case(9, "dynamic", n_kc=2, tt=16, cb=4)
+        # make sure the planted consumer really reads what the dropped producer writes
+        g = _drop(g, pred)
+        recs = _trace_priority(g, first, last)
+        assert dag.check_trace(g, recs) == []
+        errs = dag.check_dataflow(rw, recs)
+        assert any("read before write" in e for e in errs), errs[:3]

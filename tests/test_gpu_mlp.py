@@ -70,7 +70,13 @@ def test_mlp_dependency_order(sched):
         info = et.et_get_info(g)
         graph = dag.mlp_graph(B, hidden, inter, info["mlp_gu_tile"], info["mlp_down_tile"], info["mlp_kchunk"],
                               sched)
-        errs = dag.check_trace(graph, et.et_get_trace(g))
+        trace = et.et_get_trace(g)
+        errs = dag.check_trace(graph, trace)
+        assert errs == [], errs[:5]
+        rw = dag.mlp_dataflow(B, hidden, inter, info["mlp_gu_tile"], info["mlp_down_tile"], info["mlp_kchunk"])
+        errs = dag.check_dataflow(rw, trace)
+        assert errs == [], errs[:5]
+        errs = dag.check_event_counts(graph, et.et_get_event_counts(g))
         assert errs == [], errs[:5]
         assert maxnorm_err(Y, oracle.mlp(d["X"], d["gamma"], d["Wgu"], d["Wd"])) <= TOL
     finally:
@@ -84,10 +90,10 @@ def full_mlp():
 
 
 @pytest.mark.parametrize("sched", ["static", "dynamic"])
-@pytest.mark.parametrize("B", [1, 4, 16])
-def test_mlp_full_size_sampled_rows(full_mlp, sched, B):
-    """Llama-3-8B-shaped MLP (4096 -> 2x14336 -> 4096) at B in {1,4,16}; the
-    oracle evaluates sampled rows."""
+@pytest.mark.parametrize("B", [1, 4, 16, 64])
+def test_mlp_full_size_every_row(full_mlp, sched, B):
+    """Llama-3-8B-shaped MLP (4096 -> 2x14336 -> 4096) at B in {1,4,16,64};
+    the oracle evaluates every row."""
     d, t = full_mlp
     g = et.et_build_graph(et.ET_GRAPH_MLP, sched, 64)
     try:
@@ -95,7 +101,7 @@ def test_mlp_full_size_sampled_rows(full_mlp, sched, B):
         Y = empty_bf16(B, 4096)
         et.et_run_mlp(g, B, dev(X), t["gamma"], t["Wgu"], t["Wd"], Y)
         assert et.et_sync_status(g) == 0
-        rows = sorted({0, B - 1, B // 2})
+        rows = list(range(B))
         ref = oracle.mlp_rows(X, d["gamma"], d["Wgu"], d["Wd"], rows)
         assert maxnorm_err(host(Y, np.uint16)[rows], ref) <= TOL
     finally:

@@ -141,11 +141,19 @@ def test_moe_dependency_order(small_inputs, sched, T):
         assert st == 0
         info = et.et_get_info(g)
         # the router split of a run is fixed by its size bucket; read it from the trace
-        rt = [r for r in et.et_get_trace(g) if r[0] == dag.OP_MOE_ROUTER]
+        trace = et.et_get_trace(g)
+        rt = [r for r in trace if r[0] == dag.OP_MOE_ROUTER]
         n_kc = max(r[2] for r in rt) + 1
+        n_n1, n_n2 = 128 // info["moe_n1_tile"], 256 // info["moe_n2_tile"]
         graph, _ = dag.moe_graph(out["topk"], 16, info["moe_tt"], n_kc, info["moe_tkt"], info["moe_gt"], info["moe_bm"],
-                                 128 // info["moe_n1_tile"], 256 // info["moe_n2_tile"], info["moe_cb"], sched)
-        errs = dag.check_trace(graph, et.et_get_trace(g))
+                                 n_n1, n_n2, info["moe_cb"], sched)
+        errs = dag.check_trace(graph, trace)
+        assert errs == [], errs[:5]
+        rw = dag.moe_dataflow(out["topk"], n_kc, info["moe_tkt"], info["moe_tt"], info["moe_bm"], n_n1, n_n2,
+                              info["moe_cb"], 16)
+        errs = dag.check_dataflow(rw, trace)
+        assert errs == [], errs[:5]
+        errs = dag.check_event_counts(graph, et.et_get_event_counts(g))
         assert errs == [], errs[:5]
     finally:
         et.et_destroy_graph(g)
@@ -162,29 +170,95 @@ def test_moe_timeout_reports(small_inputs, sched):
         et.et_destroy_graph(g)
 
 
+@pytest.mark.parametrize("sched", ["static", "dynamic"])
+def test_moe_pending_error_refuses_next_run(small_inputs, sched):
+    """A device error (a wait count one too high, 50 ms limit) makes the next
+    et_run_moe return ET_ERR_PENDING without launching, until et_sync_status
+    collects the error."""
+    d = small_inputs
+    g = et.et_build_graph(et.ET_GRAPH_MOE, sched, 64, debug_flags=et.ET_DEBUG_BAD_COUNT, timeout_ms=50.0, **SMALL)
+    try:
+        t = {n: dev(d[n]) for n in ("Wr", "bias", "W1", "W2")}
+        X = dev(d["X"][:10])
+        Y = empty_bf16(10, 256)
+        et.et_run_moe(g, 10, X, t["Wr"], t["bias"], t["W1"], t["W2"], Y)
+        torch.cuda.synchronize()
+        with pytest.raises(et.EtError) as e:
+            et.et_run_moe(g, 10, X, t["Wr"], t["bias"], t["W1"], t["W2"], Y)
+        assert e.value.status == et.ET_ERR_PENDING
+        assert et.et_sync_status(g) == et.ET_ERR_TIMEOUT
+    finally:
+        et.et_destroy_graph(g)
+
+
+# ------------------------------------------------------------- full size --
+# Qwen3-30B-A3B-shaped layer (hidden 2048 -> 128 experts x SwiGLU 768, top-8,
+# Zipf(s) expert bias), every size the benchmark times, both schedules.
+
+FULL_T = [1, 16, 128, 256, 1024, 4096]
+FULL_S = [0.0, 1.2, 1.5]
+
+
 @pytest.fixture(scope="module")
 def full_moe():
-    d = W.moe_inputs(128, zipf_s=1.2)
-    t = {n: dev(d[n]) for n in ("Wr", "bias", "W1", "W2")}
-    return d, t
+    d = W.moe_inputs(1, zipf_s=1.2)
+    t = {n: dev(d[n]) for n in ("Wr", "W1", "W2")}
+    g = {s: et.et_build_graph(et.ET_GRAPH_MOE, s, 4096) for s in ("static", "dynamic")}
+    cache = {}
+    yield d, t, g, cache
+    for h in g.values():
+        et.et_destroy_graph(h)
+
+
+def _sample_tokens(T, topk, k, E, seed):
+    """Every token up to 256; beyond, one routed pair of every m-tile
+    (128 grouped rows of one expert) plus the first and last token."""
+    if T <= 256:
+        return list(range(T))
+    grp = oracle.group(topk, E, 128)
+    rng = np.random.default_rng(seed)
+    toks = {0, T - 1}
+    for e in range(E):
+        for r0 in range(grp["indptr"][e], grp["indptr"][e + 1], 128):
+            r1 = min(r0 + 128, grp["indptr"][e + 1])
+            toks.add(int(grp["perm"][rng.integers(r0, r1)]) // k)
+    return sorted(toks)
 
 
 @pytest.mark.parametrize("sched", ["static", "dynamic"])
-@pytest.mark.parametrize("T", [1, 16, 128])
-def test_moe_full_size_sampled_tokens(full_moe, sched, T):
-    """Qwen3-30B-A3B-shaped layer (2048 -> 128 experts x SwiGLU 768, top-8,
-    Zipf(1.2) expert bias); the oracle evaluates sampled tokens per token
-    with the device's routing."""
-    d, t = full_moe
+@pytest.mark.parametrize("zipf", FULL_S)
+@pytest.mark.parametrize("T", FULL_T)
+def test_moe_full_size(full_moe, sched, zipf, T):
+    """Routing bit-exact for every token (on the device's logits), event
+    counts equal to the expansion's wait counts, and Y against the oracle's
+    per-token evaluation with the device's routing: every token up to
+    T = 256, a token of every m-tile beyond."""
+    d, t, graphs, cache = full_moe
+    E, k = 128, 8
     dT = dict(d)
     dT["X"] = W.moe_inputs(T, weights=False)["X"]
-    g = et.et_build_graph(et.ET_GRAPH_MOE, sched, 4096)
-    try:
-        st, out = run_moe(g, dT, T, 8, 128, t)
-        assert st == 0
-        w_o, grp = check_routing(dT, out, 8, 128, T)
-        toks = sorted({0, T - 1, T // 2, T // 3})
-        y_ref = oracle.moe_rows_given_routing(dT["X"], d["W1"], d["W2"], toks, out["topk"][toks], w_o[toks])
-        assert maxnorm_err(out["y"][toks], y_ref) <= TOL_Y
-    finally:
-        et.et_destroy_graph(g)
+    dT["bias"] = W.expert_bias(E, zipf)
+    tt = dict(t)
+    tt["bias"] = dev(dT["bias"])
+    g = graphs[sched]
+    st, out = run_moe(g, dT, T, k, E, tt)
+    assert st == 0
+    w_o, grp = check_routing(dT, out, k, E, T)
+    # every event received its wait count (data-dependent ones from this routing)
+    counts = et.et_get_event_counts(g)
+    n_kc = max([c for kind, _, c in counts if kind == 20] + [1])
+    n_cb = sum(1 for kind, _, _ in counts if kind == 26)
+    cb = 1 if n_cb == T else -(-T // n_cb)
+    info = et.et_get_info(g)
+    graph, _ = dag.moe_graph(out["topk"], E, info["moe_tt"], n_kc, info["moe_tkt"], info["moe_gt"], info["moe_bm"],
+                             768 // info["moe_n1_tile"], 2048 // info["moe_n2_tile"], cb, sched)
+    errs = dag.check_event_counts(graph, counts)
+    assert errs == [], errs[:5]
+    toks = _sample_tokens(T, out["topk"], k, E, seed=T)
+    need = [i for i in toks if (zipf, T, i, out["topk"][i].tobytes(), w_o[i].tobytes()) not in cache]
+    if need:
+        ref = oracle.moe_rows_given_routing(dT["X"], d["W1"], d["W2"], need, out["topk"][need], w_o[need])
+        for i, row in zip(need, ref):
+            cache[(zipf, T, i, out["topk"][i].tobytes(), w_o[i].tobytes())] = row
+    y_ref = np.stack([cache[(zipf, T, i, out["topk"][i].tobytes(), w_o[i].tobytes())] for i in toks])
+    assert maxnorm_err(out["y"][toks], y_ref) <= TOL_Y

@@ -91,7 +91,12 @@ def test_splitk_dependency_order(sched, delay):
         assert st == 0
         check(A, B, C)
         graph = dag.splitk_graph(512, 128, 32, 32, sched)
-        errs = dag.check_trace(graph, et.et_get_trace(g))
+        trace = et.et_get_trace(g)
+        errs = dag.check_trace(graph, trace)
+        assert errs == [], errs[:5]
+        errs = dag.check_dataflow(dag.splitk_dataflow(512, 128, 32, 32), trace)
+        assert errs == [], errs[:5]
+        errs = dag.check_event_counts(graph, et.et_get_event_counts(g))
         assert errs == [], errs[:5]
     finally:
         et.et_destroy_graph(g)
@@ -114,3 +119,25 @@ def test_splitk_wait_timeout_reports_and_recovers(sched):
         check(A, B, C)
     finally:
         et.et_destroy_graph(good)
+
+
+@pytest.mark.parametrize("sched", ["static", "dynamic"])
+def test_splitk_pending_error_refuses_next_run(sched):
+    """After a device error the next run is refused with ET_ERR_PENDING (the
+    failing kernel mirrors its status into mapped host memory) until
+    et_sync_status collects the error; then runs launch again."""
+    g = et.et_build_graph(et.ET_GRAPH_SPLITK, sched, 256, debug_flags=et.ET_DEBUG_BAD_COUNT, timeout_ms=50.0)
+    try:
+        A = dev(W.splitk_inputs(256))
+        B = torch.zeros((256, 4), device="cuda")
+        C = torch.zeros((256,), device="cuda")
+        et.et_run_splitk(g, A, 256, B, C)
+        torch.cuda.synchronize()      # the run has ended in its timeout; the error is not collected
+        with pytest.raises(et.EtError) as e:
+            et.et_run_splitk(g, A, 256, B, C)
+        assert e.value.status == et.ET_ERR_PENDING
+        assert et.et_sync_status(g) == et.ET_ERR_TIMEOUT
+        et.et_run_splitk(g, A, 256, B, C)   # launches again (and times out again: the count is still wrong)
+        assert et.et_sync_status(g) == et.ET_ERR_TIMEOUT
+    finally:
+        et.et_destroy_graph(g)

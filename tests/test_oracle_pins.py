@@ -209,3 +209,41 @@ def test_zipf_bias_recipe():
     assert np.all(b0 == 0)
     b = W.expert_bias(128, 1.2)
     assert np.allclose(np.sort(-b.astype(np.float64) / 1.2), np.log(np.arange(1, 129)), rtol=1e-6, atol=1e-6)
+
+
+# -------------------------------------------------------- failure / threads --
+
+def test_moe_grouped_rejects_malformed_grouping():
+    """A grouping that does not list every pair of topk under its own expert
+    is an error, not an all-zero output."""
+    d = W.moe_inputs(6, hidden=64, inter=32, E=4, zipf_s=0.0)
+    tk, w = oracle.topk_softmax(oracle.router_logits(d["X"], d["Wr"], d["bias"]), 2)
+    g = oracle.group(tk, 4, 128)
+    oracle.moe_grouped(d["X"], d["W1"], d["W2"], tk, w, g["indptr"], g["perm"])  # well formed: fine
+    cases = [
+        (g["indptr"], np.r_[g["perm"][1:], g["perm"][:1]]),        # pairs listed under the wrong expert
+        (g["indptr"], np.r_[g["perm"][:1], g["perm"][:-1]]),       # a pair listed twice, one missing
+        (np.r_[g["indptr"][:-1], g["indptr"][-1] - 1], g["perm"]),  # indptr does not cover every pair
+    ]
+    for ip, pm in cases:
+        with pytest.raises(ValueError):
+            oracle.moe_grouped(d["X"], d["W1"], d["W2"], tk, w, ip, pm)
+
+
+def test_results_do_not_depend_on_thread_count():
+    d = W.moe_inputs(9, hidden=128, inter=64, E=8, zipf_s=0.8)
+    before = oracle.get_threads()
+    outs = []
+    try:
+        for n in (1, 3):
+            oracle.set_threads(n)
+            lg = oracle.router_logits(d["X"], d["Wr"], d["bias"])
+            tk, w = oracle.topk_softmax(lg, 3)
+            g = oracle.group(tk, 8, 128)
+            y = oracle.moe_grouped(d["X"], d["W1"], d["W2"], tk, w, g["indptr"], g["perm"])
+            yt, _, _ = oracle.moe_per_token(d["X"], d["Wr"], d["bias"], d["W1"], d["W2"], list(range(9)), 3)
+            outs.append((lg, y, yt))
+    finally:
+        oracle.set_threads(before)
+    for a, b in zip(outs[0], outs[1]):
+        assert np.array_equal(a, b)

@@ -16,6 +16,11 @@ Recipe (numpy PCG64 ``default_rng(seed)``):
            0..E-1 (a Zipf(s) popularity prior on the experts; s = 0 gives
            zero bias)                                              seeds 100+log2(T) (1000+T when T is
            not a power of two), 20, 21, 22, 23
+  decode   X [B, hidden] ~ N(0,1); context lengths ~ U{512..4096} (the
+           new token's position); K and V caches [B, n_kv, max_ctx, hd]
+           ~ N(0,1) at the cached positions, zero beyond;
+           g1, gq, gk, g2 ~ N(1, 0.1); Wqkv [(n_q+2n_kv)*hd, hidden],
+           Wo [hidden, n_q*hd] ~ N(0, 0.02); Wgu, Wd as for the MLP   seeds 40+B, 41, 42, 43, 44..49, 12, 13
 """
 import math
 
@@ -85,4 +90,31 @@ def moe_inputs(T, hidden=2048, inter=768, E=128, zipf_s=1.2, weights=True):
     if weights:
         d["W1"] = _normal_bf16(np.random.default_rng(21), (E, 2 * inter, hidden), 0.0, 0.02)
         d["W2"] = _normal_bf16(np.random.default_rng(22), (E, hidden, inter), 0.0, 0.02)
+    return d
+
+
+def decode_inputs(B, hidden=4096, n_q=32, n_kv=8, hd=128, inter=14336, ctx_lo=512, ctx_hi=4096, max_ctx=None,
+                  weights=True):
+    """dict(X, pos, Kc, Vc[, g1, Wqkv, gq, gk, Wo, g2, Wgu, Wd]) for one decode
+    step of B requests; pos[b] = tokens already cached for request b."""
+    if max_ctx is None:
+        max_ctx = ctx_hi + 1
+    pos = np.random.default_rng(41).integers(ctx_lo, ctx_hi + 1, size=64 if B <= 64 else B)[:B].astype(np.int32)
+    Kc = np.zeros((B, n_kv, max_ctx, hd), np.uint16)
+    Vc = np.zeros((B, n_kv, max_ctx, hd), np.uint16)
+    rk, rv = np.random.default_rng(42), np.random.default_rng(43)
+    for b in range(B):
+        n = int(pos[b])
+        Kc[b, :, :n] = _normal_bf16(rk, (n_kv, n, hd), 0.0, 1.0)
+        Vc[b, :, :n] = _normal_bf16(rv, (n_kv, n, hd), 0.0, 1.0)
+    d = dict(X=_normal_bf16(np.random.default_rng(40 + B), (B, hidden), 0.0, 1.0), pos=pos, Kc=Kc, Vc=Vc)
+    if weights:
+        d["g1"] = _normal_bf16(np.random.default_rng(44), (hidden,), 1.0, 0.1)
+        d["Wqkv"] = _normal_bf16(np.random.default_rng(45), ((n_q + 2 * n_kv) * hd, hidden), 0.0, 0.02)
+        d["gq"] = _normal_bf16(np.random.default_rng(46), (hd,), 1.0, 0.1)
+        d["gk"] = _normal_bf16(np.random.default_rng(47), (hd,), 1.0, 0.1)
+        d["Wo"] = _normal_bf16(np.random.default_rng(48), (hidden, n_q * hd), 0.0, 0.02)
+        d["g2"] = _normal_bf16(np.random.default_rng(49), (hidden,), 1.0, 0.1)
+        d["Wgu"] = _normal_bf16(np.random.default_rng(12), (2 * inter, hidden), 0.0, 0.02)
+        d["Wd"] = _normal_bf16(np.random.default_rng(13), (hidden, inter), 0.0, 0.02)
     return d
