@@ -14,7 +14,7 @@ ranks).  The L2 is flushed before every step, outside the timed events.
 Several GPUs run independent replicas (the layer does not shard here).
 
 The line also carries a driver-timed `sweep` (T in {1, 16, 128, 1024, 4096}
-x static / dynamic / unfused schedules, Zipf 1.2, same graph and binary) and
+x static / dynamic / hybrid / unfused schedules, Zipf 1.2, same binary) and
 the CPU oracle timed on this host's cores (`cpu_baseline`: the whole layer,
 single thread and all threads, median of 3).
 
@@ -245,13 +245,13 @@ def gpu_arm(args, rank, world, local_rank):
 
 
 def run_sweep(args, et, g_dyn, t, dev, stream, flush):
-    """Device time of the layer over the token range and the three schedules
+    """Device time of the layer over the token range and the four schedules
     (same binary; one graph per schedule, max_T 4096), Zipf s = 1.2: median
     of `sweep_steps` launches, L2 flushed before each."""
     import torch
     hbm, tc, _ = load_peaks()
     graphs = {"dynamic": g_dyn}
-    for s in ("static", "unfused"):
+    for s in ("static", "hybrid", "unfused"):
         graphs[s] = et.et_build_graph(et.ET_GRAPH_MOE, s, max(4096, args.max_T), device=dev.index)
     out = []
     try:
@@ -285,7 +285,7 @@ def run_sweep(args, et, g_dyn, t, dev, stream, flush):
                 row["experts_touched"] = touched
             out.append(row)
     finally:
-        for s in ("static", "unfused"):
+        for s in ("static", "hybrid", "unfused"):
             et.et_destroy_graph(graphs[s])
     return {"zipf_s": args.zipf, "steps_per_point": args.sweep_steps, "timing": "median, L2 flushed before each launch",
             "points": out}
@@ -307,7 +307,22 @@ def other_arm(args):
         a = np.ascontiguousarray(a)
         return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
 
-    if args.workload == "mlp":
+    if args.workload == "decode":
+        B = args.B
+        d = W.decode_inputs(B)
+        wkeys = ("g1", "Wqkv", "gq", "gk", "Wo", "g2", "Wgu", "Wd")
+        t = {n: to_dev(d[n]) for n in wkeys + ("X", "pos", "Kc", "Vc")}
+        Y = torch.empty((B, 4096), dtype=torch.int16, device=dev)
+        sched = args.sched
+        g = et.et_build_graph(et.ET_GRAPH_DECODE, sched, 64)
+        run = lambda: et.et_run_decode(g, B, t["X"], t["pos"], t, t["Kc"], t["Vc"], Y)  # noqa: E731
+        wbytes = sum(d[n].nbytes for n in wkeys)
+        kv = int(np.sum(d["pos"].astype(np.int64) + 1)) * 8 * 128 * 2 * 2   # K and V read, new entry included
+        nbytes = wbytes + kv + B * 8 * 128 * 2 * 2 + 2 * B * 4096 * 2     # + appended K, V; X in, Y out
+        workload = ("Llama-3-8B-shaped decode layer B=%d (hidden 4096, 32/8 heads x 128, SwiGLU 14336, "
+                    "context %d..%d, mean %.0f), %s schedule" % (B, d["pos"].min(), d["pos"].max(),
+                                                                 d["pos"].mean(), sched))
+    elif args.workload == "mlp":
         B = args.B
         d = W.mlp_inputs(B)
         t = {n: to_dev(d[n]) for n in ("X", "gamma", "Wgu", "Wd")}
@@ -320,8 +335,11 @@ def other_arm(args):
         A = to_dev(W.splitk_inputs(2048))
         Bp = torch.zeros((2048, 4), device=dev)
         C = torch.zeros((2048,), device=dev)
-        g = et.et_build_graph(et.ET_GRAPH_SPLITK, args.sched, 2048)
-        run = lambda: et.et_run_splitk(g, A, 2048, Bp, C)
+        g = et.et_build_graph(et.ET_GRAPH_SPLITK, "static" if args.sched == "two_launch" else args.sched, 2048)
+        if args.sched == "two_launch":  # the kernel-per-operator control
+            run = lambda: et.et_run_splitk_two_launch(A, 2048, 128, 32, Bp, C)  # noqa: E731
+        else:
+            run = lambda: et.et_run_splitk(g, A, 2048, Bp, C)  # noqa: E731
         nbytes = 2048 * 128 * 4 + 2048 * 5 * 4
         workload = "split-K 2048 x 128 fp32, chunks of 32, %s schedule" % args.sched
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -341,7 +359,7 @@ def other_arm(args):
     if et.et_sync_status(g) != 0:
         raise RuntimeError("run reported a device error")
     et.et_destroy_graph(g)
-    ms = sum(times) / len(times)
+    ms = statistics.median(times)
     hbm, _, src = load_peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"workload": workload, "latency_us": round(ms * 1e3, 2), "value": round(gbs, 1), "unit": "GB/s",
@@ -445,13 +463,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--T", type=int, default=128)
     ap.add_argument("--max_T", type=int, default=4096)
-    ap.add_argument("--sched", default="dynamic", choices=["static", "dynamic", "unfused"])
+    ap.add_argument("--sched", default="dynamic", choices=["static", "dynamic", "unfused", "hybrid", "two_launch"],
+                    help="two_launch (split-K only): the kernel-per-operator control")
     ap.add_argument("--zipf", type=float, default=1.2)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="moe", choices=["moe", "mlp", "splitk"],
-                    help="moe (the benchmark line); mlp or splitk print a kernel timing line")
-    ap.add_argument("--B", type=int, default=1, help="decode MLP batch (--workload mlp)")
+    ap.add_argument("--workload", default="moe", choices=["moe", "mlp", "splitk", "decode"],
+                    help="moe (the benchmark line); mlp, splitk or decode print a kernel timing line")
+    ap.add_argument("--B", type=int, default=1, help="batch (--workload mlp or decode)")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false", help="skip the T x schedule sweep")
     ap.add_argument("--sweep-steps", type=int, default=50)
     args = ap.parse_args()

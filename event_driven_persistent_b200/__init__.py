@@ -20,10 +20,11 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 # ------------------------------------------------------------ constants --
 ET_OK, ET_ERR_INVALID, ET_ERR_CUDA, ET_ERR_TIMEOUT, ET_ERR_OOM, ET_ERR_UNSUPPORTED, ET_ERR_PENDING, ET_ERR_INTERNAL = range(8)
-ET_SCHED_STATIC, ET_SCHED_DYNAMIC, ET_SCHED_UNFUSED = 0, 1, 2
-ET_GRAPH_SPLITK, ET_GRAPH_MLP, ET_GRAPH_MOE = 0, 1, 2
+ET_SCHED_STATIC, ET_SCHED_DYNAMIC, ET_SCHED_UNFUSED, ET_SCHED_HYBRID = 0, 1, 2, 3
+ET_GRAPH_SPLITK, ET_GRAPH_MLP, ET_GRAPH_MOE, ET_GRAPH_DECODE = 0, 1, 2, 3
 ET_DEBUG_TRACE, ET_DEBUG_DELAY, ET_DEBUG_BAD_COUNT = 1, 2, 4
-SCHED = {"static": ET_SCHED_STATIC, "dynamic": ET_SCHED_DYNAMIC, "unfused": ET_SCHED_UNFUSED}
+SCHED = {"static": ET_SCHED_STATIC, "dynamic": ET_SCHED_DYNAMIC, "unfused": ET_SCHED_UNFUSED,
+         "hybrid": ET_SCHED_HYBRID}
 
 
 class EtError(RuntimeError):
@@ -37,14 +38,21 @@ class et_graph_desc(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "kind", "sched", "max_T", "hidden", "inter", "n_experts", "top_k", "splitk_cols", "splitk_chunk",
         "splitk_tile_rows")] + [("rms_eps", ctypes.c_float)] + [(n, ctypes.c_int) for n in (
-            "fetch_batch", "debug_flags", "device", "n_ctas")] + [("timeout_ms", ctypes.c_float)]
+            "fetch_batch", "debug_flags", "device", "n_ctas")] + [("timeout_ms", ctypes.c_float)] + [
+            (n, ctypes.c_int) for n in ("n_heads", "n_kv_heads", "head_dim", "max_ctx")] + [
+            ("rope_base", ctypes.c_float)]
 
 
 class et_graph_info(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "kind", "sched", "max_T", "n_ctas", "threads", "smem_bytes", "fetch_batch", "hidden", "inter",
         "n_experts", "top_k", "splitk_cols", "splitk_chunk", "splitk_tile_rows", "mlp_gu_tile", "mlp_down_tile",
-        "mlp_kchunk", "moe_tt", "moe_gt", "moe_tkt", "moe_bm", "moe_n1_tile", "moe_n2_tile", "moe_cb")]
+        "mlp_kchunk", "moe_tt", "moe_gt", "moe_tkt", "moe_bm", "moe_n1_tile", "moe_n2_tile", "moe_cb",
+        "dec_split", "dec_qkv_kc", "dec_o_kc")]
+
+
+class et_decode_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("g1", "Wqkv", "gq", "gk", "Wo", "g2", "Wgu", "Wd")]
 
 
 class et_trace_record(ctypes.Structure):
@@ -65,6 +73,8 @@ _sigs = {
     "et_run_mlp": ([_P, _I, _P, _P, _P, _P, _P, _P], _I),
     "et_run_moe": ([_P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], _I),
     "et_run_splitk_noalloc": ([_P, _I, _P, _P, _P], _I),
+    "et_run_splitk_two_launch": ([_P, _I, _I, _I, _P, _P, _P], _I),
+    "et_run_decode": ([_P, _I, _P, _P, ctypes.POINTER(et_decode_weights), _P, _P, _P, _P, _P], _I),
     "et_sync_status": ([_P, _P], _I),
     "et_get_trace": ([_P, _P, ctypes.c_size_t, ctypes.POINTER(_I)], _I),
     "et_get_info": ([_P, ctypes.POINTER(et_graph_info)], _I),
@@ -119,6 +129,12 @@ def et_run_splitk(g, A, n_rows, Bpart, C, stream=None):
     _check(_lib.et_run_splitk(g, _ptr(A), n_rows, _ptr(Bpart), _ptr(C), _stream(stream)), "et_run_splitk")
 
 
+def et_run_splitk_two_launch(A, n_rows, cols, chunk, Bpart, C, stream=None):
+    """Control: split-K as two plain kernel launches (partials, finals)."""
+    _check(_lib.et_run_splitk_two_launch(_ptr(A), n_rows, cols, chunk, _ptr(Bpart), _ptr(C), _stream(stream)),
+           "et_run_splitk_two_launch")
+
+
 def et_run_splitk_noalloc(A, n_rows, Bpart, C, stream=None):
     """Allocation-free split-K (synchronous); returns the status code."""
     return _lib.et_run_splitk_noalloc(_ptr(A), n_rows, _ptr(Bpart), _ptr(C), _stream(stream))
@@ -133,6 +149,15 @@ def et_run_moe(g, T, X, Wr, bias, W1, W2, Y, topk=None, topk_w=None, indptr=None
                stream=None):
     _check(_lib.et_run_moe(g, T, _ptr(X), _ptr(Wr), _ptr(bias), _ptr(W1), _ptr(W2), _ptr(Y), _ptr(topk),
                            _ptr(topk_w), _ptr(indptr), _ptr(perm), _ptr(logits), _stream(stream)), "et_run_moe")
+
+
+def et_run_decode(g, B, X, pos, w, Kc, Vc, Y, h1=None, stream=None):
+    """w: dict or object with g1, Wqkv, gq, gk, Wo, g2, Wgu, Wd (tensors or addresses)."""
+    ws = et_decode_weights()
+    for f, _ in et_decode_weights._fields_:
+        setattr(ws, f, _ptr(w[f] if isinstance(w, dict) else getattr(w, f)))
+    _check(_lib.et_run_decode(g, B, _ptr(X), _ptr(pos), ctypes.byref(ws), _ptr(Kc), _ptr(Vc), _ptr(Y), _ptr(h1),
+                              _stream(stream)), "et_run_decode")
 
 
 def et_sync_status(g, stream=None):

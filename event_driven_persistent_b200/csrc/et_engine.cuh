@@ -38,9 +38,14 @@ struct TaskDesc {
     int a_map, a_row0, a_row1;  // A: tensor map id, rows of the two 64-row boxes
     int b_map, b_row0;          // B: tensor map id, first row
     int n;                      // MMA N (multiple of 16, <= kMaxN)
-    int k0, nk;                 // first K element, number of 64-wide K stages
+    int k0, nk;                 // first K element, number of 128-wide K stages (stream: stages)
+    int stream;                 // 1 = stream task: warp 0 copies nk byte blocks into arena stages,
+                                //     the exec group consumes them (no tensor-core work)
+    uint32_t sbytes;            // stream: bytes reserved per stage (1 KB multiple)
+    uint32_t st0, off0;         // stream: global index and arena offset of the task's first stage
     int p[6];                   // workload-specific
 };
+
 
 struct SmemCtl {
     uint64_t full[kSlots];
@@ -76,6 +81,21 @@ struct Ctx {
     uint8_t* simt;       // CUDA-core task scratch
     SmemCtl* sc;
     int tid;             // exec-group thread index 0..127 (exec warps only)
+};
+
+// Defaults of the workload interface for what a workload does not use.
+struct WorkloadBase {
+    // stream tasks: stages that may be copied before the task's input wait,
+    // the bytes stage s delivers, and the copies of stage s into `dst`
+    // (completing on `bar`)
+    template <class P>
+    __device__ static int stream_prefetch(const P&, const TaskDesc&) { return 0; }
+    template <class P>
+    __device__ static uint32_t stream_bytes(const P&, const TaskDesc&, int) { return 0; }
+    template <class P>
+    __device__ static void stream_copy(const P&, const TaskDesc&, int, uint8_t*, uint64_t*, uint64_t) {}
+    template <class P>
+    __device__ static bool stream_exec(const P&, Ctx&, TaskDesc&) { return false; }
 };
 
 __device__ __forceinline__ void exec_bar() { named_bar_sync(1, kExecThreads); }
@@ -182,6 +202,31 @@ struct StageAlloc {
     }
 };
 
+// Stream tasks, exec group: wait for stage s of the task (all 128 threads
+// call; false on timeout/abort) and return its arena offset in *off.
+__device__ __forceinline__ bool stream_stage_wait(Ctx& x, const TaskDesc& d, int s, StageAlloc& a, uint32_t* off) {
+    const uint32_t g = d.st0 + (uint32_t)s;
+    const uint32_t slot = g % kSlots, par = (g / kSlots) & 1;
+    *off = a.next(d.sbytes);
+    if (x.tid == 0) x.sc->bcast[5] = mbar_wait(&x.sc->full[slot], par, x.ctl, x.timeout_ns, 925);
+    exec_bar();
+    const bool ok = x.sc->bcast[5] != 0;
+    if (ok)
+        while (!mbar_try_wait(&x.sc->full[slot], par)) {
+        }
+    return ok;
+}
+// ... and hand stage s back to the producer once every thread is done with it.
+__device__ __forceinline__ void stream_stage_release(Ctx& x, const TaskDesc& d, int s) {
+    exec_bar();
+    if (x.tid == 0) mbar_arrive(&x.sc->empty[(d.st0 + (uint32_t)s) % kSlots]);
+}
+__device__ __forceinline__ StageAlloc stream_alloc(const TaskDesc& d) {
+    StageAlloc a;
+    a.head = d.off0;
+    return a;
+}
+
 // Megakernel body.  W supplies the task semantics:
 //   W::fetch_init(p, idx)              initial dynamic task word for slot idx
 //   W::derive(p, x, word, d)           fill a TaskDesc (warp 0; may wait in
@@ -191,6 +236,11 @@ struct StageAlloc {
 //   W::a_map(p, id), W::b_map(p, id)   tensor maps
 //   W::epilogue(p, x, d, acc_taddr)    exec group, after the accumulator is ready
 //   W::simt(p, x, d)                   exec group, a CUDA-core task
+//   W::stream_prefetch / stream_copy   (stream tasks) warp 0, see WorkloadBase
+//   W::stream_exec(p, x, d)            exec group, a stream task (stream_stage_wait/release)
+// Task sources: static (this CTA's list), dynamic (the ready queue), or
+// hybrid: this CTA's list part A, then the ready queue until it is
+// exhausted, then its list part B.
 template <class W>
 __device__ __forceinline__ void megakernel_body(const typename W::Params& p, const RunArgs& ra) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -267,8 +317,9 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
         // are gathered through an index list, all 32 lanes issue the row copies.
         const uint64_t pol_w = policy_evict_first();
         const uint64_t pol_a = policy_evict_last();
-        int lpos = 0, lend = 0;
-        if (!x.dynamic) {
+        // phase 0: list part A; 1: ready queue; 2: list part B
+        int lpos = 0, lend = 0, phase = x.dynamic && !ra.hybrid ? 1 : 0;
+        if (phase == 0) {
             lpos = ra.lists.off[blockIdx.x];
             lend = ra.lists.off[blockIdx.x + 1];
         }
@@ -284,8 +335,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
         // the arena from the tail stage to the allocation head, so the new
         // stage can only collide with the oldest ones: consume (wait for)
         // tail stages until its slot and its bytes are free.  O(1) amortised.
-        auto reserve = [&](int n, uint32_t* slot_out, uint32_t* off_out) -> bool {
-            const uint32_t size = stage_bytes(n);
+        auto reserve = [&](uint32_t size, uint32_t* slot_out, uint32_t* off_out) -> bool {
             const uint32_t off = alloc.next(size);
             while (tail < nst) {
                 const uint32_t ts = tail % kSlots;
@@ -333,13 +383,24 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 d.valid = 0;
                 d.gemm = 0;
                 d.gather = 0;
+                d.stream = 0;
                 d.start = 0;
                 d.t_fetch = d.t_ready = d.t_acc = 0;
-                int r;
-                if (!x.dynamic) {
-                    r = lpos < lend ? 1 : 0;
-                    if (r) d.word = ra.lists.words[lpos++];
-                } else {
+                int r = 0;
+                for (;;) {
+                    if (phase != 1) {
+                        const uint32_t* words = phase == 0 ? ra.lists.words : ra.lists.words_b;
+                        r = lpos < lend ? 1 : 0;
+                        if (r) {
+                            d.word = words[lpos++];
+                            break;
+                        }
+                        if (phase == 0 && ra.hybrid) {
+                            phase = 1;
+                            continue;
+                        }
+                        break;
+                    }
                     if (qn == qe) {
                         qn = atom_add_relaxed(x.q.head, ra.fetch_batch);
                         qe = qn + ra.fetch_batch;
@@ -348,6 +409,13 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     r = q_resolve(x.q, qn, &w, [&](int i) { return W::fetch_init(p, i); }, ctl, x.timeout_ns);
                     ++qn;
                     if (r == 1) d.word = w;
+                    if (r == 0 && ra.hybrid && ra.lists.off_b) {
+                        phase = 2;
+                        lpos = ra.lists.off_b[blockIdx.x];
+                        lend = ra.lists.off_b[blockIdx.x + 1];
+                        continue;
+                    }
+                    break;
                 }
                 bool brk = r < 0;
                 if (!brk && (x.debug & ET_DEBUG_TRACE)) d.t_fetch = globaltimer();
@@ -364,7 +432,46 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             TaskDesc d = sc->pd;
             __syncwarp();
             if (brk) break;
-            if (r == 1 && d.valid && d.gemm) {
+            if (r == 1 && d.valid && d.stream) {
+                // stream task: stages that do not depend on the task's input
+                // events first, then the wait, then the rest
+                bool ok = true;
+                if (lane == 0) {
+                    const int fit = kArenaBytes / (int)d.sbytes - 1;
+                    int npre = W::stream_prefetch(p, d);
+                    npre = npre < fit ? npre : fit;
+                    npre = npre < kSlots - 1 ? npre : kSlots - 1;
+                    npre = npre < d.nk ? npre : d.nk;
+                    d.st0 = nst;
+                    {
+                        StageAlloc probe = alloc;  // where the first stage will land
+                        d.off0 = probe.head;
+                    }
+                    auto issue_s = [&](int st) -> bool {
+                        uint32_t sl, of;
+                        if (!reserve(d.sbytes, &sl, &of)) return false;
+                        mbar_arrive_expect_tx(&sc->full[sl], W::stream_bytes(p, d, st));
+                        ++armed[sl];
+                        W::stream_copy(p, d, st, arena + of, &sc->full[sl], pol_w);
+                        return true;
+                    };
+                    int s2 = 0;
+                    for (; s2 < npre && ok; ++s2) ok = issue_s(s2);
+                    if (ok) ok = W::gemm_wait(p, x, d);  // the task's input events
+                    if (ok && (x.debug & ET_DEBUG_TRACE)) {
+                        d.start = take_ticket(ctl);
+                        d.t_ready = globaltimer();
+                    }
+                    sc->ring[slot] = d;
+                    mbar_arrive(&sc->ring_full[slot]);
+                    for (; ok && s2 < d.nk; ++s2) ok = issue_s(s2);
+                    sc->pok = ok;
+                }
+                __syncwarp();
+                ok = sc->pok;
+                __syncwarp();
+                if (!ok) break;
+            } else if (r == 1 && d.valid && d.gemm) {
                 const CUtensorMap* am = W::a_map(p, d.a_map);
                 const uint32_t bbytes = 2u * (uint32_t)d.n * 128u;  // both K atoms
                 bool ok = true;
@@ -379,7 +486,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         uint32_t pslot[kSlots], poff[kSlots];
                         int s = 0;
                         for (; s < npre && ok; ++s) {
-                            ok = reserve(d.n, &pslot[s], &poff[s]);
+                            ok = reserve(stage_bytes(d.n), &pslot[s], &poff[s]);
                             if (ok) issue_a(pslot[s], poff[s], am, d, s, kAStageBytes + bbytes, pol_w);
                         }
                         if (ok) ok = W::gemm_wait(p, x, d);  // the task's input event
@@ -391,12 +498,13 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         sc->ring[slot] = d;
                         mbar_arrive(&sc->ring_full[slot]);
                         // 2. activation tiles of the prefetched stages
-                        for (int i = 0; ok && i < npre; ++i)
+                        for (int i = 0; ok && i < npre; ++i) {
                             issue_b(pslot[i], poff[i], bm, d, i, pol_a);
+                        }
                         // 3. the remaining stages, weights and activations together
                         for (; ok && s < d.nk; ++s) {
                             uint32_t sl, of;
-                            ok = reserve(d.n, &sl, &of);
+                            ok = reserve(stage_bytes(d.n), &sl, &of);
                             if (!ok) break;
                             issue_a(sl, of, am, d, s, kAStageBytes + bbytes, pol_w);
                             issue_b(sl, of, bm, d, s, pol_a);
@@ -431,7 +539,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     for (int s = 0; s < d.nk && ok; ++s) {
                         if (lane == 0) {
                             uint32_t sl = 0, of = 0;
-                            sc->pok = reserve(d.n, &sl, &of);
+                            sc->pok = reserve(stage_bytes(d.n), &sl, &of);
                             sc->pslot = sl;
                             sc->poff = of;
                         }
@@ -489,6 +597,10 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 TaskDesc d = sc->ring[slot];
                 mbar_arrive(&sc->ring_empty[slot]);
                 if (d.word == kExitWord) break;
+                if (d.valid && d.stream) {  // stages consumed by the exec group: keep the sequence
+                    for (int s = 0; s < d.nk; ++s, ++nst) alloc.next(d.sbytes);
+                    continue;
+                }
                 if (!(d.valid && d.gemm)) continue;
                 const uint32_t buf = g & 1;
                 if (!mbar_wait(&sc->acc_empty[buf], ((g >> 1) & 1) ^ 1, ctl, x.timeout_ns, 911)) break;
@@ -546,7 +658,9 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             if (d.word == kExitWord) break;
             if (!d.valid) continue;
             if (x.debug & ET_DEBUG_DELAY) debug_delay(d.word ^ (ra.epoch * 977u));
-            if (d.gemm) {
+            if (d.stream) {
+                if (!W::stream_exec(p, x, d)) break;
+            } else if (d.gemm) {
                 const uint32_t buf = g & 1;
                 const uint32_t par = (g >> 1) & 1;
                 if (x.tid == 0) sc->bcast[5] = mbar_wait(&sc->acc_full[buf], par, ctl, x.timeout_ns, 921);

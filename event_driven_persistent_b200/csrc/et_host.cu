@@ -17,10 +17,13 @@
 namespace et {
 cudaError_t splitk_setup(int* max_blocks_per_sm);
 cudaError_t launch_splitk(const SplitKParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
+cudaError_t launch_splitk_two(const float* A, int rows, int cols, int chunk, float* Bp, float* C, cudaStream_t s);
 cudaError_t mlp_setup(int* max_blocks_per_sm);
 cudaError_t launch_mlp(const MlpParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
 cudaError_t moe_setup(int* max_blocks_per_sm);
 cudaError_t launch_moe(const MoeParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
+cudaError_t decode_setup(int* max_blocks_per_sm);
+cudaError_t launch_decode(const DecodeParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
 }  // namespace et
 
 using namespace et;
@@ -83,6 +86,7 @@ struct MapCache {
 struct Slot {
     uint32_t word;
     float cost;
+    int part = 0;  // hybrid schedules: 0 = list part A (before the queue), 1 = part B (after it)
 };
 
 inline uint32_t tw(int op, int a, int b) {
@@ -130,21 +134,24 @@ struct et_graph {
     TraceRec* trace = nullptr;
     int trace_cap = 0;
     uint32_t epoch = 0;
-    // static lists: one CSR per bucket, concatenated
+    // static lists: one CSR per bucket (and list part), concatenated
     std::vector<int> bucket_T;
-    std::vector<size_t> off_at, words_at;
+    std::vector<size_t> off_at, words_at, off_b_at, words_b_at;
     int* lists_off = nullptr;
     uint32_t* lists_words = nullptr;
+    bool hybrid = false;  // the run uses list part A, the queue, then list part B
     std::vector<void*> allocs;
     // the last launched run (event-count introspection)
     int last_T = 0;
     SplitKParams last_sk;
     MlpParams last_mlp;
     MoeParams last_moe;
+    DecodeParams last_dec;
     // workload state
     SplitKParams sk;
     MlpParams mlp;
     MoeParams moe;
+    DecodeParams dec;
     MapCache mc[6];
     int bucket_of(int T) const {
         for (size_t i = 0; i < bucket_T.size(); ++i)
@@ -187,22 +194,27 @@ et_status galloc(et_graph* g, T** p, size_t n) {
 
 bool aligned16(const void* p) { return p && ((uintptr_t)p & 15) == 0; }
 
-// Build every bucket's lists with `gen(T_b, slots)`, upload them.
+// Build every bucket's lists with `gen(T_b, slots)`, upload them.  Hybrid
+// graphs keep a slot's part (A before the queue, B after it) as two lists
+// per CTA; the other schedules list every slot in one list, in order.
 et_status build_lists(et_graph* g, const std::function<void(int, std::vector<Slot>&)>& gen) {
     std::vector<int> all_off;
     std::vector<uint32_t> all_words;
     for (int T = 1;; T <<= 1) {
         int Tb = std::min(T, g->d.max_T);
-        std::vector<Slot> slots;
+        std::vector<Slot> slots, part_a, part_b;
         gen(Tb, slots);
-        std::vector<int> off;
-        std::vector<uint32_t> words;
-        assign(slots, g->n_ctas, off, words);
+        for (const Slot& sl : slots) (g->hybrid && sl.part == 1 ? part_b : part_a).push_back(sl);
         g->bucket_T.push_back(Tb);
-        g->off_at.push_back(all_off.size());
-        g->words_at.push_back(all_words.size());
-        for (int o : off) all_off.push_back(o);
-        all_words.insert(all_words.end(), words.begin(), words.end());
+        for (int part = 0; part < 2; ++part) {
+            std::vector<int> off;
+            std::vector<uint32_t> words;
+            assign(part == 0 ? part_a : part_b, g->n_ctas, off, words);
+            (part == 0 ? g->off_at : g->off_b_at).push_back(all_off.size());
+            (part == 0 ? g->words_at : g->words_b_at).push_back(all_words.size());
+            for (int o : off) all_off.push_back(o);
+            all_words.insert(all_words.end(), words.begin(), words.end());
+        }
         if (Tb >= g->d.max_T) break;
     }
     ET_TRY(galloc(g, &g->lists_off, all_off.size()));
@@ -229,7 +241,8 @@ RunArgs run_args(et_graph* g, int T, int n_init, int total_static) {
     ra.epoch = ep;
     ra.n_init = n_init;
     ra.total_static = total_static;
-    ra.dynamic = g->d.sched == ET_SCHED_DYNAMIC;
+    ra.dynamic = g->d.sched == ET_SCHED_DYNAMIC || g->hybrid;
+    ra.hybrid = g->hybrid;
     ra.fetch_batch = g->d.fetch_batch;
     ra.debug = g->d.debug_flags;
     ra.trace = g->trace;
@@ -237,6 +250,10 @@ RunArgs run_args(et_graph* g, int T, int n_init, int total_static) {
     int b = g->bucket_of(T);
     ra.lists.off = g->lists_off + g->off_at[b];
     ra.lists.words = g->lists_words + g->words_at[b];
+    if (g->hybrid) {
+        ra.lists.off_b = g->lists_off + g->off_b_at[b];
+        ra.lists.words_b = g->lists_words + g->words_b_at[b];
+    }
     ra.timeout_ns = (unsigned long long)((double)g->d.timeout_ms * 1e6);
     return ra;
 }
@@ -300,7 +317,8 @@ et_status build_splitk(et_graph* g) {
         int nt = cdiv(Tb, d.splitk_tile_rows);
         for (int i = 0; i < nt; ++i)
             for (int j = 0; j < nch; ++j) s.push_back({tw(ET_OP_SK_PARTIAL, i, j), 1.0f});
-        for (int i = 0; i < nt; ++i) s.push_back({tw(ET_OP_SK_FINAL, i, 0), 0.5f});
+        if (!g->hybrid)  // hybrid: a final task is queued by the partial that completes its event
+            for (int i = 0; i < nt; ++i) s.push_back({tw(ET_OP_SK_FINAL, i, 0), 0.5f});
     });
 }
 
@@ -338,7 +356,7 @@ et_status build_mlp(et_graph* g) {
     g->qcap = d.max_T + p.n_gu + p.n_m * p.n_c + p.n_m + g->n_ctas * d.fetch_batch + 64;
     ET_TRY(galloc(g, &p.xn, (size_t)p.maxB * p.hidden));
     ET_TRY(galloc(g, &p.h, (size_t)p.maxB * p.inter));
-    ET_TRY(galloc(g, &p.part, (size_t)p.n_c * p.maxB * p.hidden));
+    ET_TRY(galloc(g, &p.yacc, (size_t)p.maxB * p.hidden));
     if (!make_map(&p.tm_xn, p.xn, p.maxB, p.hidden, 16)) return ET_ERR_CUDA;
     if (!make_map(&p.tm_h, p.h, p.maxB, p.inter, 16)) return ET_ERR_CUDA;
     int mb = 0;
@@ -454,6 +472,7 @@ et_status build_moe(et_graph* g) {
         const float c_rt = (float)p.E * p.hidden * 2 / m.n_kc / 1024.f;
         for (int j = 0; j < m.n_tk; ++j)
             for (int c = 0; c < m.n_kc; ++c) s.push_back({tw(ET_OP_MOE_ROUTER, j, c), c_rt});
+        if (g->hybrid) return;  // grouping, expert stages and combine go through the queue
         s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 8.f});
         if (m.n_tt > 1)
             for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_GROUP, t, 0), 8.f});
@@ -462,6 +481,115 @@ et_status build_moe(et_graph* g) {
         for (int f = 0; f < m.f_max; ++f)
             for (int n = 0; n < p.n_n2; ++n) s.push_back({tw(ET_OP_MOE_S2, f, n), c_s2});
         for (int b = 0; b < m.n_cb; ++b) s.push_back({tw(ET_OP_MOE_COMBINE, b, 0), 2.f});
+    });
+}
+
+// --------------------------------------------------------- decode layer ----
+constexpr int kDecSplit = 256;  // keys per attention split task
+
+et_status build_decode(et_graph* g) {
+    et_graph_desc& d = g->d;
+    if (d.hidden <= 0) d.hidden = 4096;
+    if (d.inter <= 0) d.inter = 14336;
+    if (d.n_heads <= 0) d.n_heads = 32;
+    if (d.n_kv_heads <= 0) d.n_kv_heads = 8;
+    if (d.head_dim <= 0) d.head_dim = 128;
+    if (d.max_ctx <= 0) d.max_ctx = 4097;
+    if (d.rope_base <= 0.f) d.rope_base = 500000.f;
+    if (d.rms_eps <= 0.f) d.rms_eps = 1e-5f;
+    if (d.fetch_batch <= 0) d.fetch_batch = 1;
+    if (d.max_T > kMaxN) return ET_ERR_UNSUPPORTED;  // one token tile
+    if (d.head_dim != 128 || d.n_heads % d.n_kv_heads || d.n_heads / d.n_kv_heads > 4) return ET_ERR_UNSUPPORTED;
+    if (d.hidden % 1024 || d.hidden > 4096 || d.inter % 128) return ET_ERR_UNSUPPORTED;
+    DecodeParams& p = g->dec;
+    memset(&p, 0, sizeof(p));
+    p.maxB = d.max_T;
+    p.hidden = d.hidden;
+    p.inter = d.inter;
+    p.nq = d.n_heads;
+    p.nkv = d.n_kv_heads;
+    p.hd = d.head_dim;
+    p.grp = p.nq / p.nkv;
+    p.max_ctx = d.max_ctx;
+    p.split = kDecSplit;
+    p.s_max = cdiv(d.max_ctx, kDecSplit);
+    p.eps = d.rms_eps;
+    p.rope_base = (double)d.rope_base;
+    p.n_heads = p.nq + 2 * p.nkv;
+    const int kt = p.hidden / kTileK;
+    p.n_kc = kt % 4 == 0 ? 4 : (kt % 2 == 0 ? 2 : 1);
+    p.o_kc = p.grp * p.hd;
+    p.gu_tile = 64;
+    p.kchunk = d.inter % 1024 == 0 ? 1024 : (d.inter % 256 == 0 ? 256 : 128);
+    p.n_gu = d.inter / p.gu_tile;
+    p.n_m = d.hidden / 128;
+    p.n_c = d.inter / p.kchunk;
+    p.gu_per_chunk = p.kchunk / p.gu_tile;
+    p.sched = d.sched;
+    p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
+    const int nq_rows = p.maxB * p.nkv;
+    if (nq_rows > 0xFFFF || p.s_max > 0x3FF || p.n_heads > 0xFFFF || p.n_c > 0x3FF || p.nkv > 0x3FF)
+        return ET_ERR_UNSUPPORTED;
+    int ev = kCtrFirstEvent;
+    p.ev_n1 = ev++;
+    p.ev_qkv = ev;
+    ev += p.n_heads;
+    p.ev_g = ev;
+    ev += p.nkv;
+    p.ev_att = ev;
+    ev += p.maxB * p.nkv;
+    p.ev_ag = ev;
+    ev += p.nkv;
+    p.ev_o = ev++;
+    p.ev_n2 = ev++;
+    p.ev_h = ev;
+    ev += p.n_c;
+    p.ev_y = ev;
+    ev += p.n_m;
+    p.ev_branch_all = ev++;
+    p.ev_merge_all = ev++;
+    p.ev_gu_all = ev++;
+    p.ev_down_all = ev++;
+    g->n_ctr = ev;
+    g->qcap = p.n_heads * p.n_kc + p.nkv * p.maxB * p.s_max + p.n_m * p.nkv + p.maxB + p.n_gu + p.n_m * p.n_c +
+              p.n_m + g->n_ctas * d.fetch_batch + 64;
+    const size_t rows = (size_t)std::max(p.maxB, 16);  // at least one 16-row TMA box
+    ET_TRY(galloc(g, &p.xn, rows * p.hidden));
+    ET_TRY(galloc(g, &p.qkvacc, (size_t)p.maxB * p.n_heads * p.hd));
+    ET_TRY(galloc(g, &p.q, (size_t)p.maxB * p.nq * p.hd));
+    ET_TRY(galloc(g, &p.part, (size_t)p.maxB * p.nkv * p.s_max * p.grp * (p.hd + 2)));
+    ET_TRY(galloc(g, &p.attn, rows * p.nq * p.hd));
+    ET_TRY(galloc(g, &p.h1acc, (size_t)p.maxB * p.hidden));
+    ET_TRY(galloc(g, &p.h1, (size_t)p.maxB * p.hidden));
+    ET_TRY(galloc(g, &p.xn2, rows * p.hidden));
+    ET_TRY(galloc(g, &p.hm, rows * p.inter));
+    ET_TRY(galloc(g, &p.yacc, (size_t)p.maxB * p.hidden));
+    if (!make_map(&p.tm_xn, p.xn, rows, p.hidden, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_attn, p.attn, rows, (uint64_t)p.nq * p.hd, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_xn2, p.xn2, rows, p.hidden, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_hm, p.hm, rows, p.inter, 16)) return ET_ERR_CUDA;
+    int mb = 0;
+    ET_CU(decode_setup(&mb));
+    if (mb < 1) return ET_ERR_UNSUPPORTED;
+    // cost ~ KB a task streams
+    const float c_qkv = 128.f * p.hidden / p.n_kc * 2 / 1024.f, c_att = 2.f * kDecSplit * 256 / 1024.f,
+                c_o = 128.f * p.o_kc * 2 / 1024.f, c_gu = 2.f * p.gu_tile * p.hidden * 2 / 1024.f,
+                c_dn = 128.f * p.kchunk * 2 / 1024.f;
+    return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
+        for (int b = 0; b < Tb; ++b) s.push_back({tw(ET_OP_DEC_NORM1, b, 0), 1.f, 0});
+        for (int n = 0; n < p.n_heads; ++n)
+            for (int c = 0; c < p.n_kc; ++c) s.push_back({tw(ET_OP_DEC_QKV, n, c), c_qkv, 0});
+        if (!g->hybrid)  // hybrid: the splits are queued once their group's branches are done
+            for (int s2 = 0; s2 < p.s_max; ++s2)
+                for (int b = 0; b < Tb; ++b)
+                    for (int gg = 0; gg < p.nkv; ++gg) s.push_back({tw(ET_OP_DEC_ATTN, b * p.nkv + gg, s2), c_att, 0});
+        for (int c = 0; c < p.nkv; ++c)
+            for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_DEC_OPROJ, m, c), c_o, 1});
+        for (int b = 0; b < Tb; ++b) s.push_back({tw(ET_OP_DEC_NORM2, b, 0), 1.f, 1});
+        for (int n = 0; n < p.n_gu; ++n) s.push_back({tw(ET_OP_DEC_GATEUP, n, 0), c_gu, 1});
+        for (int c = 0; c < p.n_c; ++c)
+            for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_DEC_DOWN, m, c), c_dn, 1});
+        for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_DEC_RED, m, 0), 2.f, 1});
     });
 }
 
@@ -489,7 +617,7 @@ const char* et_status_str(et_status s) {
 et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     if (!desc || !out) return ET_ERR_INVALID;
     *out = nullptr;
-    if (desc->max_T < 1 || desc->kind < 0 || desc->kind > 2 || desc->sched < 0 || desc->sched > 2)
+    if (desc->max_T < 1 || desc->kind < 0 || desc->kind > 3 || desc->sched < 0 || desc->sched > 3)
         return ET_ERR_INVALID;
     et_graph* g = new et_graph();
     g->d = *desc;
@@ -505,10 +633,13 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     g->dev = desc->device;
     g->n_sm = prop.multiProcessorCount;
     g->n_ctas = desc->n_ctas > 0 ? std::min(desc->n_ctas, g->n_sm) : g->n_sm;
+    // the decode MLP has no irregular operator: its hybrid schedule is the static one
+    g->hybrid = desc->sched == ET_SCHED_HYBRID && desc->kind != ET_GRAPH_MLP;
     et_status st = ET_ERR_INVALID;
     if (desc->kind == ET_GRAPH_SPLITK) st = build_splitk(g);
     else if (desc->kind == ET_GRAPH_MLP) st = build_mlp(g);
-    else st = build_moe(g);
+    else if (desc->kind == ET_GRAPH_MOE) st = build_moe(g);
+    else st = build_decode(g);
     if (st != ET_OK) return fail(st);
     // common workspace
     if ((st = galloc(g, &g->ctl, 1)) != ET_OK) return fail(st);
@@ -558,6 +689,14 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
         in.moe_n2_tile = g->moe.n2_tile;
         in.moe_cb = moe_cb_for(g->d.max_T);
     }
+    if (desc->kind == ET_GRAPH_DECODE) {
+        in.dec_split = g->dec.split;
+        in.dec_qkv_kc = g->dec.n_kc;
+        in.dec_o_kc = g->dec.o_kc;
+        in.mlp_gu_tile = g->dec.gu_tile;
+        in.mlp_down_tile = 128;
+        in.mlp_kchunk = g->dec.kchunk;
+    }
     *out = g;
     return ET_OK;
 }
@@ -591,11 +730,20 @@ et_status et_run_splitk(et_graph* g, const float* A, int n_rows, float* Bpart, f
     p.rows = n_rows;
     p.n_tiles = cdiv(n_rows, p.tile_rows);
     ET_TRY(pre_run(g, s));
-    const int n_init = p.n_tiles * p.n_chunks;
+    const int n_init = g->hybrid ? 0 : p.n_tiles * p.n_chunks;  // hybrid: partials are listed
     RunArgs ra = run_args(g, n_rows, n_init, n_init + p.n_tiles);
     ET_TRY(launched(g, launch_splitk(p, ra, g->n_ctas, s)));
     g->last_T = n_rows;
     g->last_sk = p;
+    return ET_OK;
+}
+
+et_status et_run_splitk_two_launch(const float* A, int n_rows, int cols, int chunk, float* Bpart, float* C,
+                                   void* stream) {
+    if (n_rows < 0 || cols < 1 || chunk < 1) return ET_ERR_INVALID;
+    if (n_rows == 0) return ET_OK;
+    if (!aligned16(A) || !aligned16(Bpart) || !aligned16(C)) return ET_ERR_INVALID;
+    ET_CU(launch_splitk_two(A, n_rows, cols, chunk, Bpart, C, (cudaStream_t)stream));
     return ET_OK;
 }
 
@@ -656,10 +804,45 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
     p.n_cb = cdiv(T, p.cb);
     p.f_max = mb.f_max;
     ET_TRY(pre_run(g, s));
-    RunArgs ra = run_args(g, T, p.n_tk * p.n_kc, 0);
+    RunArgs ra = run_args(g, T, g->hybrid ? 0 : p.n_tk * p.n_kc, 0);  // hybrid: router tasks are listed
     ET_TRY(launched(g, launch_moe(p, ra, g->n_ctas, s)));
     g->last_T = T;
     g->last_moe = p;
+    return ET_OK;
+}
+
+et_status et_run_decode(et_graph* g, int B, const uint16_t* X, const int32_t* pos, const et_decode_weights* w,
+                        uint16_t* Kc, uint16_t* Vc, uint16_t* Y, uint16_t* h1, void* stream) {
+    if (!g || g->d.kind != ET_GRAPH_DECODE || !w) return ET_ERR_INVALID;
+    if (B < 1 || B > g->d.max_T) return ET_ERR_INVALID;
+    if (!aligned16(X) || !aligned16(pos) || !aligned16(w->g1) || !aligned16(w->Wqkv) || !aligned16(w->gq) ||
+        !aligned16(w->gk) || !aligned16(w->Wo) || !aligned16(w->g2) || !aligned16(w->Wgu) || !aligned16(w->Wd) ||
+        !aligned16(Kc) || !aligned16(Vc) || !aligned16(Y) || (h1 && !aligned16(h1)))
+        return ET_ERR_INVALID;
+    cudaStream_t s = (cudaStream_t)stream;
+    ET_CU(cudaSetDevice(g->dev));
+    DecodeParams& p = g->dec;
+    if (!g->mc[0].get(&p.tm_wqkv, w->Wqkv, (uint64_t)p.n_heads * p.hd, p.hidden, 64)) return ET_ERR_CUDA;
+    if (!g->mc[1].get(&p.tm_wo, w->Wo, p.hidden, (uint64_t)p.nq * p.hd, 64)) return ET_ERR_CUDA;
+    if (!g->mc[2].get(&p.tm_wgu, w->Wgu, 2ull * p.inter, p.hidden, 64)) return ET_ERR_CUDA;
+    if (!g->mc[3].get(&p.tm_wd, w->Wd, p.hidden, p.inter, 64)) return ET_ERR_CUDA;
+    p.X = X;
+    p.pos = pos;
+    p.g1 = w->g1;
+    p.gq = w->gq;
+    p.gk = w->gk;
+    p.g2 = w->g2;
+    p.Kc = Kc;
+    p.Vc = Vc;
+    p.Y = Y;
+    p.out_h1 = h1;
+    p.out_q = nullptr;
+    p.B = B;
+    ET_TRY(pre_run(g, s));
+    RunArgs ra = run_args(g, B, g->d.sched == ET_SCHED_DYNAMIC ? B : 0, 0);
+    ET_TRY(launched(g, launch_decode(p, ra, g->n_ctas, s)));
+    g->last_T = B;
+    g->last_dec = p;
     return ET_OK;
 }
 
@@ -675,6 +858,14 @@ et_status et_sync_status(et_graph* g, void* stream) {
     ET_TRY(reset_ctl(g));
     ET_CU(cudaMemset(g->ctr[0], 0, g->n_ctr * sizeof(int)));
     ET_CU(cudaMemset(g->ctr[1], 0, g->n_ctr * sizeof(int)));
+    if (g->d.kind == ET_GRAPH_MLP)  // sums kept zero between runs
+        ET_CU(cudaMemset(g->mlp.yacc, 0, (size_t)g->mlp.maxB * g->mlp.hidden * sizeof(float)));
+    if (g->d.kind == ET_GRAPH_DECODE) {
+        const DecodeParams& p = g->dec;
+        ET_CU(cudaMemset(p.qkvacc, 0, (size_t)p.maxB * p.n_heads * p.hd * sizeof(float)));
+        ET_CU(cudaMemset(p.h1acc, 0, (size_t)p.maxB * p.hidden * sizeof(float)));
+        ET_CU(cudaMemset(p.yacc, 0, (size_t)p.maxB * p.hidden * sizeof(float)));
+    }
     if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc) {
         ET_CU(cudaMemset(g->moe.Yacc, 0, (size_t)g->moe.maxT * g->moe.hidden * sizeof(float)));
         ET_CU(cudaMemset(g->moe.lacc, 0, (size_t)g->moe.maxT * g->moe.E * sizeof(float)));
@@ -718,6 +909,21 @@ et_status et_get_event_counts(et_graph* g, et_event_count* buf, int cap, int* n_
         for (int i = 0; i < p.n_m; ++i) add(ET_EV_MLP_Y, i, p.ev_y + i);
         add(ET_EV_MLP_GU_ALL, 0, p.ev_gu_all);
         add(ET_EV_MLP_DOWN_ALL, 0, p.ev_down_all);
+    } else if (g->d.kind == ET_GRAPH_DECODE) {
+        const DecodeParams& p = g->last_dec;
+        add(ET_EV_DEC_N1, 0, p.ev_n1);
+        for (int n = 0; n < p.n_heads; ++n) add(ET_EV_DEC_QKV, n, p.ev_qkv + n);
+        for (int gg = 0; gg < p.nkv; ++gg) add(ET_EV_DEC_G, gg, p.ev_g + gg);
+        for (int i = 0; i < p.B * p.nkv; ++i) add(ET_EV_DEC_ATT, i, p.ev_att + i);
+        for (int gg = 0; gg < p.nkv; ++gg) add(ET_EV_DEC_AG, gg, p.ev_ag + gg);
+        add(ET_EV_DEC_O, 0, p.ev_o);
+        add(ET_EV_DEC_N2, 0, p.ev_n2);
+        for (int c = 0; c < p.n_c; ++c) add(ET_EV_DEC_H, c, p.ev_h + c);
+        for (int m = 0; m < p.n_m; ++m) add(ET_EV_DEC_Y, m, p.ev_y + m);
+        add(ET_EV_DEC_BRANCH_ALL, 0, p.ev_branch_all);
+        add(ET_EV_DEC_MERGE_ALL, 0, p.ev_merge_all);
+        add(ET_EV_DEC_GU_ALL, 0, p.ev_gu_all);
+        add(ET_EV_DEC_DOWN_ALL, 0, p.ev_down_all);
     } else {
         const MoeParams& p = g->last_moe;
         for (int j = 0; j < p.n_tk; ++j) add(ET_EV_MOE_RT, j, p.ev_rt + j);

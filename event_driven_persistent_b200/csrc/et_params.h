@@ -35,7 +35,7 @@ struct MlpParams {
     const uint16_t* gamma;
     uint16_t* xn;
     uint16_t* h;
-    float* part;         // [n_c, maxB, H] fp32 partial sums of the down GEMM
+    float* yacc;         // [maxB, H] fp32 sums of the down GEMM's K chunks (zero between runs)
     uint16_t* Y;
     int B, hidden, inter, maxB;
     float eps;
@@ -91,6 +91,50 @@ struct MoeParams {
     int ev_rt, ev_tk, ev_sc, ev_grp, ev_exp, ev_s1, ev_cb, ev_s1_all, ev_s2_all;
     int ev_gcnt;        // counter-set block [n_tt, E]: pairs of 128-token tile g per expert
     int sched;          // et_sched
+    int bad_count;
+};
+
+// ------------------------------------------------------------ decode layer
+// One decode step of a transformer layer (B requests, one new token each).
+// Tasks: N1(b) norm; QKV(n, c) head tile n, K chunk c (the chunk completing
+// a head runs its branch: Q norm + RoPE, K norm + RoPE + cache append, V
+// cache append); ATTN(b*nkv + g, s) split s of request b, KV head g (a
+// stream task; the split completing (b, g) merges the splits); OPROJ(m, c)
+// output tile m, K chunk = KV group c; N2(b) residual + norm; GU(n);
+// DOWN(m, c); RED(m) residual + output.
+enum { DEC_MAP_WQKV = 0, DEC_MAP_WO = 1, DEC_MAP_WGU = 2, DEC_MAP_WD = 3,
+       DEC_MAP_XN = 4, DEC_MAP_ATTN = 5, DEC_MAP_XN2 = 6, DEC_MAP_HM = 7 };
+struct DecodeParams {
+    CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd;   // weights, box 64 x 64
+    CUtensorMap tm_xn, tm_attn, tm_xn2, tm_hm;   // workspace activations, box 64 x 16
+    // inputs / outputs
+    const uint16_t* X;
+    const int32_t* pos;        // [B] tokens already cached per request (= the new token's position)
+    const uint16_t *g1, *gq, *gk, *g2;
+    uint16_t *Kc, *Vc;         // [maxB, nkv, max_ctx, hd] caches (appended in place)
+    uint16_t* Y;
+    uint16_t* out_h1;          // optional [B, H] attention-block output (residual stream)
+    uint16_t* out_q;           // optional [B, nq*hd] rotated queries
+    // workspace
+    uint16_t* xn;              // [maxB, H]
+    float* qkvacc;             // [maxB, nqkv*hd] K-chunk sums (zero between runs)
+    uint16_t* q;               // [maxB, nq, hd] rotated queries
+    float* part;               // [maxB*nkv, S_max, grp, hd + 2] split partials (o, m, l)
+    uint16_t* attn;            // [maxB, nq*hd] attention output (o-proj B operand)
+    float* h1acc;              // [maxB, H] o-proj sums (zero between runs)
+    uint16_t* h1;              // [maxB, H]
+    uint16_t* xn2;             // [maxB, H]
+    uint16_t* hm;              // [maxB, I]
+    float* yacc;               // [maxB, H] down-projection sums (zero between runs)
+    int B, maxB, hidden, inter, nq, nkv, hd, grp, max_ctx, split, s_max;
+    float eps;
+    double rope_base;
+    int n_kc, n_heads;         // QKV K chunks, head tiles (nq + 2 nkv)
+    int gu_tile, kchunk, n_gu, n_m, n_c, gu_per_chunk, o_kc;  // MLP tiles; o-proj K chunk (grp*hd)
+    // events
+    int ev_n1, ev_qkv, ev_g, ev_att, ev_ag, ev_o, ev_n2, ev_h, ev_y;
+    int ev_branch_all, ev_merge_all, ev_gu_all, ev_down_all;
+    int sched;
     int bad_count;
 };
 

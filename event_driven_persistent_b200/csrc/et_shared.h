@@ -21,6 +21,7 @@ constexpr int kAtomK = 64;         // K elements per swizzle atom (one 128-byte 
 // 1 KB), so tasks with few token rows keep more weight bytes in flight
 // (11 stages at N = 16, 6 at N = 128).  kSlots mbarrier pairs track stages.
 constexpr int kSlots = 12;
+
 constexpr int kArenaBytes = 208 * 1024;
 constexpr int kAAtomBytes = 128 * 128;   // weight tile of one atom: 128 rows x 128 B
 constexpr int kAStageBytes = 2 * kAAtomBytes;
@@ -33,10 +34,13 @@ constexpr int kCtlBytes = 2048;          // mbarriers, task ring, broadcast word
 constexpr int kSmemBytes = 1024 /*align slack*/ + kArenaBytes + kScratchBytes + kCtlBytes;
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
-// Per-bucket static task lists: CSR over CTAs.
+// Per-bucket static task lists: CSR over CTAs.  Hybrid schedules have a
+// second list per CTA (part B), run after the ready queue is exhausted.
 struct StaticLists {
     const int* off;    // [n_ctas + 1]
     const uint32_t* words;
+    const int* off_b;  // [n_ctas + 1] or null
+    const uint32_t* words_b;
 };
 
 // Device control block of a graph (lives in its workspace).
@@ -61,7 +65,8 @@ struct RunArgs {
     uint32_t epoch;            // run number, >= 1
     int n_init;                // dynamic: initial tasks (implicit slots)
     int total_static;          // dynamic: task count when known at launch (else 0)
-    int dynamic;
+    int dynamic;               // 1 = ready queue (alone, or between the list parts when hybrid)
+    int hybrid;                // 1 = list part A, then the queue, then list part B
     int fetch_batch;
     int debug;
     TraceRec* trace;

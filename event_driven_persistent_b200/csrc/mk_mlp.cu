@@ -11,8 +11,8 @@
 //   E_norm          --"->n"-->   GU n                (64 gate + 64 up rows)
 //   GU n            --"n->c"-->  E_h[c] [kchunk/64]  (c = 64n / kchunk)
 //   E_h[c]          --"mc->c"--> DOWN (m, c)         (128 output rows, K chunk c)
-//   DOWN (m, c)     --"mc->m"--> E_y[m] [#chunks]
-//   E_y[m]          --"m->m"-->  RED m
+//   DOWN (m, c)     --"mc->m"--> E_y[m] [#chunks]   (partial sums added at L2 into yacc)
+//   E_y[m]          --"m->m"-->  RED m               (Y = bf16(yacc), yacc back to zero)
 // GEMMs run on tcgen05 with swap-AB: the weight rows are the M = 128 side,
 // the B tokens (rounded up to 16) are N, so one tile shape serves every B.
 #include <cuda_bf16.h>
@@ -25,8 +25,11 @@ namespace et {
 __device__ __forceinline__ uint16_t bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
 __device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+__device__ __forceinline__ void red_add(float* p, float v) {
+    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
 
-struct Mlp {
+struct Mlp : WorkloadBase {
     using Params = MlpParams;
     static constexpr bool kGemm = true;
 
@@ -123,9 +126,10 @@ struct Mlp {
                 group_push(x, p.n_m, [&](int m) { return task_word(ET_OP_MLP_DOWN, m, cc); });
             }
         } else {
-            // DOWN: row r = output column a*128 + r; columns = tokens
+            // DOWN: row r = output column a*128 + r; columns = tokens.  The
+            // K chunk's partial sums are added at L2 (a warp adds 32
+            // consecutive columns of one token per instruction).
             const int col = a * p.down_tile + r;
-            float* part = p.part + (size_t)c * p.maxB * p.hidden;
             for (int c0 = 0; c0 < d.n; c0 += 16) {
                 float v[16];
                 acc_load16(taddr, c0, v);
@@ -133,7 +137,7 @@ struct Mlp {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int b = c0 + i;
-                    if (b < p.B) part[(size_t)b * p.hidden + col] = v[i];
+                    if (b < p.B) red_add(p.yacc + (size_t)b * p.hidden + col, v[i]);
                 }
             }
             int* ev = x.ctr + (p.unfused ? p.ev_down_all : p.ev_y + a);
@@ -190,9 +194,9 @@ struct Mlp {
             for (int j = x.tid; j < p.down_tile; j += kExecThreads) {
                 const int col = a * p.down_tile + j;
                 for (int b = 0; b < p.B; ++b) {
-                    float s = 0.f;
-                    for (int c = 0; c < p.n_c; ++c) s += p.part[((size_t)c * p.maxB + b) * p.hidden + col];
-                    p.Y[(size_t)b * p.hidden + col] = bf16_bits(s);
+                    const size_t i = (size_t)b * p.hidden + col;
+                    p.Y[i] = bf16_bits(__ldcg(p.yacc + i));
+                    __stcg(p.yacc + i, 0.f);
                 }
             }
             group_finish_notify(x, d, nullptr, 0, 0);

@@ -66,7 +66,7 @@ __device__ __forceinline__ int exec_scan(int v, int tid, int* tmp, int* total) {
 }
 }  // namespace
 
-struct Moe {
+struct Moe : WorkloadBase {
     using Params = MoeParams;
     static constexpr bool kGemm = true;
 
@@ -472,7 +472,10 @@ struct Moe {
             atomicAdd(&sm.hist[e], 1);
         }
         exec_bar();
-        if (x.tid < p.E && sm.hist[x.tid] > 0) atomicAdd(x.ctr + p.ev_gcnt + tile * p.E + x.tid, sm.hist[x.tid]);
+        // per-tile pair counts (several grouping tiles only: with one tile the
+        // scan counts the pairs from the picks it loads anyway)
+        if (p.n_tt > 1 && x.tid < p.E && sm.hist[x.tid] > 0)
+            atomicAdd(x.ctr + p.ev_gcnt + tile * p.E + x.tid, sm.hist[x.tid]);
         const bool fired = group_finish_notify(x, d, x.ctr + p.ev_tk, 1, p.n_tk);
         if (fired && x.dynamic) {
             // this task completed E_tk: run the scan task here
@@ -527,7 +530,9 @@ struct Moe {
             // queued tasks of the run: router chunks, group (several tiles),
             // stage 1 and 2, combine (the scan runs inline); published once
             // the scan has queued its successors (publish_total)
-            sm.misc[6] = p.n_tk * p.n_kc + (p.n_tt > 1 ? p.n_tt : 0) + ttot * (p.n_n1 + p.n_n2) + p.n_cb;
+            // (router tasks are queue slots only when they are the queue's initial tasks)
+            sm.misc[6] = (x.q.n_init > 0 ? p.n_tk * p.n_kc : 0) + (p.n_tt > 1 ? p.n_tt : 0) +
+                         ttot * (p.n_n1 + p.n_n2) + p.n_cb;
             sm.misc[4] = ttot;
             sm.misc[5] = early;
         }
@@ -584,6 +589,26 @@ struct Moe {
         if (!group_wait(x, d, x.ctr + p.ev_tk, p.n_tk + p.bad_count, 230)) return false;
         RouteSmem sm = route_smem(x);
         const int e = x.tid;
+        if (p.n_tt == 1) {
+            // one grouping tile (T <= 128): the picks give the counts (popcounts
+            // of the per-expert token masks), the CSRs, then the placement
+            load_tile_picks(p, x, sm, 0, p.T);
+            int ex;
+            const int ttot = build_csr(p, x, sm, e < p.E ? tile_count(sm, e) : 0, &ex);
+            if (x.debug & ET_DEBUG_TRACE) d.t_acc = globaltimer();
+            if (e < p.E) sm.base[e] = ex;
+            exec_bar();
+            place_pairs(p, x, sm, 0, p.T);
+            if (!x.dynamic) {
+                group_finish_notify(x, d, x.ctr + p.ev_grp, 1, p.n_tt);
+                return true;
+            }
+            group_finish_notify(x, d, nullptr, 0, 0);
+            const bool early = sm.misc[5] != 0;
+            group_push(x, n_stage_tasks(p, ttot, early), [&](int i) { return stage_task(p, 0, ttot, i); });
+            publish_total(x, sm);
+            return true;
+        }
         int cnt = 0;
         // (plain L2 loads after the acquiring wait, sixteen tiles at a time)
 #pragma unroll 1
@@ -596,21 +621,8 @@ struct Moe {
             for (int i = 0; i < 16; ++i) cnt += v[i];
         }
         int ex;
-        const int ttot = build_csr(p, x, sm, cnt, &ex);
-        if (p.n_tt == 1) {
-            if (e < p.E) sm.base[e] = ex;
-            load_tile_picks(p, x, sm, 0, p.T);
-            place_pairs(p, x, sm, 0, p.T);
-            if (!x.dynamic) {
-                group_finish_notify(x, d, x.ctr + p.ev_grp, 1, p.n_tt);
-                return true;
-            }
-            group_finish_notify(x, d, nullptr, 0, 0);
-            const bool early = sm.misc[5] != 0;
-            group_push(x, n_stage_tasks(p, ttot, early), [&](int i) { return stage_task(p, 0, ttot, i); });
-            publish_total(x, sm);
-            return true;
-        }
+        build_csr(p, x, sm, cnt, &ex);
+        if (x.debug & ET_DEBUG_TRACE) d.t_acc = globaltimer();
         if (e < p.E) {
             int run = ex;
 #pragma unroll 1

@@ -11,7 +11,7 @@
 
 namespace et {
 
-struct SplitK {
+struct SplitK : WorkloadBase {
     using Params = SplitKParams;
     static constexpr bool kGemm = false;
 
@@ -79,6 +79,37 @@ cudaError_t splitk_setup(int* max_blocks_per_sm) {
     cudaError_t e = cudaFuncSetAttribute(splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(max_blocks_per_sm, splitk_kernel, kThreads, kSmemBytes);
+}
+
+// The two-launch control: the same two operators as plain kernels, one
+// launch each, ordered only by the stream (kernel-per-operator execution).
+// Partial kernel: one warp per (row, chunk); final kernel: one thread per row.
+__global__ void splitk_partial_kernel(const float* A, int rows, int cols, int chunk, int nch, float* Bp) {
+    const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (gw >= rows * nch) return;
+    const int r = gw / nch, j = gw % nch, c0 = j * chunk, nc = min(chunk, cols - c0);
+    const float* row = A + (size_t)r * cols + c0;
+    float s = 0.f;
+    for (int c = lane; c < nc; c += 32) s += row[c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) Bp[(size_t)r * nch + j] = s;
+}
+__global__ void splitk_final_kernel(const float* Bp, int rows, int nch, float* C) {
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    float s = 0.f;
+    for (int j = 0; j < nch; ++j) s += Bp[(size_t)r * nch + j];
+    C[r] = s;
+}
+cudaError_t launch_splitk_two(const float* A, int rows, int cols, int chunk, float* Bp, float* C, cudaStream_t s) {
+    const int nch = (cols + chunk - 1) / chunk;
+    const long warps = (long)rows * nch;
+    splitk_partial_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(A, rows, cols, chunk, nch, Bp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    splitk_final_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(Bp, rows, nch, C);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_splitk(const SplitKParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s) {

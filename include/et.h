@@ -65,11 +65,18 @@ typedef enum {
                              size bucket); consumers spin-wait on their events */
     ET_SCHED_DYNAMIC = 1, /* a device-side ready queue: a producer that brings an event to its
                              wait count pushes the consumers; SMs pop in batches */
-    ET_SCHED_UNFUSED = 2  /* control: the static lists with one barrier event between
+    ET_SCHED_UNFUSED = 2, /* control: the static lists with one barrier event between
                              consecutive operators (the "unfused megakernel" baseline) */
+    ET_SCHED_HYBRID = 3   /* per operator: regular operators from static per-SM lists, irregular
+                             (data-dependent) ones through the ready queue, in one launch.  Each
+                             CTA runs its list part A, pops the queue until it is exhausted, then
+                             runs its list part B.  split-K: partials static, finals queued;
+                             MoE: router static, grouping, expert stages and combine queued;
+                             decode layer: QKV static (part A), attention splits queued,
+                             o-proj and MLP static (part B); decode MLP: all static */
 } et_sched;
 
-typedef enum { ET_GRAPH_SPLITK = 0, ET_GRAPH_MLP = 1, ET_GRAPH_MOE = 2 } et_graph_kind;
+typedef enum { ET_GRAPH_SPLITK = 0, ET_GRAPH_MLP = 1, ET_GRAPH_MOE = 2, ET_GRAPH_DECODE = 3 } et_graph_kind;
 
 /* debug_flags bits */
 #define ET_DEBUG_TRACE 1      /* record one et_trace_record per task (tickets from one global counter) */
@@ -95,6 +102,12 @@ typedef struct {
     int device;          /* CUDA device ordinal */
     int n_ctas;          /* persistent CTAs [0 = one per SM] */
     float timeout_ms;    /* per-wait device time limit [1000] */
+    /* decode layer (ET_GRAPH_DECODE); hidden/inter above default to 4096 / 14336 */
+    int n_heads;         /* query heads [32] */
+    int n_kv_heads;      /* key/value heads [8]; n_heads / n_kv_heads <= 4 */
+    int head_dim;        /* [128]; only 128 is supported */
+    int max_ctx;         /* cache positions per request [4097]; a run's positions must be < max_ctx */
+    float rope_base;     /* rotary embedding base [500000] */
 } et_graph_desc;
 
 typedef struct et_graph et_graph; /* opaque, library-owned */
@@ -115,6 +128,9 @@ typedef struct {
     int moe_n2_tile;     /* output columns per stage-2 task */
     int moe_cb;          /* tokens per combine task at this graph's max_T; a run whose size
                             bucket (the power of two >= T, capped at max_T) is <= 256 uses 1 */
+    int dec_split;       /* decode: keys per attention split task */
+    int dec_qkv_kc;      /* decode: K chunks of a QKV head tile */
+    int dec_o_kc;        /* decode: K columns per o-proj task (the heads of one KV group) */
 } et_graph_info;
 
 /* Trace record (ET_DEBUG_TRACE): one per executed task. */
@@ -142,6 +158,18 @@ typedef struct {
 #define ET_OP_MOE_S1 24
 #define ET_OP_MOE_S2 25
 #define ET_OP_MOE_COMBINE 26
+#define ET_OP_DEC_NORM1 30    /* a = request */
+#define ET_OP_DEC_QKV 31      /* a = head tile (query heads, then key heads, then value heads), b = K chunk */
+#define ET_OP_DEC_QBR 32      /* inline: Q branch (norm + RoPE) of head a, run by the QKV task completing it */
+#define ET_OP_DEC_KBR 33      /* inline: K branch (norm + RoPE + cache append) of head tile a */
+#define ET_OP_DEC_VBR 34      /* inline: V cache append of head tile a */
+#define ET_OP_DEC_ATTN 35     /* a = request * n_kv_heads + KV head, b = split */
+#define ET_OP_DEC_MERGE 36    /* inline: merge of the splits of (request, KV head) a */
+#define ET_OP_DEC_OPROJ 37    /* a = output tile, b = K chunk (= KV head group) */
+#define ET_OP_DEC_NORM2 38    /* a = request */
+#define ET_OP_DEC_GATEUP 39   /* a = intermediate tile */
+#define ET_OP_DEC_DOWN 40     /* a = output tile, b = K chunk */
+#define ET_OP_DEC_RED 41      /* a = output tile */
 
 /* Event kinds of et_event_count records; index = the event's coordinate. */
 #define ET_EV_SK_TILE 1       /* split-K E[i]: partial tasks of row tile i done (count = #chunks) */
@@ -161,6 +189,20 @@ typedef struct {
 #define ET_EV_MOE_CB 26       /* E_cb[b]: stage-2 row contributions to combine block b */
 #define ET_EV_MOE_S1_ALL 27   /* unfused control: every stage-1 tile */
 #define ET_EV_MOE_S2_ALL 28   /* unfused control: every stage-2 tile */
+#define ET_EV_DEC_N1 40        /* E_n1: normalised rows (count B) */
+#define ET_EV_DEC_QKV 41       /* E_qkv[n]: K chunks of head tile n */
+#define ET_EV_DEC_G 42         /* E_g[g]: branches of KV group g done (its query heads, K and V) */
+#define ET_EV_DEC_ATT 43       /* E_att[b * n_kv + g]: attention splits of (request b, KV head g);
+                                  wait count = the request's split count (data-dependent) */
+#define ET_EV_DEC_AG 44        /* E_ag[g]: attention output of KV group g merged for every request */
+#define ET_EV_DEC_O 45         /* E_o: o-proj tiles */
+#define ET_EV_DEC_N2 46        /* E_n2: residual + norm rows */
+#define ET_EV_DEC_H 47         /* E_h[c]: gate/up tiles of down K-chunk c */
+#define ET_EV_DEC_Y 48         /* E_y[m]: down tiles of output tile m */
+#define ET_EV_DEC_BRANCH_ALL 49 /* unfused control: every head branch */
+#define ET_EV_DEC_MERGE_ALL 50 /* unfused control: every merge */
+#define ET_EV_DEC_GU_ALL 51    /* unfused control: every gate/up tile */
+#define ET_EV_DEC_DOWN_ALL 52  /* unfused control: every down tile */
 
 /* Notifications one event received in the last run (debug introspection). */
 typedef struct {
@@ -186,6 +228,16 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out);
  * 0 <= n_rows <= max_T (n_rows = 0 launches nothing). */
 et_status et_run_splitk(et_graph* g, const float* A, int n_rows, float* Bpart, float* C,
                         void* stream);
+
+/* Measurement control, not part of the event-tensor runtime: the same
+ * split-K reduction as two plain kernel launches on `stream` (all partials,
+ * then all finals), i.e. kernel-per-operator execution, the baseline the
+ * megakernel removes ([ETN] §背景: a launch costs several microseconds while
+ * a small kernel runs about two).  A fp32 [n_rows, cols]; Bpart fp32
+ * [n_rows, ceil(cols/chunk)]; C fp32 [n_rows].  Asynchronous; allocates
+ * nothing.  ET_ERR_INVALID on bad sizes or null/misaligned pointers. */
+et_status et_run_splitk_two_launch(const float* A, int n_rows, int cols, int chunk, float* Bpart, float* C,
+                                   void* stream);
 
 /* Fused decode MLP (RMSNorm -> gate/up GEMM -> SiLU*mul -> down GEMM) of
  * [ETN] §端到端低 batch serving ("Norm, MLP" of the decoding pipeline,
@@ -217,6 +269,42 @@ et_status et_run_mlp(et_graph* g, int B, const uint16_t* X, const uint16_t* gamm
 et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
                      const uint16_t* W1, const uint16_t* W2, uint16_t* Y, int32_t* topk,
                      float* topk_w, int32_t* indptr, int32_t* perm, float* logits, void* stream);
+
+/* Weights of the decode layer (bf16 bits, device memory, row-major). */
+typedef struct {
+    const uint16_t* g1;    /* [hidden] attention rmsnorm weight */
+    const uint16_t* Wqkv;  /* [(n_heads + 2 n_kv_heads) * head_dim, hidden]: query heads, key heads,
+                              value heads */
+    const uint16_t* gq;    /* [head_dim] per-head query rmsnorm weight */
+    const uint16_t* gk;    /* [head_dim] per-head key rmsnorm weight */
+    const uint16_t* Wo;    /* [hidden, n_heads * head_dim] */
+    const uint16_t* g2;    /* [hidden] MLP rmsnorm weight */
+    const uint16_t* Wgu;   /* [2 * inter, hidden]: gate rows, then up rows */
+    const uint16_t* Wd;    /* [hidden, inter] */
+} et_decode_weights;
+
+/* One decode step of a transformer layer for B requests, each adding one
+ * token ([ETN] §端到端低 batch serving: Attention, RoPE, KV-cache, Norm and
+ * MLP in one megakernel; the Q branch (norm + RoPE) and the K branch
+ * (norm + RoPE + cache append) run in parallel; weights of the next stage
+ * are prefetched before its activations arrive; §Data-dependent task
+ * triggering: request b's attention runs as ceil((pos[b] + 1) / dec_split)
+ * split tasks, a run-time count).  Per request b at position p = pos[b]:
+ *   xn  = bf16(rmsnorm(x) g1);  qkv = bf16(xn Wqkv^T)
+ *   q_h = bf16(rope(rmsnorm(q_h) gq, p)),  k_g = bf16(rope(rmsnorm(k_g) gk, p))
+ *   Kc[b,g,p] = k_g, Vc[b,g,p] = v_g          (written in place)
+ *   o_h = softmax over j <= p of (q_h . Kc[b,g,j] / sqrt(head_dim)) . Vc[b,g,j],
+ *         g = h / (n_heads / n_kv_heads)
+ *   h1  = bf16(x + bf16(o) Wo^T)
+ *   Y   = bf16(h1 + (bf16(silu(xn2 Wg^T) * (xn2 Wu^T))) Wd^T),  xn2 = bf16(rmsnorm(h1) g2)
+ * RoPE pairs element i with element i + head_dim/2 at angle p * base^(-2i/head_dim).
+ * X bf16 [B, hidden]; pos int32 [B] (device), 0 <= pos[b] < max_ctx, else the
+ * run ends with ET_ERR_INVALID from et_sync_status; Kc, Vc bf16 [max_T,
+ * n_kv_heads, max_ctx, head_dim] (device, updated in place at pos[b]);
+ * Y bf16 [B, hidden]; h1 (optional, NULL to skip) bf16 [B, hidden].
+ * 1 <= B <= max_T <= 128. */
+et_status et_run_decode(et_graph* g, int B, const uint16_t* X, const int32_t* pos, const et_decode_weights* w,
+                        uint16_t* Kc, uint16_t* Vc, uint16_t* Y, uint16_t* h1, void* stream);
 
 /* Split-K reduction without any device allocation.  (No counterpart in the
  * paper: this is an interface addition of this library.)

@@ -41,6 +41,8 @@ OP_SK_PARTIAL, OP_SK_FINAL = 1, 2
 OP_MLP_NORM, OP_MLP_GATEUP, OP_MLP_DOWN, OP_MLP_REDUCE = 10, 11, 12, 13
 OP_MOE_ROUTER, OP_MOE_SCAN, OP_MOE_GROUP, OP_MOE_S1, OP_MOE_S2, OP_MOE_COMBINE = (
     20, 22, 23, 24, 25, 26)
+(OP_DEC_NORM1, OP_DEC_QKV, OP_DEC_QBR, OP_DEC_KBR, OP_DEC_VBR, OP_DEC_ATTN, OP_DEC_MERGE, OP_DEC_OPROJ,
+ OP_DEC_NORM2, OP_DEC_GATEUP, OP_DEC_DOWN, OP_DEC_RED) = range(30, 42)
 
 
 def _cdiv(a, b):
@@ -51,8 +53,11 @@ def _cdiv(a, b):
 # numbers are declared in include/et.h) -> event names used below
 EVENT_KIND = {1: "E", 2: "Eall", 10: "E_norm", 11: "E_h", 12: "E_y", 13: "E_h_all", 14: "E_y_all",
               20: "E_rt", 21: "E_tk", 22: "E_sc", 23: "E_grp", 24: "E_exp", 25: "E_s1", 26: "E_cb",
-              27: "E_s1_all", 28: "E_s2_all"}
-_SCALAR_EVENTS = {"Eall", "E_norm", "E_h_all", "E_y_all", "E_tk", "E_sc", "E_grp", "E_s1_all", "E_s2_all"}
+              27: "E_s1_all", 28: "E_s2_all",
+              40: "D_n1", 41: "D_qkv", 42: "D_g", 43: "D_att", 44: "D_ag", 45: "D_o", 46: "D_n2", 47: "D_h",
+              48: "D_y", 49: "D_branch_all", 50: "D_merge_all", 51: "D_gu_all", 52: "D_down_all"}
+_SCALAR_EVENTS = {"Eall", "E_norm", "E_h_all", "E_y_all", "E_tk", "E_sc", "E_grp", "E_s1_all", "E_s2_all",
+                  "D_n1", "D_o", "D_n2", "D_branch_all", "D_merge_all", "D_gu_all", "D_down_all"}
 
 
 def event_key(kind, index):
@@ -484,3 +489,165 @@ def check_dataflow(rw, records):
                     errs.append("read before write: %r reads %r, written by %r (end %d, start %d)"
                                 % (task, it, w, end[w], start[task]))
     return errs
+
+
+# ------------------------------------------------------------ decode layer --
+
+def decode_graph(pos, nq, nkv, n_kc, split, n_m, n_gu, gu_tile, kchunk, n_c, sched):
+    """One decode step for len(pos) requests (pos[b] = the new token's
+    position), expanded with the run-time positions:
+      N1 b          --"b->"-->      D_n1              (count B)
+      D_n1          --"->nc"-->     QKV (n, c)
+      QKV (n, c)    --"nc->n"-->    D_qkv[n]          (count = #K chunks)
+      D_qkv[n]      -->             branch n          (Q: norm + RoPE; K: norm + RoPE +
+                                                       cache append; V: cache append)
+      branch n      --"n->g"-->     D_g[g]            (count = query heads per group + 2)
+      D_g[g]        --"g->bgs"-->   ATTN (b, g, s)    s < ceil((pos[b] + 1) / split):
+                                                      tasks[split_indptr[b] : split_indptr[b+1]]
+      ATTN (b,g,s)  --"bgs->bg"-->  D_att[b, g]       (count = the request's split count)
+      D_att[b, g]   -->             merge (b, g)
+      merge (b, g)  --"bg->g"-->    D_ag[g]           (count B)
+      D_ag[g]       --"g->mg"-->    o-proj (m, g)
+      o-proj (m, c) -->             D_o               (count = #tiles x #groups)
+      D_o           -->             N2 b  --> D_n2 (count B) --> gate/up n --> D_h[c] --> down (m, c)
+                                    --> D_y[m] (count = #K chunks) --> reduce m
+    Unfused: branch -> D_branch_all -> every split; merge -> D_merge_all ->
+    every o-proj; gate/up -> D_gu_all -> every down; down -> D_down_all ->
+    every reduce (the other edges are already operator-wide)."""
+    pos = [int(v) for v in pos]
+    B = len(pos)
+    grp = nq // nkv
+    n_heads = nq + 2 * nkv
+    unf = sched == "unfused"
+    g = Graph()
+    for b in range(B):
+        t = (OP_DEC_NORM1, b, 0)
+        g.add_task(t)
+        g.produce(t, ("D_n1",))
+    g.counted(("D_n1",), B)
+    for n in range(n_heads):
+        kind = OP_DEC_QBR if n < nq else (OP_DEC_KBR if n < nq + nkv else OP_DEC_VBR)
+        grp_of = n // grp if n < nq else (n - nq if n < nq + nkv else n - nq - nkv)
+        br = (kind, n, 0)
+        g.add_task(br)
+        for c in range(n_kc):
+            t = (OP_DEC_QKV, n, c)
+            g.add_task(t)
+            g.consume(t, ("D_n1",))
+            g.produce(t, ("D_qkv", n))
+        g.counted(("D_qkv", n), n_kc)
+        g.consume(br, ("D_qkv", n))
+        g.produce(br, ("D_branch_all",) if unf else ("D_g", grp_of))
+    if unf:
+        g.counted(("D_branch_all",), n_heads)
+    else:
+        for gg in range(nkv):
+            g.counted(("D_g", gg), grp + 2)
+    for b in range(B):
+        ns = (pos[b] + 1 + split - 1) // split
+        for gg in range(nkv):
+            bg = b * nkv + gg
+            mg = (OP_DEC_MERGE, bg, 0)
+            g.add_task(mg)
+            for s_ in range(ns):
+                t = (OP_DEC_ATTN, bg, s_)
+                g.add_task(t)
+                g.consume(t, ("D_branch_all",) if unf else ("D_g", gg))
+                g.produce(t, ("D_att", bg))
+            g.counted(("D_att", bg), ns)
+            g.consume(mg, ("D_att", bg))
+            g.produce(mg, ("D_merge_all",) if unf else ("D_ag", gg))
+    if unf:
+        g.counted(("D_merge_all",), B * nkv)
+    else:
+        for gg in range(nkv):
+            g.counted(("D_ag", gg), B)
+    for c in range(nkv):
+        for m in range(n_m):
+            t = (OP_DEC_OPROJ, m, c)
+            g.add_task(t)
+            g.consume(t, ("D_merge_all",) if unf else ("D_ag", c))
+            g.produce(t, ("D_o",))
+    g.counted(("D_o",), n_m * nkv)
+    for b in range(B):
+        t = (OP_DEC_NORM2, b, 0)
+        g.add_task(t)
+        g.consume(t, ("D_o",))
+        g.produce(t, ("D_n2",))
+    g.counted(("D_n2",), B)
+    for n in range(n_gu):
+        t = (OP_DEC_GATEUP, n, 0)
+        g.add_task(t)
+        g.consume(t, ("D_n2",))
+        g.produce(t, ("D_gu_all",) if unf else ("D_h", (n * gu_tile) // kchunk))
+    if unf:
+        g.counted(("D_gu_all",), n_gu)
+    else:
+        for c in range(n_c):
+            g.counted(("D_h", c), sum(1 for n in range(n_gu) if (n * gu_tile) // kchunk == c))
+    for m in range(n_m):
+        for c in range(n_c):
+            t = (OP_DEC_DOWN, m, c)
+            g.add_task(t)
+            g.consume(t, ("D_gu_all",) if unf else ("D_h", c))
+            g.produce(t, ("D_down_all",) if unf else ("D_y", m))
+        if not unf:
+            g.counted(("D_y", m), n_c)
+    if unf:
+        g.counted(("D_down_all",), n_m * n_c)
+    for m in range(n_m):
+        t = (OP_DEC_RED, m, 0)
+        g.add_task(t)
+        g.consume(t, ("D_down_all",) if unf else ("D_y", m))
+    return g.finish()
+
+
+def decode_dataflow(pos, nq, nkv, n_kc, split, n_m, n_gu, gu_tile, kchunk, n_c):
+    """{task: (reads, writes)} of one decode step, from what each operator
+    computes.  Items: ("xn", b), ("qkv", n) (head tile n's sums over every K
+    chunk), ("q", h), ("knew", g) / ("vnew", g) (the cache entries of this
+    step: position pos[b] of every request b), ("part", b, g, s),
+    ("attn", b, g), ("o", m) (o-proj sums), ("h1", b), ("xn2", b), ("hm", n),
+    ("down", m), ("y", m).  A split reads the new cache entries only if its
+    keys include pos[b]; the older entries are not written in this step."""
+    pos = [int(v) for v in pos]
+    B = len(pos)
+    grp = nq // nkv
+    n_heads = nq + 2 * nkv
+    rw = {}
+    for b in range(B):
+        rw[(OP_DEC_NORM1, b, 0)] = (set(), {("xn", b)})
+    xn_all = {("xn", b) for b in range(B)}
+    for n in range(n_heads):
+        for c in range(n_kc):
+            rw[(OP_DEC_QKV, n, c)] = (set(xn_all), {("qkv", n)})
+        if n < nq:
+            rw[(OP_DEC_QBR, n, 0)] = ({("qkv", n)}, {("q", n)})
+        elif n < nq + nkv:
+            rw[(OP_DEC_KBR, n, 0)] = ({("qkv", n)}, {("knew", n - nq)})
+        else:
+            rw[(OP_DEC_VBR, n, 0)] = ({("qkv", n)}, {("vnew", n - nq - nkv)})
+    for b in range(B):
+        ns = (pos[b] + 1 + split - 1) // split
+        for gg in range(nkv):
+            bg = b * nkv + gg
+            qs = {("q", gg * grp + h) for h in range(grp)}
+            for s_ in range(ns):
+                reads = set(qs)
+                if s_ * split <= pos[b] < (s_ + 1) * split:
+                    reads |= {("knew", gg), ("vnew", gg)}
+                rw[(OP_DEC_ATTN, bg, s_)] = (reads, {("part", b, gg, s_)})
+            rw[(OP_DEC_MERGE, bg, 0)] = ({("part", b, gg, s_) for s_ in range(ns)}, {("attn", b, gg)})
+    for c in range(nkv):
+        for m in range(n_m):
+            rw[(OP_DEC_OPROJ, m, c)] = ({("attn", b, c) for b in range(B)}, {("o", m)})
+    for b in range(B):
+        rw[(OP_DEC_NORM2, b, 0)] = ({("o", m) for m in range(n_m)}, {("h1", b), ("xn2", b)})
+    for n in range(n_gu):
+        rw[(OP_DEC_GATEUP, n, 0)] = ({("xn2", b) for b in range(B)}, {("hm", n)})
+    for m in range(n_m):
+        for c in range(n_c):
+            cols = {("hm", n) for n in range(n_gu) if c * kchunk <= n * gu_tile < (c + 1) * kchunk}
+            rw[(OP_DEC_DOWN, m, c)] = (cols, {("down", m)})
+        rw[(OP_DEC_RED, m, 0)] = ({("down", m)} | {("h1", b) for b in range(B)}, {("y", m)})
+    return rw

@@ -214,3 +214,47 @@ def test_dataflow_catches_a_dependency_missing_from_the_event_design():
         assert dag.check_trace(g, recs) == []
         errs = dag.check_dataflow(rw, recs)
         assert any("read before write" in e for e in errs), errs[:3]
+
+
+# ----------------------------------------------------------- decode layer --
+# §端到端低 batch serving (Q and K branches in parallel), §Data-dependent task
+# triggering (the split count of a request follows its context length).
+
+def _decode_case(sched, pos=(3, 9, 0)):
+    kw = dict(nq=4, nkv=2, n_kc=2, split=4, n_m=2, n_gu=4, gu_tile=64, kchunk=128, n_c=2)
+    g = dag.decode_graph(list(pos), sched=sched, **kw)
+    rw = dag.decode_dataflow(list(pos), **kw)
+    return g, rw
+
+
+def test_decode_splits_follow_positions():
+    g, _ = _decode_case("static", pos=(3, 9, 0))
+    A = dag.OP_DEC_ATTN
+    splits = sorted((t[1], t[2]) for t in g.tasks if t[0] == A)
+    # request 0 (4 keys): 1 split, request 1 (10 keys): 3 splits, request 2 (1 key): 1 split; 2 KV heads
+    assert splits == sorted([(0, 0), (1, 0)] + [(2, s) for s in range(3)] + [(3, s) for s in range(3)] +
+                            [(4, 0), (5, 0)])
+    assert g.wait_count[("D_att", 2)] == 3 and g.wait_count[("D_att", 0)] == 1
+    # the Q branch of head 1 (group 0) precedes every split of group 0 only
+    assert ((dag.OP_DEC_QBR, 1, 0), (A, 2, 1)) in g.edges
+    assert ((dag.OP_DEC_QBR, 1, 0), (A, 3, 1)) not in g.edges
+
+
+def test_decode_wait_counts_and_dataflow():
+    for sched in ("static", "dynamic", "hybrid", "unfused"):
+        g, rw = _decode_case(sched)
+        assert dag.check_wait_counts(g) == []
+        assert dag.check_dataflow(rw, _trace_priority(g, set())) == []
+
+
+def test_decode_dataflow_catches_a_split_before_its_cache_append():
+    """A split holding the new position read before the K branch appended
+    the new key is a real violation; the event-level check misses it once
+    the edge is dropped from the event graph."""
+    g, rw = _decode_case("static", pos=(3, 9, 0))
+    A, KBR = dag.OP_DEC_ATTN, dag.OP_DEC_KBR
+    # request 1, group 0 is bg = 2; position 9 lies in split 2 (keys 8..11); K head tile of group 0 is n = 4
+    g2 = _drop(g, lambda p, c: p == (KBR, 4, 0) and c == (A, 2, 2))
+    recs = _trace_priority(g2, {(A, 2, 2)}, {(KBR, 4, 0)})
+    assert dag.check_trace(g2, recs) == []
+    assert any("read before write" in e for e in dag.check_dataflow(rw, recs))

@@ -29,7 +29,7 @@ def run_mlp(g, d, B):
     return st, host(Y, np.uint16)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic", "unfused"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid", "unfused"])
 @pytest.mark.parametrize("B", [1, 5, 16, 33])
 def test_mlp_small_dims(sched, B):
     hidden, inter = 256, 512
@@ -58,7 +58,7 @@ def test_mlp_multi_chunk_and_repeat(sched):
         et.et_destroy_graph(g)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic", "unfused"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid", "unfused"])
 def test_mlp_dependency_order(sched):
     hidden, inter, B = 256, 2048, 3
     flags = et.ET_DEBUG_TRACE | et.ET_DEBUG_DELAY

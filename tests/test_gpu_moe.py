@@ -81,7 +81,7 @@ def small_inputs():
     return W.moe_inputs(300, hidden=256, inter=128, E=16, zipf_s=0.8)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic", "unfused"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid", "unfused"])
 @pytest.mark.parametrize("T", [1, 5, 37, 300])
 def test_moe_small_dims(small_inputs, sched, T):
     d = small_inputs
@@ -96,7 +96,7 @@ def test_moe_small_dims(small_inputs, sched, T):
         et.et_destroy_graph(g)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid"])
 @pytest.mark.parametrize("T", [1, 21, 150])
 def test_moe_e24_top8(sched, T):
     """E = 24 (the last 16-expert group of a router thread holds 8 experts),
@@ -114,7 +114,7 @@ def test_moe_e24_top8(sched, T):
         et.et_destroy_graph(g)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid"])
 def test_moe_symbolic_T_repeated_runs(small_inputs, sched):
     """One graph, one binary, T changing from run to run (no rebuild)."""
     d = small_inputs
@@ -130,7 +130,7 @@ def test_moe_symbolic_T_repeated_runs(small_inputs, sched):
         et.et_destroy_graph(g)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic", "unfused"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid", "unfused"])
 @pytest.mark.parametrize("T", [3, 200])
 def test_moe_dependency_order(small_inputs, sched, T):
     d = small_inputs
@@ -203,7 +203,7 @@ FULL_S = [0.0, 1.2, 1.5]
 def full_moe():
     d = W.moe_inputs(1, zipf_s=1.2)
     t = {n: dev(d[n]) for n in ("Wr", "W1", "W2")}
-    g = {s: et.et_build_graph(et.ET_GRAPH_MOE, s, 4096) for s in ("static", "dynamic")}
+    g = {s: et.et_build_graph(et.ET_GRAPH_MOE, s, 4096) for s in ("static", "dynamic", "hybrid")}
     cache = {}
     yield d, t, g, cache
     for h in g.values():
@@ -225,9 +225,11 @@ def _sample_tokens(T, topk, k, E, seed):
     return sorted(toks)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic"])
-@pytest.mark.parametrize("zipf", FULL_S)
-@pytest.mark.parametrize("T", FULL_T)
+FULL_CASES = [(T, z, s) for T in FULL_T for z in FULL_S for s in ("static", "dynamic")] + \
+    [(T, 1.2, "hybrid") for T in (1, 128, 4096)]
+
+
+@pytest.mark.parametrize("T,zipf,sched", FULL_CASES)
 def test_moe_full_size(full_moe, sched, zipf, T):
     """Routing bit-exact for every token (on the device's logits), event
     counts equal to the expansion's wait counts, and Y against the oracle's

@@ -39,7 +39,7 @@ def check(A, B, C):
     assert np.max(np.abs(C - Cref)) / np.max(np.abs(Cref)) <= 1e-5
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic", "unfused"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid", "unfused"])
 def test_splitk_config_parity(sched):
     g = et.et_build_graph(et.ET_GRAPH_SPLITK, sched, 2048)
     try:
@@ -52,7 +52,7 @@ def test_splitk_config_parity(sched):
         et.et_destroy_graph(g)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid"])
 @pytest.mark.parametrize("rows", [1, 31, 33, 1000, 4096])
 def test_splitk_ragged_and_symbolic_rows(sched, rows):
     g = et.et_build_graph(et.ET_GRAPH_SPLITK, sched, 4096)
@@ -80,7 +80,7 @@ def test_splitk_ragged_columns():
         et.et_destroy_graph(g)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic", "unfused"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid", "unfused"])
 @pytest.mark.parametrize("delay", [False, True])
 def test_splitk_dependency_order(sched, delay):
     flags = et.ET_DEBUG_TRACE | (et.ET_DEBUG_DELAY if delay else 0)
@@ -141,3 +141,19 @@ def test_splitk_pending_error_refuses_next_run(sched):
         assert et.et_sync_status(g) == et.ET_ERR_TIMEOUT
     finally:
         et.et_destroy_graph(g)
+
+
+def test_splitk_two_launch_control():
+    """The kernel-per-operator control computes the same reduction."""
+    for rows, cols in ((2048, 128), (77, 100)):
+        A = np.random.default_rng(rows).uniform(-1, 1, (rows, cols)).astype(np.float32)
+        nch = -(-cols // 32)
+        Bd = torch.zeros((rows, nch), device="cuda")
+        Cd = torch.zeros((rows,), device="cuda")
+        et.et_run_splitk_two_launch(dev(A), rows, cols, 32, Bd, Cd)
+        torch.cuda.synchronize()
+        Bref, Cref = oracle.splitk(A, 32)
+        scale = np.abs(A.astype(np.float64)).sum(1)
+        assert np.all(np.abs(host(Cd) - Cref) <= 1e-5 * scale)
+        scale_b = np.stack([np.abs(A[:, 32 * j:32 * j + 32]).astype(np.float64).sum(1) for j in range(nch)], 1)
+        assert np.all(np.abs(host(Bd) - Bref) <= 1e-5 * scale_b)
