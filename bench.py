@@ -307,6 +307,7 @@ def other_arm(args):
         a = np.ascontiguousarray(a)
         return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
 
+    control = None  # (description, callable) of a control timed beside the workload
     if args.workload == "decode":
         B = args.B
         d = W.decode_inputs(B)
@@ -322,6 +323,34 @@ def other_arm(args):
         workload = ("Llama-3-8B-shaped decode layer B=%d (hidden 4096, 32/8 heads x 128, SwiGLU 14336, "
                     "context %d..%d, mean %.0f), %s schedule" % (B, d["pos"].min(), d["pos"].max(),
                                                                  d["pos"].mean(), sched))
+    elif args.workload == "moe_mlp":
+        T = args.T if args.T <= 128 else 128
+        d = W.moe_inputs(T, zipf_s=args.zipf)
+        m = W.dense_mlp_weights()
+        t = {n: to_dev(v) for n, v in list(d.items()) + list(m.items())}
+        Y1 = torch.empty((T, 2048), dtype=torch.int16, device=dev)
+        Y2 = torch.empty((T, 2048), dtype=torch.int16, device=dev)
+        topk = torch.empty((T, 8), dtype=torch.int32, device=dev)
+        sched = args.sched
+        g = et.et_build_graph(et.ET_GRAPH_MOE_MLP, sched, 128)
+        g_moe = et.et_build_graph(et.ET_GRAPH_MOE, sched, 128)
+        g_mlp = et.et_build_graph(et.ET_GRAPH_MLP, "static" if sched == "dynamic" else sched, 128, hidden=2048,
+                                  inter=6144)
+        et.et_run_moe(g_moe, T, t["X"], t["Wr"], t["bias"], t["W1"], t["W2"], Y1, topk)
+        if et.et_sync_status(g_moe) != 0:
+            raise RuntimeError("MoE run reported a device error")
+        nbytes = algorithmic_bytes(topk.cpu().numpy(), T)[0] + sum(m[n].nbytes for n in ("gamma", "Wgu", "Wd")) + \
+            2 * T * 2048 * 2
+
+        def two():
+            et.et_run_moe(g_moe, T, t["X"], t["Wr"], t["bias"], t["W1"], t["W2"], Y1)
+            et.et_run_mlp(g_mlp, T, Y1, t["gamma"], t["Wgu"], t["Wd"], Y2)
+
+        run = lambda: et.et_run_moe_mlp(g, T, t["X"], t["Wr"], t["bias"], t["W1"], t["W2"], t["gamma"],  # noqa: E731
+                                        t["Wgu"], t["Wd"], Y1, Y2)
+        control = ("two launches (MoE megakernel, then the dense-MLP megakernel)", two)
+        workload = ("MoE layer T=%d (Zipf %g) -> dense MLP 2048->6144->2048, one megakernel, %s schedule"
+                    % (T, args.zipf, sched))
     elif args.workload == "mlp":
         B = args.B
         d = W.mlp_inputs(B)
@@ -335,35 +364,42 @@ def other_arm(args):
         A = to_dev(W.splitk_inputs(2048))
         Bp = torch.zeros((2048, 4), device=dev)
         C = torch.zeros((2048,), device=dev)
-        g = et.et_build_graph(et.ET_GRAPH_SPLITK, "static" if args.sched == "two_launch" else args.sched, 2048)
-        if args.sched == "two_launch":  # the kernel-per-operator control
-            run = lambda: et.et_run_splitk_two_launch(A, 2048, 128, 32, Bp, C)  # noqa: E731
-        else:
-            run = lambda: et.et_run_splitk(g, A, 2048, Bp, C)  # noqa: E731
+        g = et.et_build_graph(et.ET_GRAPH_SPLITK, args.sched, 2048)
+        run = lambda: et.et_run_splitk(g, A, 2048, Bp, C)  # noqa: E731
+        control = ("two launches (partials kernel, then finals kernel)",
+                   lambda: et.et_run_splitk_two_launch(A, 2048, 128, 32, Bp, C))
         nbytes = 2048 * 128 * 4 + 2048 * 5 * 4
         workload = "split-K 2048 x 128 fp32, chunks of 32, %s schedule" % args.sched
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    for _ in range(args.warmup):
-        flush.zero_()
-        run()
-    torch.cuda.synchronize(dev)
-    times = []
-    for _ in range(args.steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        run()
-        b.record()
-        b.synchronize()
-        times.append(a.elapsed_time(b))
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize(dev)
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    ms = timed(run)
     if et.et_sync_status(g) != 0:
         raise RuntimeError("run reported a device error")
+    extra = {}
+    if control is not None:
+        ms_c = timed(control[1])
+        extra["control"] = {"what": control[0], "latency_us": round(ms_c * 1e3, 2)}
     et.et_destroy_graph(g)
-    ms = statistics.median(times)
     hbm, _, src = load_peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"workload": workload, "latency_us": round(ms * 1e3, 2), "value": round(gbs, 1), "unit": "GB/s",
-            "steps": args.steps, "warmup": args.warmup, "bytes_per_launch": nbytes,
+            "steps": args.steps, "warmup": args.warmup, "bytes_per_launch": nbytes, **extra,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
                          "frac": round(gbs / hbm, 4), "peak_source": src}}
 
@@ -463,13 +499,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--T", type=int, default=128)
     ap.add_argument("--max_T", type=int, default=4096)
-    ap.add_argument("--sched", default="dynamic", choices=["static", "dynamic", "unfused", "hybrid", "two_launch"],
-                    help="two_launch (split-K only): the kernel-per-operator control")
+    ap.add_argument("--sched", default="dynamic", choices=["static", "dynamic", "unfused", "hybrid"])
     ap.add_argument("--zipf", type=float, default=1.2)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="moe", choices=["moe", "mlp", "splitk", "decode"],
-                    help="moe (the benchmark line); mlp, splitk or decode print a kernel timing line")
+    ap.add_argument("--workload", default="moe", choices=["moe", "mlp", "splitk", "decode", "moe_mlp"],
+                    help="moe (the benchmark line); mlp, splitk, decode or moe_mlp print a kernel timing line")
     ap.add_argument("--B", type=int, default=1, help="batch (--workload mlp or decode)")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false", help="skip the T x schedule sweep")
     ap.add_argument("--sweep-steps", type=int, default=50)

@@ -21,7 +21,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 # ------------------------------------------------------------ constants --
 ET_OK, ET_ERR_INVALID, ET_ERR_CUDA, ET_ERR_TIMEOUT, ET_ERR_OOM, ET_ERR_UNSUPPORTED, ET_ERR_PENDING, ET_ERR_INTERNAL = range(8)
 ET_SCHED_STATIC, ET_SCHED_DYNAMIC, ET_SCHED_UNFUSED, ET_SCHED_HYBRID = 0, 1, 2, 3
-ET_GRAPH_SPLITK, ET_GRAPH_MLP, ET_GRAPH_MOE, ET_GRAPH_DECODE = 0, 1, 2, 3
+ET_GRAPH_SPLITK, ET_GRAPH_MLP, ET_GRAPH_MOE, ET_GRAPH_DECODE, ET_GRAPH_MOE_MLP = 0, 1, 2, 3, 4
 ET_DEBUG_TRACE, ET_DEBUG_DELAY, ET_DEBUG_BAD_COUNT = 1, 2, 4
 SCHED = {"static": ET_SCHED_STATIC, "dynamic": ET_SCHED_DYNAMIC, "unfused": ET_SCHED_UNFUSED,
          "hybrid": ET_SCHED_HYBRID}
@@ -40,7 +40,7 @@ class et_graph_desc(ctypes.Structure):
         "splitk_tile_rows")] + [("rms_eps", ctypes.c_float)] + [(n, ctypes.c_int) for n in (
             "fetch_batch", "debug_flags", "device", "n_ctas")] + [("timeout_ms", ctypes.c_float)] + [
             (n, ctypes.c_int) for n in ("n_heads", "n_kv_heads", "head_dim", "max_ctx")] + [
-            ("rope_base", ctypes.c_float)]
+            ("rope_base", ctypes.c_float), ("mlp_inter", ctypes.c_int)]
 
 
 class et_graph_info(ctypes.Structure):
@@ -75,6 +75,7 @@ _sigs = {
     "et_run_splitk_noalloc": ([_P, _I, _P, _P, _P], _I),
     "et_run_splitk_two_launch": ([_P, _I, _I, _I, _P, _P, _P], _I),
     "et_run_decode": ([_P, _I, _P, _P, ctypes.POINTER(et_decode_weights), _P, _P, _P, _P, _P], _I),
+    "et_run_moe_mlp": ([_P, _I] + [_P] * 11, _I),
     "et_sync_status": ([_P, _P], _I),
     "et_get_trace": ([_P, _P, ctypes.c_size_t, ctypes.POINTER(_I)], _I),
     "et_get_info": ([_P, ctypes.POINTER(et_graph_info)], _I),
@@ -149,6 +150,11 @@ def et_run_moe(g, T, X, Wr, bias, W1, W2, Y, topk=None, topk_w=None, indptr=None
                stream=None):
     _check(_lib.et_run_moe(g, T, _ptr(X), _ptr(Wr), _ptr(bias), _ptr(W1), _ptr(W2), _ptr(Y), _ptr(topk),
                            _ptr(topk_w), _ptr(indptr), _ptr(perm), _ptr(logits), _stream(stream)), "et_run_moe")
+
+
+def et_run_moe_mlp(g, T, X, Wr, bias, W1, W2, gamma, Wgu, Wd, Y1, Y2, stream=None):
+    _check(_lib.et_run_moe_mlp(g, T, _ptr(X), _ptr(Wr), _ptr(bias), _ptr(W1), _ptr(W2), _ptr(gamma), _ptr(Wgu),
+                               _ptr(Wd), _ptr(Y1), _ptr(Y2), _stream(stream)), "et_run_moe_mlp")
 
 
 def et_run_decode(g, B, X, pos, w, Kc, Vc, Y, h1=None, stream=None):

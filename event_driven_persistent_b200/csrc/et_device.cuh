@@ -228,12 +228,17 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
                      smem_u32(bar))
                  : "memory");
 }
-// 32 lanes x 16 consecutive fp32 columns: thread i of the warp gets lane (quadrant*32 + i)
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+// 32 lanes x 16 consecutive fp32 columns: thread i of the warp gets lane
+// (quadrant*32 + i).  The load and its wait are one asm statement: the
+// destination registers of tcgen05.ld are written asynchronously and are
+// only valid after tcgen05.wait::ld, so the compiler must not see them as
+// defined (and schedule their uses) before the wait.
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15}, [%16];"
+        "%14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
@@ -241,7 +246,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Instruction descriptor, kind::f16: D fp32, A/B bf16, both K-major, M x N.
 __device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {

@@ -190,17 +190,6 @@ __device__ __forceinline__ bool group_wait(Ctx& x, TaskDesc& d, const int* ctr, 
 // (per K atom: 128 weight rows, then N activation rows; n is a multiple of 16)
 __device__ __forceinline__ uint32_t stage_bytes(int n) { return kAStageBytes + 2u * (uint32_t)n * 128u; }
 
-// Circular allocation of stages in the arena; the producer and the MMA
-// issuer replay the same sequence, so both know every stage's address.
-struct StageAlloc {
-    uint32_t head = 0;
-    __device__ __forceinline__ uint32_t next(uint32_t size) {
-        if (head + size > (uint32_t)kArenaBytes) head = 0;
-        const uint32_t o = head;
-        head += size;
-        return o;
-    }
-};
 
 // Stream tasks, exec group: wait for stage s of the task (all 128 threads
 // call; false on timeout/abort) and return its arena offset in *off.
@@ -331,17 +320,12 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
         StageAlloc alloc;
         uint32_t armed[kSlots];
         for (int s2 = 0; s2 < kSlots; ++s2) armed[s2] = 0;
-        // Reserve the next stage.  In-flight stages form one circular run of
-        // the arena from the tail stage to the allocation head, so the new
-        // stage can only collide with the oldest ones: consume (wait for)
-        // tail stages until its slot and its bytes are free.  O(1) amortised.
+        // Reserve the next stage: consume (wait for) stages in order, oldest
+        // first, while the new stage is blocked (stage_blocked).
         auto reserve = [&](uint32_t size, uint32_t* slot_out, uint32_t* off_out) -> bool {
             const uint32_t off = alloc.next(size);
-            while (tail < nst) {
+            while (tail < nst && stage_blocked(off, size, tail, nst, sc->r_off, sc->r_end)) {
                 const uint32_t ts = tail % kSlots;
-                const bool slot_busy = nst - tail >= (uint32_t)kSlots;
-                const bool overlap = off < sc->r_end[ts] && sc->r_off[ts] < off + size;
-                if (!slot_busy && !overlap) break;
                 if (!mbar_wait(&sc->empty[ts], (tail / kSlots) & 1, ctl, x.timeout_ns, 902)) return false;
                 ++tail;
             }
@@ -693,8 +677,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
 // the accumulator into v (thread = lane).
 __device__ __forceinline__ void acc_load16(uint32_t taddr, int c0, float (&v)[16]) {
     __syncwarp();  // tcgen05.ld is .sync.aligned: the warp must be converged
-    tmem_ld16(taddr + (uint32_t)c0, v);
-    tmem_ld_wait();
+    tmem_ld16_wait(taddr + (uint32_t)c0, v);
 }
 
 // Release the accumulator after this warp's last tcgen05.ld.

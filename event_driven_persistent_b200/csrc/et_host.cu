@@ -22,6 +22,8 @@ cudaError_t mlp_setup(int* max_blocks_per_sm);
 cudaError_t launch_mlp(const MlpParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
 cudaError_t moe_setup(int* max_blocks_per_sm);
 cudaError_t launch_moe(const MoeParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
+cudaError_t moe_mlp_setup(int* max_blocks_per_sm);
+cudaError_t launch_moe_mlp(const MoeMlpParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
 cudaError_t decode_setup(int* max_blocks_per_sm);
 cudaError_t launch_decode(const DecodeParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s);
 }  // namespace et
@@ -147,6 +149,7 @@ struct et_graph {
     MlpParams last_mlp;
     MoeParams last_moe;
     DecodeParams last_dec;
+    MlpParams last_moe_mlp;  // the MLP half of the last MoE -> MLP run
     // workload state
     SplitKParams sk;
     MlpParams mlp;
@@ -323,54 +326,69 @@ et_status build_splitk(et_graph* g) {
 }
 
 // ----------------------------------------------------------------- MLP ----
+// MLP part of a graph: dims, events from ev0 (*ev_end = the next free
+// one), workspace; the slots of its static lists (with or without the norm
+// tasks; `part` = hybrid list part).
+et_status setup_mlp(et_graph* g, MlpParams& p, int hidden, int inter, int maxB, float eps, int ev0, int* ev_end) {
+    if (maxB > kMaxN) return ET_ERR_UNSUPPORTED;  // one token tile
+    if (hidden % 128 || inter % 128) return ET_ERR_UNSUPPORTED;
+    memset(&p, 0, sizeof(p));
+    p.hidden = hidden;
+    p.inter = inter;
+    p.maxB = maxB;
+    p.eps = eps;
+    p.gu_tile = 64;
+    p.down_tile = 128;
+    p.kchunk = inter % 1024 == 0 ? 1024 : (inter % 256 == 0 ? 256 : 128);
+    p.n_gu = inter / p.gu_tile;
+    p.n_m = hidden / p.down_tile;
+    p.n_c = inter / p.kchunk;
+    p.gu_per_chunk = p.kchunk / p.gu_tile;
+    if (p.n_gu > 0xFFFF || p.n_c > 0x3FF) return ET_ERR_UNSUPPORTED;
+    p.ev_norm = ev0;
+    p.ev_h = p.ev_norm + 1;
+    p.ev_y = p.ev_h + p.n_c;
+    p.ev_gu_all = p.ev_y + p.n_m;
+    p.ev_down_all = p.ev_gu_all + 1;
+    *ev_end = p.ev_down_all + 1;
+    p.unfused = g->d.sched == ET_SCHED_UNFUSED;
+    p.push = g->d.sched == ET_SCHED_DYNAMIC;
+    p.bad_count = (g->d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
+    const size_t rows = (size_t)std::max(maxB, 16);  // at least one 16-row TMA box
+    ET_TRY(galloc(g, &p.xn, rows * p.hidden));
+    ET_TRY(galloc(g, &p.h, rows * p.inter));
+    ET_TRY(galloc(g, &p.yacc, (size_t)p.maxB * p.hidden));
+    if (!make_map(&p.tm_xn, p.xn, rows, p.hidden, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_h, p.h, rows, p.inter, 16)) return ET_ERR_CUDA;
+    return ET_OK;
+}
+int mlp_queue_tasks(const MlpParams& p) { return p.maxB + p.n_gu + p.n_m * p.n_c + p.n_m; }
+void mlp_slots(const MlpParams& p, int Tb, std::vector<Slot>& s, bool with_norm, int part) {
+    // cost ~ bytes streamed per task (KB)
+    const float c_gu = 2.f * p.gu_tile * p.hidden * 2 / 1024.f, c_dn = (float)p.down_tile * p.kchunk * 2 / 1024.f;
+    if (with_norm)
+        for (int b = 0; b < Tb; ++b) s.push_back({tw(ET_OP_MLP_NORM, b, 0), 1.f, part});
+    for (int n = 0; n < p.n_gu; ++n) s.push_back({tw(ET_OP_MLP_GATEUP, n, 0), c_gu, part});
+    for (int c = 0; c < p.n_c; ++c)
+        for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_MLP_DOWN, m, c), c_dn, part});
+    for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_MLP_REDUCE, m, 0), 2.f, part});
+}
+
 et_status build_mlp(et_graph* g) {
     et_graph_desc& d = g->d;
     if (d.hidden <= 0) d.hidden = 4096;
     if (d.inter <= 0) d.inter = 14336;
     if (d.rms_eps <= 0.f) d.rms_eps = 1e-5f;
     if (d.fetch_batch <= 0) d.fetch_batch = 1;
-    if (d.max_T > kMaxN) return ET_ERR_UNSUPPORTED;  // one token tile
-    if (d.hidden % 128 || d.inter % 128) return ET_ERR_UNSUPPORTED;
     MlpParams& p = g->mlp;
-    memset(&p, 0, sizeof(p));
-    p.hidden = d.hidden;
-    p.inter = d.inter;
-    p.maxB = d.max_T;
-    p.eps = d.rms_eps;
-    p.gu_tile = 64;
-    p.down_tile = 128;
-    p.kchunk = d.inter % 1024 == 0 ? 1024 : (d.inter % 256 == 0 ? 256 : 128);
-    p.n_gu = d.inter / p.gu_tile;
-    p.n_m = d.hidden / p.down_tile;
-    p.n_c = d.inter / p.kchunk;
-    p.gu_per_chunk = p.kchunk / p.gu_tile;
-    if (p.n_gu > 0xFFFF || p.n_c > 0x3FF) return ET_ERR_UNSUPPORTED;
-    p.ev_norm = kCtrFirstEvent;
-    p.ev_h = p.ev_norm + 1;
-    p.ev_y = p.ev_h + p.n_c;
-    p.ev_gu_all = p.ev_y + p.n_m;
-    p.ev_down_all = p.ev_gu_all + 1;
-    p.unfused = d.sched == ET_SCHED_UNFUSED;
-    p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
-    g->n_ctr = p.ev_down_all + 1;
-    g->qcap = d.max_T + p.n_gu + p.n_m * p.n_c + p.n_m + g->n_ctas * d.fetch_batch + 64;
-    ET_TRY(galloc(g, &p.xn, (size_t)p.maxB * p.hidden));
-    ET_TRY(galloc(g, &p.h, (size_t)p.maxB * p.inter));
-    ET_TRY(galloc(g, &p.yacc, (size_t)p.maxB * p.hidden));
-    if (!make_map(&p.tm_xn, p.xn, p.maxB, p.hidden, 16)) return ET_ERR_CUDA;
-    if (!make_map(&p.tm_h, p.h, p.maxB, p.inter, 16)) return ET_ERR_CUDA;
+    int ev_end = 0;
+    ET_TRY(setup_mlp(g, p, d.hidden, d.inter, d.max_T, d.rms_eps, kCtrFirstEvent, &ev_end));
+    g->n_ctr = ev_end;
+    g->qcap = mlp_queue_tasks(p) + g->n_ctas * d.fetch_batch + 64;
     int mb = 0;
     ET_CU(mlp_setup(&mb));
     if (mb < 1) return ET_ERR_UNSUPPORTED;
-    // cost ~ bytes streamed per task (KB)
-    const float c_gu = 2.f * p.gu_tile * p.hidden * 2 / 1024.f, c_dn = (float)p.down_tile * p.kchunk * 2 / 1024.f;
-    return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
-        for (int b = 0; b < Tb; ++b) s.push_back({tw(ET_OP_MLP_NORM, b, 0), 1.f});
-        for (int n = 0; n < p.n_gu; ++n) s.push_back({tw(ET_OP_MLP_GATEUP, n, 0), c_gu});
-        for (int c = 0; c < p.n_c; ++c)
-            for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_MLP_DOWN, m, c), c_dn});
-        for (int m = 0; m < p.n_m; ++m) s.push_back({tw(ET_OP_MLP_REDUCE, m, 0), 2.f});
-    });
+    return build_lists(g, [&](int Tb, std::vector<Slot>& s) { mlp_slots(p, Tb, s, true, 0); });
 }
 
 // ----------------------------------------------------------------- MoE ----
@@ -400,7 +418,9 @@ MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
     return m;
 }
 
-et_status build_moe(et_graph* g) {
+// MoE part of a graph: dims, events from ev0 (*ev_end = the next free
+// one), queue slots it may need (*qtasks), workspace; and its list slots.
+et_status setup_moe(et_graph* g, int ev0, int* ev_end, int* qtasks) {
     et_graph_desc& d = g->d;
     if (d.hidden <= 0) d.hidden = 2048;
     if (d.inter <= 0) d.inter = 768;
@@ -429,7 +449,7 @@ et_status build_moe(et_graph* g) {
     p.bad_count = (d.debug_flags & ET_DEBUG_BAD_COUNT) ? 1 : 0;
     const MoeShape mx = moe_shape(g, p, d.max_T);
     if (mx.f_max > 0xFFFF || mx.n_tt > 0xFFFF || p.n_n1 > 0x3FF || p.n_n2 > 0x3FF) return ET_ERR_UNSUPPORTED;
-    int ev = kCtrFirstEvent;
+    int ev = ev0;
     p.ev_tk = ev++;
     p.ev_rt = ev;
     ev += mx.n_tk;
@@ -446,8 +466,8 @@ et_status build_moe(et_graph* g) {
     ev += n_cb_max;
     p.ev_gcnt = ev;
     ev += mx.n_tt * p.E;
-    g->n_ctr = ev;
-    g->qcap = mx.n_tk * 8 + mx.n_tt + 1 + mx.f_max * (p.n_n1 + p.n_n2) + n_cb_max + g->n_ctas * d.fetch_batch + 64;
+    *ev_end = ev;
+    *qtasks = mx.n_tk * 8 + mx.n_tt + 1 + mx.f_max * (p.n_n1 + p.n_n2) + n_cb_max;
     const size_t pairs = (size_t)p.maxT * p.k;
     ET_TRY(galloc(g, &p.lacc, (size_t)p.maxT * p.E));
     ET_TRY(galloc(g, &p.topk, pairs));
@@ -463,29 +483,76 @@ et_status build_moe(et_graph* g) {
     ET_TRY(galloc(g, &p.Hm, pairs * p.inter));
     ET_TRY(galloc(g, &p.Yacc, (size_t)p.maxT * p.hidden));
     if (!make_map(&p.tm_hm, p.Hm, pairs, p.inter, 16)) return ET_ERR_CUDA;
+    return ET_OK;
+}
+void moe_slots(et_graph* g, const MoeParams& p, int Tb, std::vector<Slot>& s) {
+    const float c_s1 = 2.f * p.n1_tile * p.hidden * 2 / 1024.f, c_s2 = (float)p.n2_tile * p.inter * 2 / 1024.f;
+    MoeShape m = moe_shape(g, p, Tb);
+    const float c_rt = (float)p.E * p.hidden * 2 / m.n_kc / 1024.f;
+    for (int j = 0; j < m.n_tk; ++j)
+        for (int c = 0; c < m.n_kc; ++c) s.push_back({tw(ET_OP_MOE_ROUTER, j, c), c_rt});
+    if (g->hybrid) return;  // grouping, expert stages and combine go through the queue
+    s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 8.f});
+    if (m.n_tt > 1)
+        for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_GROUP, t, 0), 8.f});
+    for (int f = 0; f < m.f_max; ++f)
+        for (int n = 0; n < p.n_n1; ++n) s.push_back({tw(ET_OP_MOE_S1, f, n), c_s1});
+    for (int f = 0; f < m.f_max; ++f)
+        for (int n = 0; n < p.n_n2; ++n) s.push_back({tw(ET_OP_MOE_S2, f, n), c_s2});
+    for (int b = 0; b < m.n_cb; ++b) s.push_back({tw(ET_OP_MOE_COMBINE, b, 0), 2.f});
+}
+
+void moe_defaults(et_graph_desc& d) {
+    if (d.hidden <= 0) d.hidden = 2048;
+    if (d.inter <= 0) d.inter = 768;
+    if (d.n_experts <= 0) d.n_experts = 128;
+    if (d.top_k <= 0) d.top_k = 8;
+    if (d.fetch_batch <= 0) d.fetch_batch = 1;
+}
+
+et_status build_moe(et_graph* g) {
+    moe_defaults(g->d);
+    int ev_end = 0, qt = 0;
+    ET_TRY(setup_moe(g, kCtrFirstEvent, &ev_end, &qt));
+    g->n_ctr = ev_end;
+    g->qcap = qt + g->n_ctas * g->d.fetch_batch + 64;
     int mb = 0;
     ET_CU(moe_setup(&mb));
     if (mb < 1) return ET_ERR_UNSUPPORTED;
-    const float c_s1 = 2.f * p.n1_tile * p.hidden * 2 / 1024.f, c_s2 = (float)p.n2_tile * p.inter * 2 / 1024.f;
+    return build_lists(g, [&](int Tb, std::vector<Slot>& s) { moe_slots(g, g->moe, Tb, s); });
+}
+
+// The MoE layer followed by a dense SwiGLU MLP (hidden -> mlp_inter ->
+// hidden) on its output, one launch; T <= 128 (the MLP's one token tile).
+et_status build_moe_mlp(et_graph* g) {
+    et_graph_desc& d = g->d;
+    moe_defaults(d);
+    if (d.mlp_inter <= 0) d.mlp_inter = 6144;
+    if (d.rms_eps <= 0.f) d.rms_eps = 1e-5f;
+    if (d.max_T > kMaxN) return ET_ERR_UNSUPPORTED;
+    int ev1 = 0, qt = 0, ev2 = 0;
+    ET_TRY(setup_moe(g, kCtrFirstEvent, &ev1, &qt));
+    ET_TRY(setup_mlp(g, g->mlp, d.hidden, d.mlp_inter, d.max_T, d.rms_eps, ev1, &ev2));
+    MoeParams& p = g->moe;
+    const MlpParams& m = g->mlp;
+    p.mlp_xn = m.xn;
+    p.mlp_eps = d.rms_eps;
+    p.mlp_ev_norm = m.ev_norm;
+    p.mlp_n_gu = m.push ? m.n_gu : 0;
+    p.extra_tasks = m.push ? m.n_gu + m.n_m * m.n_c + m.n_m : 0;
+    g->n_ctr = ev2;
+    g->qcap = qt + mlp_queue_tasks(m) + g->n_ctas * d.fetch_batch + 64;
+    int mb = 0;
+    ET_CU(moe_mlp_setup(&mb));
+    if (mb < 1) return ET_ERR_UNSUPPORTED;
     return build_lists(g, [&](int Tb, std::vector<Slot>& s) {
-        MoeShape m = moe_shape(g, p, Tb);
-        const float c_rt = (float)p.E * p.hidden * 2 / m.n_kc / 1024.f;
-        for (int j = 0; j < m.n_tk; ++j)
-            for (int c = 0; c < m.n_kc; ++c) s.push_back({tw(ET_OP_MOE_ROUTER, j, c), c_rt});
-        if (g->hybrid) return;  // grouping, expert stages and combine go through the queue
-        s.push_back({tw(ET_OP_MOE_SCAN, 0, 0), 8.f});
-        if (m.n_tt > 1)
-            for (int t = 0; t < m.n_tt; ++t) s.push_back({tw(ET_OP_MOE_GROUP, t, 0), 8.f});
-        for (int f = 0; f < m.f_max; ++f)
-            for (int n = 0; n < p.n_n1; ++n) s.push_back({tw(ET_OP_MOE_S1, f, n), c_s1});
-        for (int f = 0; f < m.f_max; ++f)
-            for (int n = 0; n < p.n_n2; ++n) s.push_back({tw(ET_OP_MOE_S2, f, n), c_s2});
-        for (int b = 0; b < m.n_cb; ++b) s.push_back({tw(ET_OP_MOE_COMBINE, b, 0), 2.f});
+        moe_slots(g, g->moe, Tb, s);
+        if (!(g->d.sched == ET_SCHED_DYNAMIC)) mlp_slots(g->mlp, Tb, s, false, 1);  // after the queue when hybrid
     });
 }
 
 // --------------------------------------------------------- decode layer ----
-constexpr int kDecSplit = 256;  // keys per attention split task
+constexpr int kDecSplit = 512;  // keys per attention split task (four 128-key stages)
 
 et_status build_decode(et_graph* g) {
     et_graph_desc& d = g->d;
@@ -530,6 +597,7 @@ et_status build_decode(et_graph* g) {
     const int nq_rows = p.maxB * p.nkv;
     if (nq_rows > 0xFFFF || p.s_max > 0x3FF || p.n_heads > 0xFFFF || p.n_c > 0x3FF || p.nkv > 0x3FF)
         return ET_ERR_UNSUPPORTED;
+    if (p.s_max * p.grp > 1024) return ET_ERR_UNSUPPORTED;  // the merge keeps every split's (max, sum) in smem
     int ev = kCtrFirstEvent;
     p.ev_n1 = ev++;
     p.ev_qkv = ev;
@@ -617,7 +685,7 @@ const char* et_status_str(et_status s) {
 et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     if (!desc || !out) return ET_ERR_INVALID;
     *out = nullptr;
-    if (desc->max_T < 1 || desc->kind < 0 || desc->kind > 3 || desc->sched < 0 || desc->sched > 3)
+    if (desc->max_T < 1 || desc->kind < 0 || desc->kind > 4 || desc->sched < 0 || desc->sched > 3)
         return ET_ERR_INVALID;
     et_graph* g = new et_graph();
     g->d = *desc;
@@ -639,6 +707,7 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     if (desc->kind == ET_GRAPH_SPLITK) st = build_splitk(g);
     else if (desc->kind == ET_GRAPH_MLP) st = build_mlp(g);
     else if (desc->kind == ET_GRAPH_MOE) st = build_moe(g);
+    else if (desc->kind == ET_GRAPH_MOE_MLP) st = build_moe_mlp(g);
     else st = build_decode(g);
     if (st != ET_OK) return fail(st);
     // common workspace
@@ -680,7 +749,12 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
         in.mlp_down_tile = g->mlp.down_tile;
         in.mlp_kchunk = g->mlp.kchunk;
     }
-    if (desc->kind == ET_GRAPH_MOE) {
+    if (desc->kind == ET_GRAPH_MOE_MLP) {
+        in.mlp_gu_tile = g->mlp.gu_tile;
+        in.mlp_down_tile = g->mlp.down_tile;
+        in.mlp_kchunk = g->mlp.kchunk;
+    }
+    if (desc->kind == ET_GRAPH_MOE || desc->kind == ET_GRAPH_MOE_MLP) {
         in.moe_tt = g->moe.tt;
         in.moe_gt = g->moe.tt;
         in.moe_tkt = g->moe.tkt;
@@ -771,15 +845,9 @@ et_status et_run_mlp(et_graph* g, int B, const uint16_t* X, const uint16_t* gamm
     return ET_OK;
 }
 
-et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
-                     const uint16_t* W1, const uint16_t* W2, uint16_t* Y, int32_t* topk, float* topk_w,
-                     int32_t* indptr, int32_t* perm, float* logits, void* stream) {
-    if (!g || g->d.kind != ET_GRAPH_MOE) return ET_ERR_INVALID;
-    if (T < 1 || T > g->d.max_T) return ET_ERR_INVALID;
-    if (!aligned16(X) || !aligned16(Wr) || !bias || !aligned16(W1) || !aligned16(W2) || !aligned16(Y))
-        return ET_ERR_INVALID;
-    cudaStream_t s = (cudaStream_t)stream;
-    ET_CU(cudaSetDevice(g->dev));
+// Fill the MoE half's per-run fields (shared by et_run_moe and et_run_moe_mlp).
+et_status moe_run_params(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
+                         const uint16_t* W1, const uint16_t* W2, uint16_t* Y) {
     MoeParams& p = g->moe;
     if (!g->mc[0].get(&p.tm_wr, Wr, p.E, p.hidden, 64)) return ET_ERR_CUDA;
     if (!g->mc[1].get(&p.tm_w1, W1, (uint64_t)p.E * 2 * p.inter, p.hidden, 64)) return ET_ERR_CUDA;
@@ -788,11 +856,11 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
     p.X = X;
     p.bias = bias;
     p.Y = Y;
-    p.out_topk = topk;
-    p.out_w = topk_w;
-    p.out_indptr = indptr;
-    p.out_perm = perm;
-    p.out_logits = logits;
+    p.out_topk = nullptr;
+    p.out_w = nullptr;
+    p.out_indptr = nullptr;
+    p.out_perm = nullptr;
+    p.out_logits = nullptr;
     p.T = T;
     const int b = g->bucket_of(T);
     const MoeShape mb = moe_shape(g, p, g->bucket_T[b]);
@@ -803,6 +871,25 @@ et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, 
     p.cb = mb.cb;      // (static lists and dynamic alike)
     p.n_cb = cdiv(T, p.cb);
     p.f_max = mb.f_max;
+    return ET_OK;
+}
+
+et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
+                     const uint16_t* W1, const uint16_t* W2, uint16_t* Y, int32_t* topk, float* topk_w,
+                     int32_t* indptr, int32_t* perm, float* logits, void* stream) {
+    if (!g || g->d.kind != ET_GRAPH_MOE) return ET_ERR_INVALID;
+    if (T < 1 || T > g->d.max_T) return ET_ERR_INVALID;
+    if (!aligned16(X) || !aligned16(Wr) || !bias || !aligned16(W1) || !aligned16(W2) || !aligned16(Y))
+        return ET_ERR_INVALID;
+    cudaStream_t s = (cudaStream_t)stream;
+    ET_CU(cudaSetDevice(g->dev));
+    ET_TRY(moe_run_params(g, T, X, Wr, bias, W1, W2, Y));
+    MoeParams& p = g->moe;
+    p.out_topk = topk;
+    p.out_w = topk_w;
+    p.out_indptr = indptr;
+    p.out_perm = perm;
+    p.out_logits = logits;
     ET_TRY(pre_run(g, s));
     RunArgs ra = run_args(g, T, g->hybrid ? 0 : p.n_tk * p.n_kc, 0);  // hybrid: router tasks are listed
     ET_TRY(launched(g, launch_moe(p, ra, g->n_ctas, s)));
@@ -846,6 +933,36 @@ et_status et_run_decode(et_graph* g, int B, const uint16_t* X, const int32_t* po
     return ET_OK;
 }
 
+et_status et_run_moe_mlp(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
+                         const uint16_t* W1, const uint16_t* W2, const uint16_t* gamma, const uint16_t* Wgu,
+                         const uint16_t* Wd, uint16_t* Y1, uint16_t* Y2, void* stream) {
+    if (!g || g->d.kind != ET_GRAPH_MOE_MLP) return ET_ERR_INVALID;
+    if (T < 1 || T > g->d.max_T) return ET_ERR_INVALID;
+    if (!aligned16(X) || !aligned16(Wr) || !bias || !aligned16(W1) || !aligned16(W2) || !aligned16(gamma) ||
+        !aligned16(Wgu) || !aligned16(Wd) || !aligned16(Y1) || !aligned16(Y2))
+        return ET_ERR_INVALID;
+    cudaStream_t s = (cudaStream_t)stream;
+    ET_CU(cudaSetDevice(g->dev));
+    ET_TRY(moe_run_params(g, T, X, Wr, bias, W1, W2, Y1));
+    MlpParams& m = g->mlp;
+    if (!g->mc[4].get(&m.tm_wgu, Wgu, 2ull * m.inter, m.hidden, 64)) return ET_ERR_CUDA;
+    if (!g->mc[5].get(&m.tm_wd, Wd, m.hidden, m.inter, 64)) return ET_ERR_CUDA;
+    m.gamma = gamma;
+    m.Y = Y2;
+    m.B = T;
+    g->moe.mlp_gamma = gamma;
+    ET_TRY(pre_run(g, s));
+    MoeMlpParams pp;
+    pp.moe = g->moe;
+    pp.mlp = m;
+    RunArgs ra = run_args(g, T, g->hybrid ? 0 : g->moe.n_tk * g->moe.n_kc, 0);
+    ET_TRY(launched(g, launch_moe_mlp(pp, ra, g->n_ctas, s)));
+    g->last_T = T;
+    g->last_moe = g->moe;
+    g->last_moe_mlp = m;
+    return ET_OK;
+}
+
 et_status et_sync_status(et_graph* g, void* stream) {
     if (!g) return ET_ERR_INVALID;
     ET_CU(cudaSetDevice(g->dev));
@@ -858,7 +975,7 @@ et_status et_sync_status(et_graph* g, void* stream) {
     ET_TRY(reset_ctl(g));
     ET_CU(cudaMemset(g->ctr[0], 0, g->n_ctr * sizeof(int)));
     ET_CU(cudaMemset(g->ctr[1], 0, g->n_ctr * sizeof(int)));
-    if (g->d.kind == ET_GRAPH_MLP)  // sums kept zero between runs
+    if (g->d.kind == ET_GRAPH_MLP || g->d.kind == ET_GRAPH_MOE_MLP)  // sums kept zero between runs
         ET_CU(cudaMemset(g->mlp.yacc, 0, (size_t)g->mlp.maxB * g->mlp.hidden * sizeof(float)));
     if (g->d.kind == ET_GRAPH_DECODE) {
         const DecodeParams& p = g->dec;
@@ -866,7 +983,7 @@ et_status et_sync_status(et_graph* g, void* stream) {
         ET_CU(cudaMemset(p.h1acc, 0, (size_t)p.maxB * p.hidden * sizeof(float)));
         ET_CU(cudaMemset(p.yacc, 0, (size_t)p.maxB * p.hidden * sizeof(float)));
     }
-    if (g->d.kind == ET_GRAPH_MOE && g->moe.Yacc) {
+    if ((g->d.kind == ET_GRAPH_MOE || g->d.kind == ET_GRAPH_MOE_MLP) && g->moe.Yacc) {
         ET_CU(cudaMemset(g->moe.Yacc, 0, (size_t)g->moe.maxT * g->moe.hidden * sizeof(float)));
         ET_CU(cudaMemset(g->moe.lacc, 0, (size_t)g->moe.maxT * g->moe.E * sizeof(float)));
     }
@@ -935,6 +1052,14 @@ et_status et_get_event_counts(et_graph* g, et_event_count* buf, int cap, int* n_
         for (int b = 0; b < p.n_cb; ++b) add(ET_EV_MOE_CB, b, p.ev_cb + b);
         add(ET_EV_MOE_S1_ALL, 0, p.ev_s1_all);
         add(ET_EV_MOE_S2_ALL, 0, p.ev_s2_all);
+        if (g->d.kind == ET_GRAPH_MOE_MLP) {
+            const MlpParams& m = g->last_moe_mlp;
+            add(ET_EV_MLP_NORM, 0, m.ev_norm);
+            for (int i = 0; i < m.n_c; ++i) add(ET_EV_MLP_H, i, m.ev_h + i);
+            for (int i = 0; i < m.n_m; ++i) add(ET_EV_MLP_Y, i, m.ev_y + i);
+            add(ET_EV_MLP_GU_ALL, 0, m.ev_gu_all);
+            add(ET_EV_MLP_DOWN_ALL, 0, m.ev_down_all);
+        }
     }
     *n_events = (int)v.size();
     for (int i = 0; i < cap && i < (int)v.size(); ++i) buf[i] = v[i];

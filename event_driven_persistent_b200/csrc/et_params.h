@@ -43,6 +43,7 @@ struct MlpParams {
     int n_gu, n_m, n_c, gu_per_chunk;
     int ev_norm, ev_h, ev_y, ev_gu_all, ev_down_all;
     int unfused;
+    int push;            // 1 = a task that completes an event queues its consumers (dynamic schedule)
     int bad_count;
 };
 
@@ -92,6 +93,14 @@ struct MoeParams {
     int ev_gcnt;        // counter-set block [n_tt, E]: pairs of 128-token tile g per expert
     int sched;          // et_sched
     int bad_count;
+    // a dense MLP after the layer (the MoE -> MLP graph; mlp_xn null otherwise):
+    // each combine task also normalises its tokens' outputs for the MLP
+    uint16_t* mlp_xn;          // [maxT, hidden] MLP input rows, bf16(rmsnorm(y) gamma)
+    const uint16_t* mlp_gamma;
+    float mlp_eps;
+    int mlp_ev_norm;           // the MLP's E_norm (count T)
+    int mlp_n_gu;              // gate/up tasks queued by the combine completing E_norm (0 = none)
+    int extra_tasks;           // tasks of the MLP in the queue's total (dynamic schedule)
 };
 
 // ------------------------------------------------------------ decode layer
@@ -136,6 +145,15 @@ struct DecodeParams {
     int ev_branch_all, ev_merge_all, ev_gu_all, ev_down_all;
     int sched;
     int bad_count;
+};
+
+// ------------------------------------------------------ MoE -> dense MLP
+// The MoE layer followed by a dense SwiGLU MLP on its output, in one launch
+// (the MLP's gate/up, down and reduce tasks; its norm is run by the MoE's
+// combine tasks).
+struct MoeMlpParams {
+    MoeParams moe;
+    MlpParams mlp;
 };
 
 }  // namespace et

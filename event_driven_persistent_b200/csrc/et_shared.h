@@ -78,4 +78,42 @@ struct RunArgs {
 // Counter-set slots every workload reserves at the front.
 constexpr int kCtrHead = 0, kCtrTail = 1, kCtrTotal = 2, kCtrFirstEvent = 4;
 
+#ifdef __CUDACC__
+#define ET_HD __host__ __device__ __forceinline__
+#else
+#define ET_HD inline
+#endif
+
+// Circular allocation of pipeline stages in the smem arena; the producer and
+// the MMA issuer replay the same sequence, so both know every stage's
+// address.  A stage that does not fit before the end of the arena starts
+// again at offset 0.
+struct StageAlloc {
+    uint32_t head = 0;
+    ET_HD uint32_t next(uint32_t size) {
+        if (head + size > (uint32_t)kArenaBytes) head = 0;
+        const uint32_t o = head;
+        head += size;
+        return o;
+    }
+};
+
+// May the stage [off, off + size) be written while stages tail .. nst-1 are
+// still in flight (stage u occupies [r_off[u % kSlots], r_end[u % kSlots]))?
+// Not while its mbarrier slot is still held by stage nst - kSlots, nor while
+// any in-flight stage shares a byte with it.  Every in-flight stage is
+// checked: with mixed stage sizes an allocation can wrap to offset 0 while
+// the oldest stage sits near the end of the arena and newer ones already
+// occupy its start.  The producer waits for the oldest stage while this is
+// true (stages are consumed in order).
+ET_HD bool stage_blocked(uint32_t off, uint32_t size, uint32_t tail, uint32_t nst, const uint32_t* r_off,
+                         const uint32_t* r_end) {
+    if (nst - tail >= (uint32_t)kSlots) return true;
+    for (uint32_t u = tail; u < nst; ++u) {
+        const uint32_t us = u % kSlots;
+        if (off < r_end[us] && r_off[us] < off + size) return true;
+    }
+    return false;
+}
+
 }  // namespace et

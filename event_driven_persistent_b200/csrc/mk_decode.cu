@@ -30,20 +30,12 @@
 //   GU(n)        SwiGLU gate/up tile n (SiLU*mul epilogue)            -> E_h[c] [kchunk / 64]
 //   DOWN(m, c)   output tile m, K chunk c, sums added at L2           -> E_y[m] [#chunks]
 //   RED(m)       Y = bf16(h1 + down) for tile m
-#include <cuda_bf16.h>
-
-#include "et_engine.cuh"
+#include "et_math.cuh"
 #include "et_params.h"
 
 namespace et {
 
 namespace {
-__device__ __forceinline__ uint16_t bf16_bits(float v) { return __bfloat16_as_ushort(__float2bfloat16_rn(v)); }
-__device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
-__device__ __forceinline__ void red_add(float* p, float v) {
-    asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
 // contiguous global -> shared copy completing on an mbarrier (no multicast)
 __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
     asm volatile(
@@ -51,35 +43,6 @@ __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t b
             smem_u32(dst)),
         "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
-}
-__device__ __forceinline__ void bf16x8(uint4 u, float* f) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-// Exclusive prefix sum over the 128 exec threads; *total gets the sum.
-__device__ __forceinline__ int exec_scan(int v, int tid, int* tmp, int* total) {
-    const int lane = tid & 31, w = tid >> 5;
-    int inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-    }
-    if (lane == 31) tmp[w] = inc;
-    exec_bar();
-    int base = 0, tot = 0;
-#pragma unroll
-    for (int i = 0; i < kExecThreads / 32; ++i) {
-        base += i < w ? tmp[i] : 0;
-        tot += tmp[i];
-    }
-    exec_bar();
-    *total = tot;
-    return base + inc - v;
 }
 constexpr int kKeysPerStage = 128;
 constexpr uint32_t kAttnStageBytes = 2u * kKeysPerStage * 256u;  // K block then V block (head dim 128)
@@ -231,8 +194,9 @@ struct Decode : WorkloadBase {
         for (int h = 0; h < 4; ++h) {
             if (h < grp) {
                 const uint16_t* qr = p.q + ((size_t)bb * p.nq + g * grp + h) * p.hd;
-                bf16x8(*reinterpret_cast<const uint4*>(qr + 8 * j8), qv[h]);
-                bf16x8(*reinterpret_cast<const uint4*>(qr + 64 + 8 * j8), qv[h] + 8);
+                // (written during the run by another SM's branch: read through L2)
+                bf16x8(__ldcg(reinterpret_cast<const uint4*>(qr + 8 * j8)), qv[h]);
+                bf16x8(__ldcg(reinterpret_cast<const uint4*>(qr + 64 + 8 * j8)), qv[h] + 8);
             } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) qv[h][i] = 0.f;
@@ -264,10 +228,16 @@ struct Decode : WorkloadBase {
                     float kv[16];
                     bf16x8(*reinterpret_cast<const uint4*>(Ks + key * 256 + j8 * 16), kv);
                     bf16x8(*reinterpret_cast<const uint4*>(Ks + key * 256 + 128 + j8 * 16), kv + 8);
+                    float acc2[4] = {0.f, 0.f, 0.f, 0.f};  // two chains per head (latency, not work)
 #pragma unroll
                     for (int h = 0; h < 4; ++h)
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) acc[h] = fmaf(qv[h][i], kv[i], acc[h]);
+                        for (int i = 0; i < 8; ++i) {
+                            acc[h] = fmaf(qv[h][i], kv[i], acc[h]);
+                            acc2[h] = fmaf(qv[h][8 + i], kv[8 + i], acc2[h]);
+                        }
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) acc[h] += acc2[h];
                 }
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
@@ -313,16 +283,34 @@ struct Decode : WorkloadBase {
                 l[h] = l[h] * alpha[h] + red[16 + h] + red[20 + h] + red[24 + h] + red[28 + h];
                 o[h] *= alpha[h];
             }
+            // two chains per head over even and odd keys (nks is even unless it is the
+            // split's last stage; the odd tail key goes to the first chain)
             const uint16_t* vcol = reinterpret_cast<const uint16_t*>(Vs) + tid;
-#pragma unroll 4
-            for (int key = 0; key < nks; ++key) {
-                const float4 pp = pk[key];
-                const float v = bf16_val(vcol[key * 128]);
-                o[0] = fmaf(pp.x, v, o[0]);
-                o[1] = fmaf(pp.y, v, o[1]);
-                o[2] = fmaf(pp.z, v, o[2]);
-                o[3] = fmaf(pp.w, v, o[3]);
+            float o2[4] = {0.f, 0.f, 0.f, 0.f};
+            int key = 0;
+#pragma unroll 2
+            for (; key + 1 < nks; key += 2) {
+                const float4 pa = pk[key], pb = pk[key + 1];
+                const float va = bf16_val(vcol[key * 128]), vb = bf16_val(vcol[(key + 1) * 128]);
+                o[0] = fmaf(pa.x, va, o[0]);
+                o[1] = fmaf(pa.y, va, o[1]);
+                o[2] = fmaf(pa.z, va, o[2]);
+                o[3] = fmaf(pa.w, va, o[3]);
+                o2[0] = fmaf(pb.x, vb, o2[0]);
+                o2[1] = fmaf(pb.y, vb, o2[1]);
+                o2[2] = fmaf(pb.z, vb, o2[2]);
+                o2[3] = fmaf(pb.w, vb, o2[3]);
             }
+            if (key < nks) {
+                const float4 pa = pk[key];
+                const float va = bf16_val(vcol[key * 128]);
+                o[0] = fmaf(pa.x, va, o[0]);
+                o[1] = fmaf(pa.y, va, o[1]);
+                o[2] = fmaf(pa.z, va, o[2]);
+                o[3] = fmaf(pa.w, va, o[3]);
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) o[h] += o2[h];
             stream_stage_release(x, d, st);
         }
         // partial of this split: o (unnormalised), running max m, sum l
@@ -352,17 +340,36 @@ struct Decode : WorkloadBase {
         if (!group_wait(x, d, nullptr, 0, 310)) return false;
         const int tid = x.tid, stride = p.hd + 2;
         const float* base = p.part + (size_t)(bb * p.nkv + g) * p.s_max * p.grp * stride;
-        for (int h = 0; h < p.grp; ++h) {
+        // every split's (max, sum) of every head at once into smem: wgt[s][h]
+        // = exp(m_s - m*) and the normaliser 1 / sum_s wgt l_s
+        float* ml = x.epi;                 // [s_max * grp][2]
+        float* wgt = x.epi + 2 * 1024;     // [s_max * grp]
+        float* inv = wgt + 1024;           // [grp]
+        const int nsh = ns * p.grp;
+        for (int i = tid; i < nsh; i += kExecThreads) {
+            const float* q = base + (size_t)i * stride + p.hd;  // i = s * grp + h
+            ml[2 * i] = __ldcg(q);
+            ml[2 * i + 1] = __ldcg(q + 1);
+        }
+        exec_bar();
+        if (tid < p.grp) {
             float ms = -INFINITY;
-            for (int s = 0; s < ns; ++s) ms = fmaxf(ms, __ldcg(base + ((size_t)s * p.grp + h) * stride + p.hd));
-            float ls = 0.f, os = 0.f;
+            for (int s = 0; s < ns; ++s) ms = fmaxf(ms, ml[2 * (s * p.grp + tid)]);
+            float ls = 0.f;
             for (int s = 0; s < ns; ++s) {
-                const float* q = base + ((size_t)s * p.grp + h) * stride;
-                const float wgt = expf(__ldcg(q + p.hd) - ms);
-                ls = fmaf(wgt, __ldcg(q + p.hd + 1), ls);
-                os = fmaf(wgt, __ldcg(q + tid), os);
+                const float w8 = expf(ml[2 * (s * p.grp + tid)] - ms);
+                wgt[s * p.grp + tid] = w8;
+                ls = fmaf(w8, ml[2 * (s * p.grp + tid) + 1], ls);
             }
-            p.attn[(size_t)bb * p.nq * p.hd + (size_t)(g * p.grp + h) * p.hd + tid] = bf16_bits(os / ls);
+            inv[tid] = 1.0f / ls;
+        }
+        exec_bar();
+        // thread t = dim t: the splits' partial outputs, loads independent of each other
+        for (int h = 0; h < p.grp; ++h) {
+            float os = 0.f;
+#pragma unroll 4
+            for (int s = 0; s < ns; ++s) os = fmaf(wgt[s * p.grp + h], __ldcg(base + ((size_t)s * p.grp + h) * stride + tid), os);
+            p.attn[(size_t)bb * p.nq * p.hd + (size_t)(g * p.grp + h) * p.hd + tid] = bf16_bits(os * inv[h]);
         }
         fence_proxy_async_global();  // attn is read by TMA in the o-proj tasks
         int* ev = x.ctr + (unfused(p) ? p.ev_merge_all : p.ev_ag + g);
@@ -666,7 +673,7 @@ struct Decode : WorkloadBase {
             const size_t i = (size_t)b * p.hidden + col;
             const float a = __ldcg(p.yacc + i);
             __stcg(p.yacc + i, 0.f);
-            p.Y[i] = bf16_bits(bf16_val(p.h1[i]) + a);
+            p.Y[i] = bf16_bits(bf16_val(__ldcg(p.h1 + i)) + a);
         }
         group_finish_notify(x, d, nullptr, 0, 0);
         return true;

@@ -61,7 +61,7 @@ struct SplitK : WorkloadBase {
             for (int r = x.tid; r < nr; r += kExecThreads) {
                 const float* b = p.Bp + (size_t)(r0 + r) * p.n_chunks;
                 float s = 0.f;
-                for (int j = 0; j < p.n_chunks; ++j) s += b[j];
+                for (int j = 0; j < p.n_chunks; ++j) s += __ldcg(b + j);  // partials of other SMs: via L2
                 p.C[r0 + r] = s;
             }
             group_finish_notify(x, d, nullptr, 0, 0);

@@ -76,7 +76,13 @@ typedef enum {
                              o-proj and MLP static (part B); decode MLP: all static */
 } et_sched;
 
-typedef enum { ET_GRAPH_SPLITK = 0, ET_GRAPH_MLP = 1, ET_GRAPH_MOE = 2, ET_GRAPH_DECODE = 3 } et_graph_kind;
+typedef enum {
+    ET_GRAPH_SPLITK = 0,
+    ET_GRAPH_MLP = 1,
+    ET_GRAPH_MOE = 2,
+    ET_GRAPH_DECODE = 3,
+    ET_GRAPH_MOE_MLP = 4  /* the MoE layer followed by a dense SwiGLU MLP on its output */
+} et_graph_kind;
 
 /* debug_flags bits */
 #define ET_DEBUG_TRACE 1      /* record one et_trace_record per task (tickets from one global counter) */
@@ -106,8 +112,11 @@ typedef struct {
     int n_heads;         /* query heads [32] */
     int n_kv_heads;      /* key/value heads [8]; n_heads / n_kv_heads <= 4 */
     int head_dim;        /* [128]; only 128 is supported */
-    int max_ctx;         /* cache positions per request [4097]; a run's positions must be < max_ctx */
+    int max_ctx;         /* cache positions per request [4097]; a run's positions must be < max_ctx;
+                            at most 1024 * 256 / (n_heads / n_kv_heads) */
     float rope_base;     /* rotary embedding base [500000] */
+    /* MoE -> dense MLP (ET_GRAPH_MOE_MLP); the MoE dims above, the MLP's width = hidden */
+    int mlp_inter;       /* dense MLP intermediate width [6144] */
 } et_graph_desc;
 
 typedef struct et_graph et_graph; /* opaque, library-owned */
@@ -269,6 +278,21 @@ et_status et_run_mlp(et_graph* g, int B, const uint16_t* X, const uint16_t* gamm
 et_status et_run_moe(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
                      const uint16_t* W1, const uint16_t* W2, uint16_t* Y, int32_t* topk,
                      float* topk_w, int32_t* indptr, int32_t* perm, float* logits, void* stream);
+
+/* The MoE layer followed by a dense SwiGLU MLP on its output, in one launch
+ * ([ETN] §端到端低 batch serving: the MoE GroupGEMM and the dense MLP GEMM
+ * pipelined across stages; weights of the next stage prefetched before
+ * its activations arrive).  Each combine task of the MoE also takes the
+ * MLP's RMSNorm of its tokens, and the MLP's gate/up tasks stream their
+ * weights while the MoE finishes:
+ *   Y1 = the MoE layer of et_run_moe on X
+ *   Y2 = bf16(h Wd^T),  h = bf16(silu(xn Wg^T) * (xn Wu^T)),  xn = bf16(rmsnorm(Y1) gamma)
+ * MoE tensors as for et_run_moe; gamma bf16 [hidden]; Wgu bf16 [2 * mlp_inter,
+ * hidden] (gate rows first); Wd bf16 [hidden, mlp_inter]; Y1, Y2 bf16 [T, hidden].
+ * 1 <= T <= max_T <= 128. */
+et_status et_run_moe_mlp(et_graph* g, int T, const uint16_t* X, const uint16_t* Wr, const float* bias,
+                         const uint16_t* W1, const uint16_t* W2, const uint16_t* gamma, const uint16_t* Wgu,
+                         const uint16_t* Wd, uint16_t* Y1, uint16_t* Y2, void* stream);
 
 /* Weights of the decode layer (bf16 bits, device memory, row-major). */
 typedef struct {

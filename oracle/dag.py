@@ -651,3 +651,49 @@ def decode_dataflow(pos, nq, nkv, n_kc, split, n_m, n_gu, gu_tile, kchunk, n_c):
             rw[(OP_DEC_DOWN, m, c)] = (cols, {("down", m)})
         rw[(OP_DEC_RED, m, 0)] = ({("down", m)} | {("h1", b) for b in range(B)}, {("y", m)})
     return rw
+
+
+# ---------------------------------------------------------- MoE -> dense MLP --
+
+def moe_mlp_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched, hidden, inter, gu_tile, down_tile,
+                  kchunk):
+    """The MoE layer (moe_graph) followed by a dense MLP on its output: each
+    combine task CB(b) also normalises its tokens for the MLP and notifies
+    E_norm once per token (count T); the MLP's gate/up, down and reduce
+    tasks follow as in mlp_graph (no norm tasks of their own)."""
+    g, mt = moe_graph(topk, E, tt, n_kc, tkt, gt, bm, n_n1, n_n2, cb, sched)
+    T = len(topk)
+    unf = sched == "unfused"
+    m = mlp_graph(T, hidden, inter, gu_tile, down_tile, kchunk, sched)
+    for b in range(_cdiv(T, cb)):
+        g.produce((OP_MOE_COMBINE, b, 0), ("E_norm",), n=min(cb, T - b * cb))
+    for t in m.tasks:
+        if t[0] != OP_MLP_NORM:
+            g.add_task(t)
+    for ev, cons in m.event_consumers.items():
+        for c in cons:
+            g.consume(c, ev)
+    for ev, prods in m.event_producers.items():
+        if ev != ("E_norm",):
+            for p_ in prods:
+                g.produce(p_, ev)
+    for ev, wc in m.wait_count.items():
+        g.counted(ev, wc)
+    # mlp_graph's finish() already ran on m; rebuild this graph's edges
+    g.edges = set()
+    g.tasks = list(dict.fromkeys(g.tasks))
+    return g.finish(), mt
+
+
+def moe_mlp_dataflow(topk, n_kc, tkt, tt, bm, n_n1, n_n2, cb, E, hidden, inter, gu_tile, down_tile, kchunk):
+    """moe_dataflow plus the MLP: CB(b) also writes ("xn", t) of its tokens,
+    the MLP tasks read and write as in mlp_dataflow."""
+    rw = moe_dataflow(topk, n_kc, tkt, tt, bm, n_n1, n_n2, cb, E)
+    T = len(topk)
+    for b in range(_cdiv(T, cb)):
+        r, w = rw[(OP_MOE_COMBINE, b, 0)]
+        rw[(OP_MOE_COMBINE, b, 0)] = (r, w | {("xn", t) for t in range(b * cb, min(T, (b + 1) * cb))})
+    for task, v in mlp_dataflow(T, hidden, inter, gu_tile, down_tile, kchunk).items():
+        if task[0] != OP_MLP_NORM:
+            rw[task] = v
+    return rw

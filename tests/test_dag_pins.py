@@ -258,3 +258,26 @@ def test_decode_dataflow_catches_a_split_before_its_cache_append():
     recs = _trace_priority(g2, {(A, 2, 2)}, {(KBR, 4, 0)})
     assert dag.check_trace(g2, recs) == []
     assert any("read before write" in e for e in dag.check_dataflow(rw, recs))
+
+
+# ------------------------------------------------------- MoE -> dense MLP --
+
+def test_moe_mlp_graph_counts_and_dataflow():
+    """The combine of block b notifies the MLP's E_norm once per token (count
+    T); the MLP's gate/up tasks follow every combine."""
+    for sched in ("static", "dynamic", "unfused"):
+        topk = np.array([[1, 0], [0, 2], [2, 1]])
+        kw = dict(E=3, tt=4, n_kc=1, tkt=2, gt=4, bm=2, n_n1=1, n_n2=1, cb=2)
+        mk = dict(hidden=256, inter=256, gu_tile=64, down_tile=128, kchunk=128)
+        g, _ = dag.moe_mlp_graph(topk, sched=sched, **kw, **mk)
+        assert dag.check_wait_counts(g) == []
+        assert g.wait_count[("E_norm",)] == 3
+        for b in range(2):
+            assert ((dag.OP_MOE_COMBINE, b, 0), (dag.OP_MLP_GATEUP, 0, 0)) in g.edges
+        rw = dag.moe_mlp_dataflow(topk, n_kc=1, tkt=2, tt=4, bm=2, n_n1=1, n_n2=1, cb=2, E=3, **mk)
+        assert dag.check_dataflow(rw, _trace_priority(g, set())) == []
+        # the MLP reading a token's input before its combine wrote it is caught
+        g2 = _drop(g, lambda p, c: p == (dag.OP_MOE_COMBINE, 1, 0) and c[0] == dag.OP_MLP_GATEUP)
+        recs = _trace_priority(g2, {t for t in g2.tasks if t[0] == dag.OP_MLP_GATEUP}, {(dag.OP_MOE_COMBINE, 1, 0)})
+        assert dag.check_trace(g2, recs) == []
+        assert any("read before write" in e for e in dag.check_dataflow(rw, recs))

@@ -79,15 +79,18 @@ def test_decode_small_dims(small_inputs, sched, B):
 
 @pytest.mark.parametrize("sched", ["static", "hybrid"])
 def test_decode_edge_positions(small_inputs, sched):
-    """One key (position 0), a split holding only the new key (256), the last
-    key of a split (255, 511), the last cache position (599)."""
+    """One key (position 0); the last key of a 128-key stage and the first of
+    the next (127, 128); the last key of a split and a split holding only the
+    new key (split - 1, split); the last cache position (599)."""
     d = small_inputs
-    pos = np.array([0, 255, 256, 511, 599], np.int32)
     g = et.et_build_graph(et.ET_GRAPH_DECODE, sched, 8, max_ctx=600, **SMALL)
     try:
-        st, out = run_decode(g, d, 5, pos=pos)
+        sp = et.et_get_info(g)["dec_split"]
+        pos = np.array([0, 127, 128, sp - 1, sp, 599], np.int32)
+        assert pos.max() < 600
+        st, out = run_decode(g, d, 6, pos=pos)
         assert st == 0
-        check(d, out, 5, 4, 2, pos=pos)
+        check(d, out, 6, 4, 2, pos=pos)
     finally:
         et.et_destroy_graph(g)
 

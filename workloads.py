@@ -16,6 +16,9 @@ Recipe (numpy PCG64 ``default_rng(seed)``):
            0..E-1 (a Zipf(s) popularity prior on the experts; s = 0 gives
            zero bias)                                              seeds 100+log2(T) (1000+T when T is
            not a power of two), 20, 21, 22, 23
+  MoE->MLP the MoE inputs above, then a dense MLP on the layer's output:
+           gamma ~ N(1, 0.1), Wgu [2*mlp_inter, hidden], Wd [hidden,
+           mlp_inter] ~ N(0, 0.02)                                  seeds 50, 51, 52
   decode   X [B, hidden] ~ N(0,1); context lengths ~ U{512..4096} (the
            new token's position); K and V caches [B, n_kv, max_ctx, hd]
            ~ N(0,1) at the cached positions, zero beyond;
@@ -118,3 +121,10 @@ def decode_inputs(B, hidden=4096, n_q=32, n_kv=8, hd=128, inter=14336, ctx_lo=51
         d["Wgu"] = _normal_bf16(np.random.default_rng(12), (2 * inter, hidden), 0.0, 0.02)
         d["Wd"] = _normal_bf16(np.random.default_rng(13), (hidden, inter), 0.0, 0.02)
     return d
+
+
+def dense_mlp_weights(hidden=2048, inter=6144):
+    """dict(gamma, Wgu, Wd) of the dense MLP after the MoE layer."""
+    return dict(gamma=_normal_bf16(np.random.default_rng(50), (hidden,), 1.0, 0.1),
+                Wgu=_normal_bf16(np.random.default_rng(51), (2 * inter, hidden), 0.0, 0.02),
+                Wd=_normal_bf16(np.random.default_rng(52), (hidden, inter), 0.0, 0.02))
