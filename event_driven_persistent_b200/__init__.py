@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 ET_OK, ET_ERR_INVALID, ET_ERR_CUDA, ET_ERR_TIMEOUT, ET_ERR_OOM, ET_ERR_UNSUPPORTED, ET_ERR_PENDING, ET_ERR_INTERNAL = range(8)
 ET_SCHED_STATIC, ET_SCHED_DYNAMIC, ET_SCHED_UNFUSED, ET_SCHED_HYBRID = 0, 1, 2, 3
 ET_GRAPH_SPLITK, ET_GRAPH_MLP, ET_GRAPH_MOE, ET_GRAPH_DECODE, ET_GRAPH_MOE_MLP = 0, 1, 2, 3, 4
-ET_DEBUG_TRACE, ET_DEBUG_DELAY, ET_DEBUG_BAD_COUNT = 1, 2, 4
+ET_DEBUG_TRACE, ET_DEBUG_DELAY, ET_DEBUG_BAD_COUNT, ET_DEBUG_CTA_TIMES = 1, 2, 4, 8
 SCHED = {"static": ET_SCHED_STATIC, "dynamic": ET_SCHED_DYNAMIC, "unfused": ET_SCHED_UNFUSED,
          "hybrid": ET_SCHED_HYBRID}
 

@@ -288,10 +288,11 @@ __device__ __forceinline__ bool aborted(const Ctl* ctl) { return ld_volatile(&ct
 // Spin budget: time limit (ns) and a hard iteration cap, whichever comes first.
 constexpr uint32_t kMaxSpinIters = 1u << 26;
 
-// wait(): spin until *ctr >= target.  false on timeout/abort.
-static __device__ __noinline__ bool wait_geq(const int* ctr, int target, Ctl* ctl, uint64_t timeout_ns, int where,
-                                      int ev) {
-    if (ld_acquire(ctr) >= target) return true;
+// wait(): spin until *ctr >= target.  false on timeout/abort.  The check
+// of an event that is already complete is inline; the bounded spin is out
+// of line (many call sites; the megakernel's instruction footprint matters).
+static __device__ __noinline__ bool wait_geq_spin(const int* ctr, int target, Ctl* ctl, uint64_t timeout_ns, int where,
+                                                  int ev) {
     uint64_t t0 = globaltimer();
     Backoff bo;
     for (uint32_t it = 1;; ++it) {
@@ -309,6 +310,10 @@ static __device__ __noinline__ bool wait_geq(const int* ctr, int target, Ctl* ct
         }
     }
 }
+__device__ __forceinline__ bool wait_geq(const int* ctr, int target, Ctl* ctl, uint64_t timeout_ns, int where, int ev) {
+    if (ld_acquire(ctr) >= target) return true;
+    return wait_geq_spin(ctr, target, ctl, timeout_ns, where, ev);
+}
 
 // notify(): add n with release (and acquire, so that the notifier that
 // completes an event has seen every earlier producer's writes before it
@@ -318,10 +323,10 @@ __device__ __forceinline__ int notify(int* ctr, int n) {
     return atom_add_acq_rel(ctr, n) + n;
 }
 
-// bounded mbarrier wait (parity); false on timeout/abort.  Out of line: it
-// has many call sites and the megakernel's instruction footprint matters.
-static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Ctl* ctl, uint64_t timeout_ns, int where) {
-    if (mbar_try_wait(b, parity)) return true;
+// bounded mbarrier wait (parity); false on timeout/abort.  A phase that is
+// already complete is seen inline; the bounded spin is out of line.
+static __device__ __noinline__ bool mbar_wait_spin(uint64_t* b, uint32_t parity, Ctl* ctl, uint64_t timeout_ns,
+                                                   int where) {
     uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(b, parity)) return true;
@@ -333,6 +338,10 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Ctl*
             }
         }
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Ctl* ctl, uint64_t timeout_ns, int where) {
+    if (mbar_try_wait(b, parity)) return true;
+    return mbar_wait_spin(b, parity, ctl, timeout_ns, where);
 }
 
 // ---------------------------------------------------------------- trace ----

@@ -243,6 +243,9 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Ctl* ctl = ra.ctl;
+    const bool cta_times = (ra.debug & (ET_DEBUG_TRACE | ET_DEBUG_CTA_TIMES)) == (ET_DEBUG_TRACE | ET_DEBUG_CTA_TIMES);
+    uint64_t t_enter = 0, t_setup = 0;
+    if (cta_times && threadIdx.x == 0) t_enter = globaltimer();
 
     // zero the other parity's counter set for the next run
     {
@@ -275,6 +278,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     __syncthreads();
     tc_fence_after();
     const bool skip = sc->start_status != 0;  // an earlier run failed: do nothing until the host resets
+    if (cta_times && threadIdx.x == 0) t_setup = globaltimer();
 
     Ctx x;
     x.ctl = ctl;
@@ -502,8 +506,14 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     // B rows gathered through an index list: every lane copies
                     // up to 4 rows per stage with cp.async into the 128-byte
                     // swizzled layout; lane 0 adds the weight tile by TMA.
-                    // (the start ticket is taken before the index list is read)
+                    // The rows' index list is read first: its L2 round trip
+                    // overlaps the hand-off.  (A gathered task's inputs are
+                    // complete when it is derived: derive waits for them, or
+                    // the queue holds the task only once they are.)
                     any_gather = true;
+                    const uint16_t* rows[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) rows[i] = W::gather_row(p, d, lane + 32 * i);
                     if (lane == 0) {
                         ok = W::gemm_wait(p, x, d);
                         if (ok && (x.debug & ET_DEBUG_TRACE)) {
@@ -517,9 +527,6 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     __syncwarp();
                     ok = sc->pok;
                     __syncwarp();
-                    const uint16_t* rows[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) rows[i] = ok ? W::gather_row(p, d, lane + 32 * i) : nullptr;
                     for (int s = 0; s < d.nk && ok; ++s) {
                         if (lane == 0) {
                             uint32_t sl = 0, of = 0;
@@ -671,6 +678,9 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
         tc_fence_after();
         tmem_dealloc(sc->tmem_base, kTmemCols);
     }
+    if (cta_times && threadIdx.x == 0)
+        trace_task(ctl, ra.trace, ra.trace_cap, task_word(ET_OP_CTA, blockIdx.x, 0), 0, t_enter, t_setup, 0, 0,
+                   globaltimer());
 }
 
 // Epilogue helper: read this warp's 32 lanes x 16 columns [c0, c0+16) of

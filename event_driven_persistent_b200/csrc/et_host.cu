@@ -724,7 +724,7 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     if ((st = galloc(g, &g->ctr[0], g->n_ctr)) != ET_OK) return fail(st);
     if ((st = galloc(g, &g->ctr[1], g->n_ctr)) != ET_OK) return fail(st);
     if ((st = galloc(g, &g->qslots, g->qcap)) != ET_OK) return fail(st);
-    g->trace_cap = (g->d.debug_flags & ET_DEBUG_TRACE) ? g->qcap + 1024 : 1;
+    g->trace_cap = (g->d.debug_flags & ET_DEBUG_TRACE) ? g->qcap + 1024 + 256 : 1;  // + one record per CTA (ET_DEBUG_CTA_TIMES)
     if ((st = galloc(g, &g->trace, g->trace_cap)) != ET_OK) return fail(st);
     if (cudaDeviceSynchronize() != cudaSuccess) return fail(ET_ERR_CUDA);
     // info

@@ -23,6 +23,12 @@ __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 __device__ __forceinline__ void red_add(float* p, float v) {
     asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
+// Four consecutive fp32 sums at L2 in one request (p 16-byte aligned).
+__device__ __forceinline__ void red_add4(float* p, float4 v) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
 
 // Exclusive prefix sum over the 128 exec threads (value v of thread tid);
 // returns the prefix, *total gets the sum.  `tmp` holds 4 ints of smem.

@@ -101,19 +101,20 @@ struct StageAlloc {
 // May the stage [off, off + size) be written while stages tail .. nst-1 are
 // still in flight (stage u occupies [r_off[u % kSlots], r_end[u % kSlots]))?
 // Not while its mbarrier slot is still held by stage nst - kSlots, nor while
-// any in-flight stage shares a byte with it.  Every in-flight stage is
-// checked: with mixed stage sizes an allocation can wrap to offset 0 while
-// the oldest stage sits near the end of the arena and newer ones already
-// occupy its start.  The producer waits for the oldest stage while this is
-// true (stages are consumed in order).
+// an in-flight stage shares a byte with it.  Consecutive stages are adjacent
+// unless an allocation wrapped to offset 0, and a second wrap cannot happen
+// while stages of the first are in flight (the wrapping stage would overlap
+// them), so the stages in flight cover exactly [lo, hi) -- lo the oldest
+// stage's start, hi the newest stage's end -- or, wrapped, [lo, arena end)
+// and [0, hi).  O(1); the producer waits for the oldest stage (stages are
+// consumed in order) while this is true.
 ET_HD bool stage_blocked(uint32_t off, uint32_t size, uint32_t tail, uint32_t nst, const uint32_t* r_off,
                          const uint32_t* r_end) {
+    if (tail == nst) return false;
     if (nst - tail >= (uint32_t)kSlots) return true;
-    for (uint32_t u = tail; u < nst; ++u) {
-        const uint32_t us = u % kSlots;
-        if (off < r_end[us] && r_off[us] < off + size) return true;
-    }
-    return false;
+    const uint32_t lo = r_off[tail % kSlots], hi = r_end[(nst - 1) % kSlots];
+    if (lo < hi) return off < hi && lo < off + size;
+    return off < hi || lo < off + size;
 }
 
 }  // namespace et

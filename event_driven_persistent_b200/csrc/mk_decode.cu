@@ -20,7 +20,7 @@
 //                  Q head:  bf16 -> per-head rmsnorm gq -> RoPE -> q
 //                  K head:  bf16 -> per-head rmsnorm gk -> RoPE -> cache[b, g, pos_b]
 //                  V head:  bf16 -> cache[b, g, pos_b]                 -> E_g[g] [grp + 2]
-//   ATTN(b, g, s) keys [256 s, 256 s + 256) of request b, KV head g, all grp
+//   ATTN(b, g, s) keys [S s, S s + S) of request b (S = the split, 512 keys), KV head g, all grp
 //                query heads: streamed through the stage arena (K and V
 //                blocks of 128 keys), online softmax; partial (o, m, l)  -> E_att[b, g] [#splits(b)]
 //                the split completing (b, g) merges the partials inline  -> E_ag[g] [B]

@@ -227,7 +227,6 @@ struct Moe : WorkloadBase {
                 group_push(x, p.n_n2, [&](int n2) { return task_word(ET_OP_MOE_S2, a, n2); });
         } else {  // S2
             const int row0 = d.p[1], cnt = d.p[2];
-            const int col = b * p.n2_tile + r;
             int* s_tok = reinterpret_cast<int*>(x.simt);  // [128] token of each row
             float* s_w = reinterpret_cast<float*>(s_tok + 128);
             if (x.tid < cnt) {
@@ -236,15 +235,26 @@ struct Moe : WorkloadBase {
                 s_w[x.tid] = __ldcg(p.topw + pp);
             }
             exec_bar();
+            // weighted rows into Yacc: each warp turns its 32 columns x 16
+            // tokens around through smem so a lane adds 4 consecutive columns
+            // of one token with one vector reduction
+            float* tr = x.epi + w * 512;  // [16 tokens][32 columns] per warp
+            const int j4 = (lane & 7) * 4;
+            float* ybase = p.Yacc + b * p.n2_tile + q * 32 + j4;
             for (int c0 = 0; c0 < d.n; c0 += 16) {
                 float v[16];
                 acc_load16(taddr, c0, v);
                 if (c0 + 16 >= d.n) acc_release(acc_empty);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int c = c0 + i;
-                    if (c < cnt) red_add(p.Yacc + (size_t)s_tok[c] * p.hidden + col, s_w[c] * v[i]);
+                for (int i = 0; i < 16; ++i) tr[i * 32 + lane] = s_w[c0 + i] * v[i];
+                __syncwarp();
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int ci = (lane >> 3) + 4 * u, c = c0 + ci;
+                    if (c < cnt)
+                        red_add4(ybase + (size_t)s_tok[c] * p.hidden, *reinterpret_cast<const float4*>(tr + ci * 32 + j4));
                 }
+                __syncwarp();
             }
             if (is_unfused(p)) {
                 group_finish_notify(x, d, x.ctr + p.ev_s2_all, 1, -1);

@@ -105,6 +105,7 @@ __global__ void splitk_final_kernel(const float* Bp, int rows, int nch, float* C
 cudaError_t launch_splitk_two(const float* A, int rows, int cols, int chunk, float* Bp, float* C, cudaStream_t s) {
     const int nch = (cols + chunk - 1) / chunk;
     const long warps = (long)rows * nch;
+    (void)cudaGetLastError();  // an earlier, unrelated non-sticky error is not this launch's
     splitk_partial_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(A, rows, cols, chunk, nch, Bp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

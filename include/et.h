@@ -89,6 +89,8 @@ typedef enum {
 #define ET_DEBUG_DELAY 2      /* each task first spins a pseudo-random 0..~20 us, to perturb the order */
 #define ET_DEBUG_BAD_COUNT 4  /* raise one event's wait count by one: a run must then end in
                                  ET_ERR_TIMEOUT (used to test the timeout path) */
+#define ET_DEBUG_CTA_TIMES 8  /* with ET_DEBUG_TRACE: also one ET_OP_CTA record per CTA (a = CTA):
+                                 t_fetch = kernel entry, t_ready = set-up done, t_end = roles done */
 
 typedef struct {
     int kind;            /* et_graph_kind */
@@ -179,6 +181,7 @@ typedef struct {
 #define ET_OP_DEC_GATEUP 39   /* a = intermediate tile */
 #define ET_OP_DEC_DOWN 40     /* a = output tile, b = K chunk */
 #define ET_OP_DEC_RED 41      /* a = output tile */
+#define ET_OP_CTA 60          /* ET_DEBUG_CTA_TIMES: a = CTA index (not a task) */
 
 /* Event kinds of et_event_count records; index = the event's coordinate. */
 #define ET_EV_SK_TILE 1       /* split-K E[i]: partial tasks of row tile i done (count = #chunks) */

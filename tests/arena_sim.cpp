@@ -6,7 +6,8 @@
 //
 // argv[1] = seed, argv[2] = reservations, argv[3] = 1 to use the rule that
 // only checks the oldest in-flight stage (expected to fail: the regression
-// this simulation guards against).
+// this simulation guards against).  With the library's rule every decision
+// is also compared with a brute-force check over the stages in flight.
 #include <cstdio>
 #include <cstdlib>
 #include <deque>
@@ -55,6 +56,17 @@ int main(int argc, char** argv) {
         for (;;) {
             const bool blocked = tail < nst && (tail_only ? tail_only_blocked(off, size, tail, nst, r_off, r_end)
                                                           : stage_blocked(off, size, tail, nst, r_off, r_end));
+            if (!tail_only) {
+                // the O(1) rule must agree with the brute-force one both ways:
+                // no overwrite, and no wait that is not needed
+                bool brute = inflight.size() >= (size_t)kSlots;
+                for (const Range& r : inflight) brute = brute || (off < r.hi && r.lo < off + size);
+                if (brute != blocked) {
+                    printf("stage %ld [%u, %u): rule says %d, brute force %d\n", i, off, off + size, (int)blocked,
+                           (int)brute);
+                    return 4;
+                }
+            }
             if (!blocked) break;
             ++tail;  // wait for the oldest stage
             inflight.pop_front();
