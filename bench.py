@@ -312,6 +312,7 @@ def other_arm(args):
         B = args.B
         d = W.decode_inputs(B)
         wkeys = ("g1", "Wqkv", "gq", "gk", "Wo", "g2", "Wgu", "Wd")
+        d["Vc"] = W.v_cache_device(d["Vc"])  # the device's V cache layout
         t = {n: to_dev(d[n]) for n in wkeys + ("X", "pos", "Kc", "Vc")}
         Y = torch.empty((B, 4096), dtype=torch.int16, device=dev)
         sched = args.sched

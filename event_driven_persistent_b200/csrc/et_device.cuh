@@ -233,6 +233,17 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 // destination registers of tcgen05.ld are written asynchronously and are
 // only valid after tcgen05.wait::ld, so the compiler must not see them as
 // defined (and schedule their uses) before the wait.
+__device__ __forceinline__ void tmem_ld4_wait(uint32_t taddr, float (&v)[4]) {
+    uint32_t r[4];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
     asm volatile(
@@ -342,6 +353,19 @@ static __device__ __noinline__ bool mbar_wait_spin(uint64_t* b, uint32_t parity,
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Ctl* ctl, uint64_t timeout_ns, int where) {
     if (mbar_try_wait(b, parity)) return true;
     return mbar_wait_spin(b, parity, ctl, timeout_ns, where);
+}
+
+// A phase that one thread of a group has already seen complete, observed by
+// every other thread of the group (acquire per thread).  It cannot advance
+// again before the whole group moves on, so this ends at once; the loop is
+// still bounded, and a bound that runs out is recorded as ET_ERR_TIMEOUT
+// (the caller carries on; the run then aborts at its next check).
+__device__ __forceinline__ void mbar_observe(uint64_t* b, uint32_t parity, Ctl* ctl, int where) {
+    for (uint32_t it = 0; !mbar_try_wait(b, parity); ++it)
+        if (it > (1u << 20)) {
+            fail(ctl, ET_ERR_TIMEOUT, where, (int)parity, -1, 0);
+            return;
+        }
 }
 
 // ---------------------------------------------------------------- trace ----

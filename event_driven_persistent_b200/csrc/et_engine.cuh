@@ -43,6 +43,8 @@ struct TaskDesc {
                                 //     the exec group consumes them (no tensor-core work)
     uint32_t sbytes;            // stream: bytes reserved per stage (1 KB multiple)
     uint32_t st0, off0;         // stream: global index and arena offset of the task's first stage
+    int attn;                   // stream task whose stages also run two tensor-core products per
+                                //     stage (the attention protocol: S = K Q^T, then O = V^T P^T)
     int p[6];                   // workload-specific
 };
 
@@ -55,6 +57,7 @@ struct SmemCtl {
     uint64_t ring_full[kRing];
     uint64_t ring_empty[kRing];
     uint64_t drain;
+    uint64_t s_full, p_full, o_full;  // attention stages: S in TMEM / P in smem / O in TMEM
     uint32_t tmem_base;
     int start_status;
     int bcast[8];
@@ -81,19 +84,30 @@ struct Ctx {
     uint8_t* simt;       // CUDA-core task scratch
     SmemCtl* sc;
     int tid;             // exec-group thread index 0..127 (exec warps only)
+    // attention stream tasks (exec group): this task's TMEM accumulator (this
+    // warp's lane quadrant), its release barrier, and the attention stages
+    // consumed so far (the phase of s_full / p_full / o_full)
+    uint32_t taddr;
+    uint64_t* acc_empty;
+    uint32_t na;
 };
 
 // Defaults of the workload interface for what a workload does not use.
 struct WorkloadBase {
     // stream tasks: stages that may be copied before the task's input wait,
     // the bytes stage s delivers, and the copies of stage s into `dst`
-    // (completing on `bar`)
+    // (completing on `bar`); `late` = issued after the input wait, so the
+    // copies that depend on the task's inputs are included
     template <class P>
     __device__ static int stream_prefetch(const P&, const TaskDesc&) { return 0; }
     template <class P>
     __device__ static uint32_t stream_bytes(const P&, const TaskDesc&, int) { return 0; }
     template <class P>
-    __device__ static void stream_copy(const P&, const TaskDesc&, int, uint8_t*, uint64_t*, uint64_t) {}
+    __device__ static void stream_copy(const P&, const TaskDesc&, int, uint8_t*, uint64_t*, uint64_t, bool) {}
+    // the input-dependent copies of stage s, which was copied before the
+    // wait (its expected bytes counted them)
+    template <class P>
+    __device__ static void stream_late(const P&, const TaskDesc&, int, uint8_t*, uint64_t*, uint64_t) {}
     template <class P>
     __device__ static bool stream_exec(const P&, Ctx&, TaskDesc&) { return false; }
 };
@@ -200,15 +214,25 @@ __device__ __forceinline__ bool stream_stage_wait(Ctx& x, const TaskDesc& d, int
     if (x.tid == 0) x.sc->bcast[5] = mbar_wait(&x.sc->full[slot], par, x.ctl, x.timeout_ns, 925);
     exec_bar();
     const bool ok = x.sc->bcast[5] != 0;
-    if (ok)
-        while (!mbar_try_wait(&x.sc->full[slot], par)) {
-        }
+    if (ok) mbar_observe(&x.sc->full[slot], par, x.ctl, 926);
     return ok;
 }
 // ... and hand stage s back to the producer once every thread is done with it.
 __device__ __forceinline__ void stream_stage_release(Ctx& x, const TaskDesc& d, int s) {
     exec_bar();
     if (x.tid == 0) mbar_arrive(&x.sc->empty[(d.st0 + (uint32_t)s) % kSlots]);
+}
+// Exec group: wait for phase `parity` of an mbarrier that another role
+// completes (all 128 threads call; false on timeout/abort).  Thread 0 waits
+// with the bound and broadcasts through bcast[slot]; then every thread
+// observes the phase itself.  A slot is written again only after another
+// exec-group barrier, so no thread can read a later call's result.
+__device__ __forceinline__ bool exec_mbar_wait(Ctx& x, uint64_t* bar, uint32_t parity, int where, int slot) {
+    if (x.tid == 0) x.sc->bcast[slot] = mbar_wait(bar, parity, x.ctl, x.timeout_ns, where);
+    exec_bar();
+    const bool ok = x.sc->bcast[slot] != 0;
+    if (ok) mbar_observe(bar, parity, x.ctl, where + 1000);
+    return ok;
 }
 __device__ __forceinline__ StageAlloc stream_alloc(const TaskDesc& d) {
     StageAlloc a;
@@ -267,6 +291,9 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             mbar_init(&sc->ring_empty[r], 2);  // MMA warp + exec group
         }
         mbar_init(&sc->drain, 1);
+        mbar_init(&sc->s_full, 1);
+        mbar_init(&sc->p_full, 1);
+        mbar_init(&sc->o_full, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
@@ -302,6 +329,9 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     x.simt = simt;
     x.sc = sc;
     x.tid = threadIdx.x - kExecWarp0 * 32;
+    x.taddr = 0;
+    x.acc_empty = nullptr;
+    x.na = 0;
 
 
     if (!skip && warp == 0) {
@@ -372,6 +402,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 d.gemm = 0;
                 d.gather = 0;
                 d.stream = 0;
+                d.attn = 0;
                 d.start = 0;
                 d.t_fetch = d.t_ready = d.t_acc = 0;
                 int r = 0;
@@ -435,24 +466,31 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         StageAlloc probe = alloc;  // where the first stage will land
                         d.off0 = probe.head;
                     }
-                    auto issue_s = [&](int st) -> bool {
+                    uint32_t pre_sl[kSlots], pre_of[kSlots];  // the stages copied before the wait
+                    auto issue_s = [&](int st, bool late) -> bool {
                         uint32_t sl, of;
                         if (!reserve(d.sbytes, &sl, &of)) return false;
+                        if (!late) {
+                            pre_sl[st] = sl;
+                            pre_of[st] = of;
+                        }
                         mbar_arrive_expect_tx(&sc->full[sl], W::stream_bytes(p, d, st));
                         ++armed[sl];
-                        W::stream_copy(p, d, st, arena + of, &sc->full[sl], pol_w);
+                        W::stream_copy(p, d, st, arena + of, &sc->full[sl], pol_w, late);
                         return true;
                     };
                     int s2 = 0;
-                    for (; s2 < npre && ok; ++s2) ok = issue_s(s2);
+                    for (; s2 < npre && ok; ++s2) ok = issue_s(s2, false);
                     if (ok) ok = W::gemm_wait(p, x, d);  // the task's input events
+                    if (ok) fence_proxy_async_global();  // inputs written this run -> the copies below
                     if (ok && (x.debug & ET_DEBUG_TRACE)) {
                         d.start = take_ticket(ctl);
                         d.t_ready = globaltimer();
                     }
                     sc->ring[slot] = d;
                     mbar_arrive(&sc->ring_full[slot]);
-                    for (; ok && s2 < d.nk; ++s2) ok = issue_s(s2);
+                    for (int i = 0; ok && i < s2; ++i) W::stream_late(p, d, i, arena + pre_of[i], &sc->full[pre_sl[i]], pol_a);
+                    for (; ok && s2 < d.nk; ++s2) ok = issue_s(s2, true);
                     sc->pok = ok;
                 }
                 __syncwarp();
@@ -579,7 +617,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     } else if (!skip && warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------------ MMA issuer
-            uint32_t nst = 0, g = 0;
+            uint32_t nst = 0, g = 0, na = 0;
             StageAlloc alloc;
             bool issued_any = false;
             for (uint32_t it = 0;; ++it) {
@@ -588,8 +626,63 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 TaskDesc d = sc->ring[slot];
                 mbar_arrive(&sc->ring_empty[slot]);
                 if (d.word == kExitWord) break;
-                if (d.valid && d.stream) {  // stages consumed by the exec group: keep the sequence
+                if (d.valid && d.stream && !d.attn) {  // stages consumed by the exec group: keep the sequence
                     for (int s = 0; s < d.nk; ++s, ++nst) alloc.next(d.sbytes);
+                    continue;
+                }
+                if (d.valid && d.stream) {
+                    // attention stages: S = K Q^T into columns [0, 16) of the
+                    // task's accumulator (keys x query heads), then, once the
+                    // exec group has read S and written P (query heads x keys,
+                    // bf16) to its scratch, O = V^T P^T into columns [16, 32)
+                    // (head dims x query heads); the stage is free after that
+                    const uint32_t buf = g & 1;
+                    if (!mbar_wait(&sc->acc_empty[buf], ((g >> 1) & 1) ^ 1, ctl, x.timeout_ns, 913)) break;
+                    tc_fence_after();
+                    const uint32_t dS = sc->tmem_base + buf * kMaxN, dO = dS + 16;
+                    const uint32_t idesc = idesc_bf16_f32(128, 16);
+                    const uint32_t pa = smem_u32(epi);
+                    bool ok = true;
+                    for (int s = 0; s < d.nk; ++s, ++nst, ++na) {
+                        const uint32_t ss = nst % kSlots;
+                        const uint32_t off = alloc.next(d.sbytes);
+                        if (!mbar_wait(&sc->full[ss], (nst / kSlots) & 1, ctl, x.timeout_ns, 914)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t ka = smem_u32(arena + off), va = ka + kAttnVOff, qa = ka + kAttnQOff;
+#pragma unroll
+                        for (int at = 0; at < 2; ++at) {
+                            const uint64_t ad = sdesc_k128(ka + at * kAAtomBytes);
+                            const uint64_t bd = sdesc_k128(qa + at * 16u * 128u);
+#pragma unroll
+                            for (int kk = 0; kk < kAtomK / 16; ++kk)
+                                tc_mma_bf16(dS, ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
+                        }
+                        tc_commit(&sc->s_full);
+                        issued_any = true;
+                        if (!mbar_wait(&sc->p_full, na & 1, ctl, x.timeout_ns, 915)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int at = 0; at < 2; ++at) {
+                            const uint64_t ad = sdesc_k128(va + at * kAAtomBytes);
+                            const uint64_t bd = sdesc_k128(pa + at * 16u * 128u);
+#pragma unroll
+                            for (int kk = 0; kk < kAtomK / 16; ++kk)
+                                tc_mma_bf16(dO, ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
+                        }
+                        tc_commit(&sc->o_full);
+                        tc_commit(&sc->empty[ss]);
+                    }
+                    if (!ok) break;
+                    // one acc_full phase per use of an accumulator, attention
+                    // tasks included: the epilogues' parity counts on it
+                    tc_commit(&sc->acc_full[buf]);
+                    ++g;
                     continue;
                 }
                 if (!(d.valid && d.gemm)) continue;
@@ -650,6 +743,12 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             if (!d.valid) continue;
             if (x.debug & ET_DEBUG_DELAY) debug_delay(d.word ^ (ra.epoch * 977u));
             if (d.stream) {
+                if (d.attn) {
+                    const uint32_t buf = g & 1;
+                    x.taddr = sc->tmem_base + buf * kMaxN + ((uint32_t)((warp & 3) * 32) << 16);
+                    x.acc_empty = &sc->acc_empty[buf];
+                    ++g;
+                }
                 if (!W::stream_exec(p, x, d)) break;
             } else if (d.gemm) {
                 const uint32_t buf = g & 1;
@@ -657,8 +756,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 if (x.tid == 0) sc->bcast[5] = mbar_wait(&sc->acc_full[buf], par, ctl, x.timeout_ns, 921);
                 exec_bar();
                 if (!sc->bcast[5]) break;
-                while (!mbar_try_wait(&sc->acc_full[buf], par)) {
-                }
+                mbar_observe(&sc->acc_full[buf], par, ctl, 922);
                 if (x.debug & ET_DEBUG_TRACE) d.t_acc = globaltimer();
                 tc_fence_after();
                 const uint32_t taddr = sc->tmem_base + buf * kMaxN + ((uint32_t)((warp & 3) * 32) << 16);
@@ -696,5 +794,6 @@ __device__ __forceinline__ void acc_release(uint64_t* acc_empty) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(acc_empty);
 }
+
 
 }  // namespace et

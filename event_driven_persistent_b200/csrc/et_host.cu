@@ -561,12 +561,13 @@ et_status build_decode(et_graph* g) {
     if (d.n_heads <= 0) d.n_heads = 32;
     if (d.n_kv_heads <= 0) d.n_kv_heads = 8;
     if (d.head_dim <= 0) d.head_dim = 128;
-    if (d.max_ctx <= 0) d.max_ctx = 4097;
+    if (d.max_ctx <= 0) d.max_ctx = 4104;
     if (d.rope_base <= 0.f) d.rope_base = 500000.f;
     if (d.rms_eps <= 0.f) d.rms_eps = 1e-5f;
     if (d.fetch_batch <= 0) d.fetch_batch = 1;
     if (d.max_T > kMaxN) return ET_ERR_UNSUPPORTED;  // one token tile
     if (d.head_dim != 128 || d.n_heads % d.n_kv_heads || d.n_heads / d.n_kv_heads > 4) return ET_ERR_UNSUPPORTED;
+    if (d.max_ctx % 8) return ET_ERR_INVALID;  // V^T cache rows are read by TMA: 16-byte multiples
     if (d.hidden % 1024 || d.hidden > 4096 || d.inter % 128) return ET_ERR_UNSUPPORTED;
     DecodeParams& p = g->dec;
     memset(&p, 0, sizeof(p));
@@ -636,6 +637,7 @@ et_status build_decode(et_graph* g) {
     if (!make_map(&p.tm_attn, p.attn, rows, (uint64_t)p.nq * p.hd, 16)) return ET_ERR_CUDA;
     if (!make_map(&p.tm_xn2, p.xn2, rows, p.hidden, 16)) return ET_ERR_CUDA;
     if (!make_map(&p.tm_hm, p.hm, rows, p.inter, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_q, p.q, (uint64_t)p.maxB * p.nq, p.hd, 16)) return ET_ERR_CUDA;
     int mb = 0;
     ET_CU(decode_setup(&mb));
     if (mb < 1) return ET_ERR_UNSUPPORTED;
@@ -913,6 +915,9 @@ et_status et_run_decode(et_graph* g, int B, const uint16_t* X, const int32_t* po
     if (!g->mc[1].get(&p.tm_wo, w->Wo, p.hidden, (uint64_t)p.nq * p.hd, 64)) return ET_ERR_CUDA;
     if (!g->mc[2].get(&p.tm_wgu, w->Wgu, 2ull * p.inter, p.hidden, 64)) return ET_ERR_CUDA;
     if (!g->mc[3].get(&p.tm_wd, w->Wd, p.hidden, p.inter, 64)) return ET_ERR_CUDA;
+    const uint64_t cache_rows = (uint64_t)B * p.nkv;
+    if (!g->mc[4].get(&p.tm_kc, Kc, cache_rows * p.max_ctx, p.hd, 128)) return ET_ERR_CUDA;
+    if (!g->mc[5].get(&p.tm_vt, Vc, cache_rows * p.hd, p.max_ctx, 128)) return ET_ERR_CUDA;
     p.X = X;
     p.pos = pos;
     p.g1 = w->g1;

@@ -53,4 +53,36 @@ __device__ __forceinline__ int exec_scan(int v, int tid, int* tmp, int* total) {
     return base + inc - v;
 }
 
+// SwiGLU epilogue of a 128-row gate/up tile (rows 0..63 gate, 64..127 up,
+// of 64 consecutive output columns) for accumulator columns (tokens)
+// [c0, c0 + 16): h[t][col] = bf16(silu(gate) * up) for the first `nt`
+// of those tokens, stored at out + t * ld + col.  Gate and up go through
+// smem ([64][17] each, at the exec scratch); then thread (token, 8-column
+// group) stores 16 bytes.  Releases the accumulator after the last chunk
+// (c0 + 16 >= n).  `out` points at the chunk's first token row.  All 128
+// exec threads call.
+__device__ __forceinline__ void swiglu_tokens16(Ctx& x, uint32_t taddr, int c0, int n, uint64_t* acc_empty,
+                                                uint16_t* out, int ld, int nt) {
+    const int w = x.tid >> 5, lane = x.tid & 31;
+    const int r = ((w + kExecWarp0) & 3) * 32 + lane;
+    float v[16];
+    acc_load16(taddr, c0, v);
+    if (c0 + 16 >= n) acc_release(acc_empty);
+    float* st = x.epi + (r >> 6) * (64 * 17) + (r & 63) * 17;  // gate rows, then up rows
+#pragma unroll
+    for (int i = 0; i < 16; ++i) st[i] = v[i];
+    exec_bar();
+    const int t = x.tid >> 3, cg = (x.tid & 7) * 8;
+    if (t < nt) {
+        const float* sg = x.epi + cg * 17 + t;
+        const float* su = sg + 64 * 17;
+        uint4 o;
+        uint16_t* oo = reinterpret_cast<uint16_t*>(&o);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) oo[e] = bf16_bits(silu(sg[e * 17]) * su[e * 17]);
+        *reinterpret_cast<uint4*>(out + (size_t)t * ld + cg) = o;
+    }
+    exec_bar();
+}
+
 }  // namespace et

@@ -116,11 +116,14 @@ enum { DEC_MAP_WQKV = 0, DEC_MAP_WO = 1, DEC_MAP_WGU = 2, DEC_MAP_WD = 3,
 struct DecodeParams {
     CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wd;   // weights, box 64 x 64
     CUtensorMap tm_xn, tm_attn, tm_xn2, tm_hm;   // workspace activations, box 64 x 16
+    CUtensorMap tm_kc;   // K cache as [B nkv max_ctx, hd], box 64 x 128 (this run's Kc)
+    CUtensorMap tm_vt;   // V^T cache as [B nkv hd, max_ctx], box 64 x 128 (this run's Vc)
+    CUtensorMap tm_q;    // q as [maxB nq, hd], box 64 x 16
     // inputs / outputs
     const uint16_t* X;
     const int32_t* pos;        // [B] tokens already cached per request (= the new token's position)
     const uint16_t *g1, *gq, *gk, *g2;
-    uint16_t *Kc, *Vc;         // [maxB, nkv, max_ctx, hd] caches (appended in place)
+    uint16_t *Kc, *Vc;         // K cache [B, nkv, max_ctx, hd], V^T cache [B, nkv, hd, max_ctx] (appended in place)
     uint16_t* Y;
     uint16_t* out_h1;          // optional [B, H] attention-block output (residual stream)
     uint16_t* out_q;           // optional [B, nq*hd] rotated queries

@@ -29,6 +29,10 @@ constexpr int kBStageBytes = 128 * 128;  // up to 128 rows x 128 B
 constexpr int kMaxN = 128;         // largest MMA N (token rows per tile)
 constexpr int kTmemCols = 256;     // two accumulators of kMaxN fp32 columns
 constexpr int kScratchBytes = 16384;     // epilogue staging and CUDA-core task scratch
+// Attention stream stages: K tile (128 keys x 128 dims), V^T tile (128 dims
+// x 128 keys), Q tile (16 rows x 128 dims), each in the 128-byte swizzled
+// K-major layout of a tensor-core operand.
+constexpr uint32_t kAttnVOff = 32768, kAttnQOff = 65536, kAttnStage = 65536 + 4096;
 constexpr int kEpiBytes = 64 * 33 * 4;   // gate/up exchange staging (start of the scratch)
 constexpr int kCtlBytes = 2048;          // mbarriers, task ring, broadcast words
 constexpr int kSmemBytes = 1024 /*align slack*/ + kArenaBytes + kScratchBytes + kCtlBytes;

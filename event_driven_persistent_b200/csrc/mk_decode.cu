@@ -21,8 +21,9 @@
 //                  K head:  bf16 -> per-head rmsnorm gk -> RoPE -> cache[b, g, pos_b]
 //                  V head:  bf16 -> cache[b, g, pos_b]                 -> E_g[g] [grp + 2]
 //   ATTN(b, g, s) keys [S s, S s + S) of request b (S = the split, 512 keys), KV head g, all grp
-//                query heads: streamed through the stage arena (K and V
-//                blocks of 128 keys), online softmax; partial (o, m, l)  -> E_att[b, g] [#splits(b)]
+//                query heads, in stages of 128 keys on the tensor cores:
+//                S = K Q^T (keys x heads), online softmax on the exec group,
+//                O += V^T P^T (head dims x heads); partial (o, m, l)     -> E_att[b, g] [#splits(b)]
 //                the split completing (b, g) merges the partials inline  -> E_ag[g] [B]
 //   OPROJ(m, c)  output tile m, K chunk = the heads of KV group c, sums
 //                added at L2                                           -> E_o [n_m * nkv]
@@ -35,18 +36,7 @@
 
 namespace et {
 
-namespace {
-// contiguous global -> shared copy completing on an mbarrier (no multicast)
-__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
-}
-constexpr int kKeysPerStage = 128;
-constexpr uint32_t kAttnStageBytes = 2u * kKeysPerStage * 256u;  // K block then V block (head dim 128)
-}  // namespace
+constexpr int kKeysPerStage = 128;  // keys of one attention stage (the M of S = K Q^T)
 
 struct Decode : WorkloadBase {
     using Params = DecodeParams;
@@ -88,7 +78,8 @@ struct Decode : WorkloadBase {
             const int key0 = s * p.split, nkeys = min(p.split, pos + 1 - key0);
             d.valid = 1;
             d.stream = 1;
-            d.sbytes = kAttnStageBytes;
+            d.attn = 1;
+            d.sbytes = kAttnStage;
             d.nk = (nkeys + kKeysPerStage - 1) / kKeysPerStage;
             d.p[0] = bb;
             d.p[1] = g;
@@ -168,44 +159,48 @@ struct Decode : WorkloadBase {
         return (pos - key0) / kKeysPerStage;   // stages before the one holding key `pos`
     }
     __device__ static int stage_keys(const TaskDesc& d, int st) { return min(kKeysPerStage, d.p[5] - st * kKeysPerStage); }
-    __device__ static uint32_t stream_bytes(const Params&, const TaskDesc& d, int st) {
-        return 2u * (uint32_t)stage_keys(d, st) * 256u;
-    }
+    // A stage: K rows [key, key + 128) of (b, g) (cache rows beyond the
+    // request's keys are masked), the V^T columns of the same keys (columns
+    // beyond them are zeroed in smem before use), and the grp query rows of
+    // (b, g) (16-row box: rows past grp only feed unused S columns).  Full
+    // boxes always land (out-of-range rows and columns are filled with 0).
+    __device__ static uint32_t stream_bytes(const Params&, const TaskDesc&, int) { return kAttnStage; }
     __device__ static void stream_copy(const Params& p, const TaskDesc& d, int st, uint8_t* dst, uint64_t* bar,
+                                       uint64_t pol, bool late) {
+        const int bb = d.p[0], g = d.p[1], key = d.p[4] + st * kKeysPerStage;
+        const int krow = (bb * p.nkv + g) * p.max_ctx + key, vrow = (bb * p.nkv + g) * p.hd;
+#pragma unroll
+        for (int at = 0; at < 2; ++at) {
+            tma_load_2d(dst + at * kAAtomBytes, &p.tm_kc, bar, at * kAtomK, krow, pol);
+            tma_load_2d(dst + kAttnVOff + at * kAAtomBytes, &p.tm_vt, bar, key + at * kAtomK, vrow, pol);
+        }
+        if (late) stream_late(p, d, st, dst, bar, pol);
+    }
+    __device__ static void stream_late(const Params& p, const TaskDesc& d, int, uint8_t* dst, uint64_t* bar,
                                        uint64_t pol) {
-        const int bb = d.p[0], g = d.p[1];
-        const size_t row = ((size_t)(bb * p.nkv + g) * p.max_ctx + d.p[4] + st * kKeysPerStage) * p.hd;
-        const uint32_t bytes = (uint32_t)stage_keys(d, st) * 256u;
-        bulk_copy(dst, p.Kc + row, bytes, bar, pol);
-        bulk_copy(dst + kKeysPerStage * 256, p.Vc + row, bytes, bar, pol);
+        const int qrow = d.p[0] * p.nq + d.p[1] * p.grp;
+#pragma unroll
+        for (int at = 0; at < 2; ++at) tma_load_2d(dst + kAttnQOff + at * 16 * 128, &p.tm_q, bar, at * kAtomK, qrow, pol);
     }
 
-    // One attention split: grp query heads against the split's keys, online
-    // softmax across its stages.  Scores: 8 threads per key, thread j of a
-    // key holding dims [8j, 8j+8) and [64+8j, 64+8j+8) of every query head
-    // (16 x grp floats in registers) -- a warp reads four whole 256-byte key
-    // rows per instruction.  Values: thread t owns dim t of every head.
+    // One attention split (exec group; the MMA warp runs the products).
+    // Per stage of 128 keys: thread r (its warp's TMEM lane) reads the scores
+    // of key r for every query head from S, the group takes the stage max and
+    // the online-softmax rescale, writes P = bf16(exp(s - max)) (query heads x
+    // keys, the 128-byte swizzled K-major layout of a tensor-core B operand)
+    // and, on a partial stage, zeroes the V^T columns of the missing keys;
+    // then thread r reads head dim r of every head from O = V^T P^T.  The
+    // normaliser sums the bf16 probabilities the product used.
     __device__ static bool stream_exec(const Params& p, Ctx& x, TaskDesc& d) {
         const int bb = d.p[0], g = d.p[1], s = d.p[2];
-        const int tid = x.tid, j8 = tid & 7, kg = tid >> 3, w = tid >> 5, lane = tid & 31;
+        const int w = x.tid >> 5, lane = x.tid & 31;
+        const int r = ((w + kExecWarp0) & 3) * 32 + lane;
         const int grp = p.grp;
-        float qv[4][16];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            if (h < grp) {
-                const uint16_t* qr = p.q + ((size_t)bb * p.nq + g * grp + h) * p.hd;
-                // (written during the run by another SM's branch: read through L2)
-                bf16x8(__ldcg(reinterpret_cast<const uint4*>(qr + 8 * j8)), qv[h]);
-                bf16x8(__ldcg(reinterpret_cast<const uint4*>(qr + 64 + 8 * j8)), qv[h] + 8);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) qv[h][i] = 0.f;
-            }
-        }
-        float* sc = x.epi;                                     // [4][128] scaled scores
-        float4* pk = reinterpret_cast<float4*>(x.epi + 512);  // [128] probabilities, one float4 per key
-        float* red = x.epi + 1024;                             // [4 warps][4 heads] x 2
-        const float scale = 0.08838834764831845f;              // 1 / sqrt(128)
+        uint8_t* P = reinterpret_cast<uint8_t*>(x.epi);  // [2 key atoms][16 rows][128 B]
+        float* red = x.epi + 1024;                          // [max: 4 warps x 4 heads][sum: same]
+        for (int i = x.tid; i < 1024; i += kExecThreads)   // query-head rows grp..15 of P stay 0
+            if (((i >> 5) & 15) >= grp) reinterpret_cast<uint32_t*>(P)[i] = 0u;
+        const float scale = 0.08838834764831845f;  // 1 / sqrt(128)
         float m[4], l[4], o[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
@@ -215,46 +210,19 @@ struct Decode : WorkloadBase {
         }
         StageAlloc al = stream_alloc(d);
         for (int st = 0; st < d.nk; ++st) {
-            uint32_t off;
-            if (!stream_stage_wait(x, d, st, al, &off)) return false;
-            const uint8_t* Ks = x.arena + off;
-            const uint8_t* Vs = Ks + kKeysPerStage * 256;
+            const uint32_t off = al.next(d.sbytes);
             const int nks = stage_keys(d, st);
-#pragma unroll 2
-            for (int pass = 0; pass < kKeysPerStage / 16; ++pass) {
-                const int key = pass * 16 + kg;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                if (key < nks) {
-                    float kv[16];
-                    bf16x8(*reinterpret_cast<const uint4*>(Ks + key * 256 + j8 * 16), kv);
-                    bf16x8(*reinterpret_cast<const uint4*>(Ks + key * 256 + 128 + j8 * 16), kv + 8);
-                    float acc2[4] = {0.f, 0.f, 0.f, 0.f};  // two chains per head (latency, not work)
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            acc[h] = fmaf(qv[h][i], kv[i], acc[h]);
-                            acc2[h] = fmaf(qv[h][8 + i], kv[8 + i], acc2[h]);
-                        }
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) acc[h] += acc2[h];
-                }
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 1);
-                    acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 2);
-                    acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 4);
-                }
-                if (j8 == 0 && key < nks)
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) sc[h * 128 + key] = acc[h] * scale;
-            }
-            exec_bar();
-            // stage maximum per head, then probabilities and their sums
+            if (!exec_mbar_wait(x, &x.sc->s_full, x.na & 1, 316, 2)) return false;
+            tc_fence_after();
+            float sv[4];
+            __syncwarp();
+            tmem_ld4_wait(x.taddr, sv);
+            const bool valid = r < nks;
             float mx[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                mx[h] = tid < nks ? sc[h * 128 + tid] : -INFINITY;
+                sv[h] = (valid && h < grp) ? sv[h] * scale : -INFINITY;
+                mx[h] = sv[h];
 #pragma unroll
                 for (int o2 = 16; o2 > 0; o2 >>= 1) mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], o2));
             }
@@ -262,57 +230,60 @@ struct Decode : WorkloadBase {
 #pragma unroll
                 for (int h = 0; h < 4; ++h) red[w * 4 + h] = mx[h];
             exec_bar();
-            float alpha[4], pr[4], ps[4];
+            float alpha[4], ps[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                const float mn = fmaxf(m[h], fmaxf(fmaxf(red[h], red[4 + h]), fmaxf(red[8 + h], red[12 + h])));
-                alpha[h] = expf(m[h] - mn);
-                m[h] = mn;
-                pr[h] = tid < nks ? expf(sc[h * 128 + tid] - mn) : 0.f;
-                ps[h] = pr[h];
+                float pv = 0.f;
+                alpha[h] = 1.f;
+                if (h < grp) {
+                    const float mn = fmaxf(m[h], fmaxf(fmaxf(red[h], red[4 + h]), fmaxf(red[8 + h], red[12 + h])));
+                    alpha[h] = expf(m[h] - mn);  // 0 on the first stage (m = -inf)
+                    m[h] = mn;
+                    if (valid) {
+                        const uint16_t pb = bf16_bits(expf(sv[h] - mn));
+                        pv = bf16_val(pb);
+                        *reinterpret_cast<uint16_t*>(P + (r >> 6) * 2048 + h * 128 +
+                                                     ((((r & 63) >> 3) ^ (h & 7)) << 4) + (r & 7) * 2) = pb;
+                    } else {
+                        *reinterpret_cast<uint16_t*>(P + (r >> 6) * 2048 + h * 128 +
+                                                     ((((r & 63) >> 3) ^ (h & 7)) << 4) + (r & 7) * 2) = 0;
+                    }
+                }
+                ps[h] = pv;
 #pragma unroll
                 for (int o2 = 16; o2 > 0; o2 >>= 1) ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], o2);
             }
-            pk[tid] = make_float4(pr[0], pr[1], pr[2], pr[3]);
+            if (nks < kKeysPerStage) {
+                // V^T row r (head dim r): the columns of keys nks..127 to 0,
+                // after the stage's copies landed (that phase is already
+                // complete: the MMA warp waited on it before S)
+                const uint32_t gs = d.st0 + (uint32_t)st;
+                if (!exec_mbar_wait(x, &x.sc->full[gs % kSlots], (gs / kSlots) & 1, 318, 5)) return false;
+                uint8_t* vr = x.arena + off + kAttnVOff + r * 128;
+                for (int k = nks; k < kKeysPerStage; ++k)
+                    *reinterpret_cast<uint16_t*>(vr + (k >> 6) * kAAtomBytes + ((((k & 63) >> 3) ^ (r & 7)) << 4) +
+                                                 (k & 7) * 2) = 0;
+            }
             if (lane == 0)
 #pragma unroll
                 for (int h = 0; h < 4; ++h) red[16 + w * 4 + h] = ps[h];
+            fence_proxy_async_smem();  // P and the zeroed V^T columns are read by the tensor core
+            tc_fence_before();
             exec_bar();
+            if (x.tid == 0) mbar_arrive(&x.sc->p_full);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                l[h] = l[h] * alpha[h] + red[16 + h] + red[20 + h] + red[24 + h] + red[28 + h];
-                o[h] *= alpha[h];
-            }
-            // two chains per head over even and odd keys (nks is even unless it is the
-            // split's last stage; the odd tail key goes to the first chain)
-            const uint16_t* vcol = reinterpret_cast<const uint16_t*>(Vs) + tid;
-            float o2[4] = {0.f, 0.f, 0.f, 0.f};
-            int key = 0;
-#pragma unroll 2
-            for (; key + 1 < nks; key += 2) {
-                const float4 pa = pk[key], pb = pk[key + 1];
-                const float va = bf16_val(vcol[key * 128]), vb = bf16_val(vcol[(key + 1) * 128]);
-                o[0] = fmaf(pa.x, va, o[0]);
-                o[1] = fmaf(pa.y, va, o[1]);
-                o[2] = fmaf(pa.z, va, o[2]);
-                o[3] = fmaf(pa.w, va, o[3]);
-                o2[0] = fmaf(pb.x, vb, o2[0]);
-                o2[1] = fmaf(pb.y, vb, o2[1]);
-                o2[2] = fmaf(pb.z, vb, o2[2]);
-                o2[3] = fmaf(pb.w, vb, o2[3]);
-            }
-            if (key < nks) {
-                const float4 pa = pk[key];
-                const float va = bf16_val(vcol[key * 128]);
-                o[0] = fmaf(pa.x, va, o[0]);
-                o[1] = fmaf(pa.y, va, o[1]);
-                o[2] = fmaf(pa.z, va, o[2]);
-                o[3] = fmaf(pa.w, va, o[3]);
-            }
+            for (int h = 0; h < 4; ++h) l[h] = l[h] * alpha[h] + red[16 + h] + red[20 + h] + red[24 + h] + red[28 + h];
+            if (!exec_mbar_wait(x, &x.sc->o_full, x.na & 1, 317, 3)) return false;
+            tc_fence_after();
+            float ov[4];
+            __syncwarp();
+            tmem_ld4_wait(x.taddr + 16, ov);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) o[h] += o2[h];
-            stream_stage_release(x, d, st);
+            for (int h = 0; h < 4; ++h) o[h] = o[h] * alpha[h] + ov[h];
+            ++x.na;
         }
+        acc_release(x.acc_empty);
+        const int tid = r;  // head dim of this thread
         // partial of this split: o (unnormalised), running max m, sum l
         const int stride = p.hd + 2;
         float* pp = p.part + ((size_t)(bb * p.nkv + g) * p.s_max + s) * grp * stride;
@@ -417,8 +388,8 @@ struct Decode : WorkloadBase {
                     const int b = b0 + j;
                     if (b < p.B) {
                         const int pos = __ldg(p.pos + b);
-                        if (pos >= 0 && pos < p.max_ctx)
-                            p.Vc[(((size_t)b * p.nkv + g) * p.max_ctx + pos) * p.hd + t] = bf16_bits(y[j]);
+                        if (pos >= 0 && pos < p.max_ctx)  // V^T cache: [b][g][dim][position]
+                            p.Vc[(((size_t)b * p.nkv + g) * p.hd + t) * p.max_ctx + pos] = bf16_bits(y[j]);
                     }
                 }
                 continue;
@@ -460,7 +431,7 @@ struct Decode : WorkloadBase {
             }
             exec_bar();  // sy / red are reused by the next 8 tokens
         }
-        fence_proxy_async_global();  // the cache is read by bulk copies in the attention tasks
+        fence_proxy_async_global();  // the caches and q are read by TMA in the attention tasks
         int* ev = x.ctr + (unfused(p) ? p.ev_branch_all : p.ev_g + g);
         const int tgt = unfused(p) ? p.n_heads : p.grp + 2;
         if (group_finish_notify(x, d, ev, 1, tgt) && push_attn(p) && !unfused(p)) push_splits(p, x, g);
@@ -537,33 +508,9 @@ struct Decode : WorkloadBase {
             return true;
         }
         // GU: rows 0..63 gate, 64..127 up, of intermediate columns a*64 + (r & 63)
-        const bool is_up = q >= 2;
-        const int j = r & 63;
-        float* stage = x.epi;  // [64][33]
-        for (int c0 = 0; c0 < d.n; c0 += 32) {
-            float va[16], vb[16];
-            acc_load16(taddr, c0, va);
-            if (c0 + 16 < d.n) acc_load16(taddr, c0 + 16, vb);
-            if (c0 + 32 >= d.n) acc_release(acc_empty);
-            if (is_up) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    stage[j * 33 + i] = va[i];
-                    stage[j * 33 + 16 + i] = vb[i];
-                }
-            }
-            exec_bar();
-            if (!is_up) {
-                const int col = a * p.gu_tile + j;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int b = c0 + i;
-                    const float gv = i < 16 ? va[i] : vb[i - 16];
-                    if (b < p.B) p.hm[(size_t)b * p.inter + col] = bf16_bits(silu(gv) * stage[j * 33 + i]);
-                }
-            }
-            exec_bar();
-        }
+        for (int c0 = 0; c0 < d.n; c0 += 16)
+            swiglu_tokens16(x, taddr, c0, d.n, acc_empty, p.hm + (size_t)c0 * p.inter + a * p.gu_tile, p.inter,
+                            p.B - c0);
         fence_proxy_async_global();  // hm is read by TMA in the down tasks
         const int cc = (a * p.gu_tile) / p.kchunk;
         int* ev = x.ctr + (unfused(p) ? p.ev_gu_all : p.ev_h + cc);
@@ -668,12 +615,36 @@ struct Decode : WorkloadBase {
         int* ev = x.ctr + (unfused(p) ? p.ev_down_all : p.ev_y + m);
         const int tgt = unfused(p) ? p.n_m * p.n_c : p.n_c;
         if (!group_wait(x, d, ev, tgt, 315)) return false;
-        const int col = m * 128 + x.tid;
-        for (int b = 0; b < p.B; ++b) {
-            const size_t i = (size_t)b * p.hidden + col;
-            const float a = __ldcg(p.yacc + i);
-            __stcg(p.yacc + i, 0.f);
-            p.Y[i] = bf16_bits(bf16_val(__ldcg(p.h1 + i)) + a);
+        // B tokens x 128 columns as float4: eight loads in flight per thread
+        // before its stores
+        const int nv = 128 / 4, total = p.B * nv;
+        for (int base = x.tid; base < total; base += kExecThreads * 8) {
+            float4 v[8];
+            uint2 hv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * kExecThreads;
+                if (i < total) {
+                    const size_t off = (size_t)(i / nv) * p.hidden + m * 128 + (i % nv) * 4;
+                    v[u] = __ldcg(reinterpret_cast<const float4*>(p.yacc + off));
+                    hv[u] = __ldcg(reinterpret_cast<const uint2*>(p.h1 + off));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = base + u * kExecThreads;
+                if (i < total) {
+                    const size_t off = (size_t)(i / nv) * p.hidden + m * 128 + (i % nv) * 4;
+                    __stcg(reinterpret_cast<float4*>(p.yacc + off), make_float4(0.f, 0.f, 0.f, 0.f));
+                    const uint16_t* h = reinterpret_cast<const uint16_t*>(&hv[u]);
+                    ushort4 o;
+                    o.x = bf16_bits(bf16_val(h[0]) + v[u].x);
+                    o.y = bf16_bits(bf16_val(h[1]) + v[u].y);
+                    o.z = bf16_bits(bf16_val(h[2]) + v[u].z);
+                    o.w = bf16_bits(bf16_val(h[3]) + v[u].w);
+                    *reinterpret_cast<ushort4*>(p.Y + off) = o;
+                }
+            }
         }
         group_finish_notify(x, d, nullptr, 0, 0);
         return true;

@@ -82,33 +82,9 @@ struct Mlp : WorkloadBase {
         const int r = q * 32 + lane;          // accumulator row (lane) held by this thread
         if (op == ET_OP_MLP_GATEUP) {
             // rows 0..63 = gate, 64..127 = up, of intermediate columns a*64 + (r & 63)
-            const bool is_up = q >= 2;
-            const int j = r & 63;
-            float* stage = x.epi;  // [64][33]
-            for (int c0 = 0; c0 < d.n; c0 += 32) {
-                float va[16], vb[16];
-                acc_load16(taddr, c0, va);
-                if (c0 + 16 < d.n) acc_load16(taddr, c0 + 16, vb);
-                if (c0 + 32 >= d.n) acc_release(acc_empty);
-                if (is_up) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        stage[j * 33 + i] = va[i];
-                        stage[j * 33 + 16 + i] = vb[i];
-                    }
-                }
-                exec_bar();
-                if (!is_up) {
-                    const int col = a * p.gu_tile + j;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int b = c0 + i;
-                        const float g = i < 16 ? va[i] : vb[i - 16];
-                        if (b < p.B) p.h[(size_t)b * p.inter + col] = bf16_bits(silu(g) * stage[j * 33 + i]);
-                    }
-                }
-                exec_bar();
-            }
+            for (int c0 = 0; c0 < d.n; c0 += 16)
+                swiglu_tokens16(x, taddr, c0, d.n, acc_empty, p.h + (size_t)c0 * p.inter + a * p.gu_tile, p.inter,
+                                p.B - c0);
             fence_proxy_async_global();  // h is read by TMA in the down tasks
             int* ev = x.ctr + (p.unfused ? p.ev_gu_all : p.ev_h + (a * p.gu_tile) / p.kchunk);
             const int tgt = p.unfused ? p.n_gu : p.gu_per_chunk;
@@ -183,12 +159,31 @@ struct Mlp : WorkloadBase {
             const int* ev = x.ctr + (p.unfused ? p.ev_down_all : p.ev_y + a);
             const int tgt = p.unfused ? p.n_m * p.n_c : p.n_c;
             if (!group_wait(x, d, ev, tgt, 104)) return false;
-            for (int j = x.tid; j < p.down_tile; j += kExecThreads) {
-                const int col = a * p.down_tile + j;
-                for (int b = 0; b < p.B; ++b) {
-                    const size_t i = (size_t)b * p.hidden + col;
-                    p.Y[i] = bf16_bits(__ldcg(p.yacc + i));
-                    __stcg(p.yacc + i, 0.f);
+            // B tokens x down_tile columns as float4: eight loads in flight
+            // per thread before its stores
+            const int nv = p.down_tile / 4, total = p.B * nv;
+            for (int base = x.tid; base < total; base += kExecThreads * 8) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = base + u * kExecThreads;
+                    if (i < total)
+                        v[u] = __ldcg(reinterpret_cast<const float4*>(p.yacc + (size_t)(i / nv) * p.hidden +
+                                                                      a * p.down_tile) + i % nv);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = base + u * kExecThreads;
+                    if (i < total) {
+                        const size_t off = (size_t)(i / nv) * p.hidden + a * p.down_tile + (i % nv) * 4;
+                        __stcg(reinterpret_cast<float4*>(p.yacc + off), make_float4(0.f, 0.f, 0.f, 0.f));
+                        ushort4 o;
+                        o.x = bf16_bits(v[u].x);
+                        o.y = bf16_bits(v[u].y);
+                        o.z = bf16_bits(v[u].z);
+                        o.w = bf16_bits(v[u].w);
+                        *reinterpret_cast<ushort4*>(p.Y + off) = o;
+                    }
                 }
             }
             group_finish_notify(x, d, nullptr, 0, 0);

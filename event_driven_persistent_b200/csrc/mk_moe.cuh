@@ -192,33 +192,9 @@ struct Moe : WorkloadBase {
             return route_topk(p, x, d, a, L);
         } else if (op == ET_OP_MOE_S1) {
             const int row0 = d.p[1], cnt = d.p[2];
-            const bool is_up = q >= 2;
-            const int j = r & 63;
-            float* stage = x.epi;  // [64][33]
-            for (int c0 = 0; c0 < d.n; c0 += 32) {
-                float va[16], vb[16];
-                acc_load16(taddr, c0, va);
-                if (c0 + 16 < d.n) acc_load16(taddr, c0 + 16, vb);
-                if (c0 + 32 >= d.n) acc_release(acc_empty);
-                if (is_up) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        stage[j * 33 + i] = va[i];
-                        stage[j * 33 + 16 + i] = vb[i];
-                    }
-                }
-                exec_bar();
-                if (!is_up) {
-                    const int col = b * p.n1_tile + j;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int c = c0 + i;
-                        const float g = i < 16 ? va[i] : vb[i - 16];
-                        if (c < cnt) p.Hm[(size_t)(row0 + c) * p.inter + col] = bf16_bits(silu(g) * stage[j * 33 + i]);
-                    }
-                }
-                exec_bar();
-            }
+            for (int c0 = 0; c0 < d.n; c0 += 16)
+                swiglu_tokens16(x, taddr, c0, d.n, acc_empty, p.Hm + (size_t)(row0 + c0) * p.inter + b * p.n1_tile,
+                                p.inter, cnt - c0);
             fence_proxy_async_global();  // Hm is read by TMA in stage 2
             int* ev = x.ctr + (is_unfused(p) ? p.ev_s1_all : p.ev_s1 + a);
             const int tgt = is_unfused(p) ? ld_volatile(p.scal) * p.n_n1 : p.n_n1;
@@ -320,11 +296,6 @@ struct Moe : WorkloadBase {
         }
         // eight float4 loads in flight per thread, then zero + convert + store
         const int nv = p.hidden / 4, total = ntok * nv;
-        float* ss = reinterpret_cast<float*>(x.simt) + 512;  // [cb] sums of squares (fused MLP)
-        if (p.mlp_xn) {
-            if (x.tid < p.cb) ss[x.tid] = 0.f;
-            exec_bar();
-        }
         for (int base = x.tid; base < total; base += kExecThreads * 8) {
             float4 v[8];
 #pragma unroll
@@ -344,30 +315,43 @@ struct Moe : WorkloadBase {
                     o.z = bf16_bits(v[u].z);
                     o.w = bf16_bits(v[u].w);
                     *reinterpret_cast<ushort4*>(p.Y + off) = o;
-                    if (p.mlp_xn) {
-                        const float a = bf16_val(o.x), b = bf16_val(o.y), c = bf16_val(o.z), e = bf16_val(o.w);
-                        atomicAdd(ss + i / nv, a * a + b * b + c * c + e * e);
-                    }
                 }
             }
         }
-        if (p.mlp_xn) return mlp_norm(p, x, d, t0, ntok, ss);
+        if (p.mlp_xn) return mlp_norm(p, x, d, t0, ntok);
         group_finish_notify(x, d, nullptr, 0, 0);
         return true;
     }
 
     // Fused dense MLP after the layer: the MLP's RMSNorm of the block's tokens
     // from the bf16 outputs just written (same CTA), then E_norm of the MLP.
-    __device__ static bool mlp_norm(const Params& p, Ctx& x, TaskDesc& d, int t0, int ntok, const float* ss) {
-        exec_bar();  // Y rows and their sums of squares complete
+    __device__ static bool mlp_norm(const Params& p, Ctx& x, TaskDesc& d, int t0, int ntok) {
+        exec_bar();  // the block's Y rows are written
+        // sums of squares of the bf16 outputs: per token, each warp's part
+        // reduced by shuffles into ssw[warp][token], then summed
         const int n8 = p.hidden / 8, total = ntok * n8;
+        float* ssw = reinterpret_cast<float*>(x.simt) + 512;  // [4 warps][cb]
+        for (int t = 0; t < ntok; ++t) {
+            float sq = 0.f;
+            for (int c = x.tid; c < n8; c += kExecThreads) {
+                float y[8];
+                bf16x8(*reinterpret_cast<const uint4*>(p.Y + (size_t)(t0 + t) * p.hidden + c * 8), y);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sq = fmaf(y[j], y[j], sq);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if ((x.tid & 31) == 0) ssw[(x.tid >> 5) * p.cb + t] = sq;
+        }
+        exec_bar();
         for (int i = x.tid; i < total; i += kExecThreads) {
             const int t = i / n8, c = (i % n8) * 8;
             const size_t off = (size_t)(t0 + t) * p.hidden + c;
             float y[8], gm[8];
             bf16x8(*reinterpret_cast<const uint4*>(p.Y + off), y);
             bf16x8(__ldg(reinterpret_cast<const uint4*>(p.mlp_gamma + c)), gm);
-            const float inv = 1.0f / sqrtf(ss[t] / (float)p.hidden + p.mlp_eps);
+            const float sst = ssw[t] + ssw[p.cb + t] + ssw[2 * p.cb + t] + ssw[3 * p.cb + t];
+            const float inv = 1.0f / sqrtf(sst / (float)p.hidden + p.mlp_eps);
             uint4 o;
             uint16_t* oo = reinterpret_cast<uint16_t*>(&o);
 #pragma unroll

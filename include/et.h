@@ -114,8 +114,8 @@ typedef struct {
     int n_heads;         /* query heads [32] */
     int n_kv_heads;      /* key/value heads [8]; n_heads / n_kv_heads <= 4 */
     int head_dim;        /* [128]; only 128 is supported */
-    int max_ctx;         /* cache positions per request [4097]; a run's positions must be < max_ctx;
-                            at most 1024 * 256 / (n_heads / n_kv_heads) */
+    int max_ctx;         /* cache positions per request [4104]: a multiple of 8, at most
+                            1024 * dec_split / (n_heads / n_kv_heads); a run's positions must be < max_ctx */
     float rope_base;     /* rotary embedding base [500000] */
     /* MoE -> dense MLP (ET_GRAPH_MOE_MLP); the MoE dims above, the MLP's width = hidden */
     int mlp_inter;       /* dense MLP intermediate width [6144] */
@@ -319,15 +319,17 @@ typedef struct {
  * split tasks, a run-time count).  Per request b at position p = pos[b]:
  *   xn  = bf16(rmsnorm(x) g1);  qkv = bf16(xn Wqkv^T)
  *   q_h = bf16(rope(rmsnorm(q_h) gq, p)),  k_g = bf16(rope(rmsnorm(k_g) gk, p))
- *   Kc[b,g,p] = k_g, Vc[b,g,p] = v_g          (written in place)
- *   o_h = softmax over j <= p of (q_h . Kc[b,g,j] / sqrt(head_dim)) . Vc[b,g,j],
+ *   Kc[b,g,p,:] = k_g, Vc[b,g,:,p] = v_g      (written in place)
+ *   o_h = softmax over j <= p of (q_h . Kc[b,g,j,:] / sqrt(head_dim)) . Vc[b,g,:,j],
  *         g = h / (n_heads / n_kv_heads)
  *   h1  = bf16(x + bf16(o) Wo^T)
  *   Y   = bf16(h1 + (bf16(silu(xn2 Wg^T) * (xn2 Wu^T))) Wd^T),  xn2 = bf16(rmsnorm(h1) g2)
  * RoPE pairs element i with element i + head_dim/2 at angle p * base^(-2i/head_dim).
  * X bf16 [B, hidden]; pos int32 [B] (device), 0 <= pos[b] < max_ctx, else the
- * run ends with ET_ERR_INVALID from et_sync_status; Kc, Vc bf16 [max_T,
- * n_kv_heads, max_ctx, head_dim] (device, updated in place at pos[b]);
+ * run ends with ET_ERR_INVALID from et_sync_status; Kc bf16 [B, n_kv_heads,
+ * max_ctx, head_dim] and Vc bf16 [B, n_kv_heads, head_dim, max_ctx] (V stored
+ * transposed, positions contiguous: both attention products then read their
+ * operands K-major on the tensor cores) (device, updated in place at pos[b]);
  * Y bf16 [B, hidden]; h1 (optional, NULL to skip) bf16 [B, hidden].
  * 1 <= B <= max_T <= 128. */
 et_status et_run_decode(et_graph* g, int B, const uint16_t* X, const int32_t* pos, const et_decode_weights* w,

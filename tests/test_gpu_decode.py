@@ -35,11 +35,12 @@ def run_decode(g, d, B, wt=None, pos=None):
     wt = wt or {k: dev(d[k]) for k in WKEYS}
     pos = d["pos"][:B] if pos is None else np.asarray(pos, np.int32)
     H = d["X"].shape[1]
-    Kc, Vc = dev(d["Kc"][:B]), dev(d["Vc"][:B])
+    Kc, Vt = dev(d["Kc"][:B]), dev(W.v_cache_device(d["Vc"][:B]))
     Y, h1 = empty_bf16(B, H), empty_bf16(B, H)
-    et.et_run_decode(g, B, dev(d["X"][:B]), dev(pos), wt, Kc, Vc, Y, h1)
+    et.et_run_decode(g, B, dev(d["X"][:B]), dev(pos), wt, Kc, Vt, Y, h1)
     st = et.et_sync_status(g)
-    return st, dict(y=host(Y, np.uint16), h1=host(h1, np.uint16), Kc=host(Kc, np.uint16), Vc=host(Vc, np.uint16))
+    return st, dict(y=host(Y, np.uint16), h1=host(h1, np.uint16), Kc=host(Kc, np.uint16),
+                    Vc=W.v_cache_device(host(Vt, np.uint16)))
 
 
 def check(d, out, B, n_q, n_kv, pos=None, rows=None):

@@ -99,9 +99,11 @@ def moe_inputs(T, hidden=2048, inter=768, E=128, zipf_s=1.2, weights=True):
 def decode_inputs(B, hidden=4096, n_q=32, n_kv=8, hd=128, inter=14336, ctx_lo=512, ctx_hi=4096, max_ctx=None,
                   weights=True):
     """dict(X, pos, Kc, Vc[, g1, Wqkv, gq, gk, Wo, g2, Wgu, Wd]) for one decode
-    step of B requests; pos[b] = tokens already cached for request b."""
+    step of B requests; pos[b] = tokens already cached for request b.  Both
+    caches are [B, n_kv, max_ctx, hd] here; the device takes V transposed
+    (v_cache_device)."""
     if max_ctx is None:
-        max_ctx = ctx_hi + 1
+        max_ctx = (ctx_hi + 1 + 7) // 8 * 8  # the device reads cache rows as 16-byte multiples
     pos = np.random.default_rng(41).integers(ctx_lo, ctx_hi + 1, size=64 if B <= 64 else B)[:B].astype(np.int32)
     Kc = np.zeros((B, n_kv, max_ctx, hd), np.uint16)
     Vc = np.zeros((B, n_kv, max_ctx, hd), np.uint16)
@@ -128,3 +130,9 @@ def dense_mlp_weights(hidden=2048, inter=6144):
     return dict(gamma=_normal_bf16(np.random.default_rng(50), (hidden,), 1.0, 0.1),
                 Wgu=_normal_bf16(np.random.default_rng(51), (2 * inter, hidden), 0.0, 0.02),
                 Wd=_normal_bf16(np.random.default_rng(52), (hidden, inter), 0.0, 0.02))
+
+
+def v_cache_device(Vc):
+    """The device's V cache layout, [B, n_kv, hd, max_ctx] (keys contiguous),
+    from [B, n_kv, max_ctx, hd]; the same function maps it back."""
+    return np.ascontiguousarray(np.swapaxes(Vc, 2, 3))
