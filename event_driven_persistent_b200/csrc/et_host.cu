@@ -626,6 +626,7 @@ et_status build_decode(et_graph* g) {
     ET_TRY(galloc(g, &p.xn, rows * p.hidden));
     ET_TRY(galloc(g, &p.qkvacc, (size_t)p.maxB * p.n_heads * p.hd));
     ET_TRY(galloc(g, &p.q, (size_t)p.maxB * p.nq * p.hd));
+    ET_TRY(galloc(g, &p.rope, (size_t)p.maxB * (p.hd / 2)));
     ET_TRY(galloc(g, &p.part, (size_t)p.maxB * p.nkv * p.s_max * p.grp * (p.hd + 2)));
     ET_TRY(galloc(g, &p.attn, rows * p.nq * p.hd));
     ET_TRY(galloc(g, &p.h1acc, (size_t)p.maxB * p.hidden));

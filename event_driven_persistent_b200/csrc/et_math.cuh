@@ -18,6 +18,12 @@ __device__ __forceinline__ void bf16x8(uint4 u, float* f) {
         f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
 }
+// 4 bf16 (8 bytes) -> fp32
+__device__ __forceinline__ void bf16x4(uint2 u, float* f) {
+    const uint16_t* e = reinterpret_cast<const uint16_t*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = bf16_val(e[i]);
+}
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 // fp32 add at L2 (fire and forget)
 __device__ __forceinline__ void red_add(float* p, float v) {

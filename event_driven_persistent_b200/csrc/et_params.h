@@ -131,6 +131,7 @@ struct DecodeParams {
     uint16_t* xn;              // [maxB, H]
     float* qkvacc;             // [maxB, nqkv*hd] K-chunk sums (zero between runs)
     uint16_t* q;               // [maxB, nq, hd] rotated queries
+    float2* rope;              // [maxB, hd/2] (cos, sin) of each request's position, per frequency
     float* part;               // [maxB*nkv, S_max, grp, hd + 2] split partials (o, m, l)
     uint16_t* attn;            // [maxB, nq*hd] attention output (o-proj B operand)
     float* h1acc;              // [maxB, H] o-proj sums (zero between runs)

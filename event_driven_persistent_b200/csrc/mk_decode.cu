@@ -352,8 +352,10 @@ struct Decode : WorkloadBase {
 
     // ------------------------------------------------------------ branches
     // Q head n, K head (n - nq) or V head (n - nq - nkv), all B tokens, from
-    // the head's K-chunk sums; thread t = dim t.  Run by the QKV task that
-    // completed E_qkv[n].
+    // the head's K-chunk sums.  Run by the QKV task that completed E_qkv[n].
+    // Warp w takes tokens w, w + 4, ...; lane l holds dims 4l..4l+3, so the
+    // per-head RMSNorm is a warp reduction and the rotate-half partner of
+    // dim i (i + 64) sits in lane l ^ 16: no exec-group barrier.
     __device__ static bool branch(const Params& p, Ctx& x, const TaskDesc& d0, int n) {
         const int kind = n < p.nq ? 0 : (n < p.nq + p.nkv ? 1 : 2);
         const int g = kind == 0 ? n / p.grp : (kind == 1 ? n - p.nq : n - p.nq - p.nkv);
@@ -362,74 +364,50 @@ struct Decode : WorkloadBase {
         d.t_fetch = d.t_acc = 0;
         if (x.debug & ET_DEBUG_TRACE) d.t_fetch = globaltimer();
         if (!group_wait(x, d, nullptr, 0, 311)) return false;
-        const int t = x.tid, w = t >> 5, lane = t & 31;
-        const int stride = p.n_heads * p.hd;
-        float* acc = p.qkvacc + (size_t)n * p.hd + t;
-        float* sy = x.epi;              // [8][128] exchange for the rotation
-        float* red = x.epi + 8 * 128;   // [4 warps][8]
-        const int ti = t & 63;
-        const double inv_freq = exp(-2.0 * (double)ti / (double)p.hd * log(p.rope_base));
-        const float gam = kind == 2 ? 1.f : bf16_val(kind == 0 ? p.gq[t] : p.gk[t]);
-        for (int b0 = 0; b0 < p.B; b0 += 8) {
-            float y[8];
+        const int w = x.tid >> 5, lane = x.tid & 31, d4 = lane * 4;
+        const size_t stride = (size_t)p.n_heads * p.hd;
+        float gam[4] = {1.f, 1.f, 1.f, 1.f};
+        if (kind < 2) bf16x4(*reinterpret_cast<const uint2*>((kind == 0 ? p.gq : p.gk) + d4), gam);
+        for (int b = w; b < p.B; b += kExecThreads / 32) {
+            float* acc = p.qkvacc + (size_t)b * stride + (size_t)n * p.hd + d4;
+            const float4 a4 = __ldcg(reinterpret_cast<const float4*>(acc));
+            __stcg(reinterpret_cast<float4*>(acc), make_float4(0.f, 0.f, 0.f, 0.f));
+            float y[4] = {bf16_val(bf16_bits(a4.x)), bf16_val(bf16_bits(a4.y)), bf16_val(bf16_bits(a4.z)),
+                          bf16_val(bf16_bits(a4.w))};  // the qkv tensor is bf16
+            const int pos = __ldg(p.pos + b);
+            if (pos < 0 || pos >= p.max_ctx) continue;  // N1 reports the bad position
+            if (kind == 2) {  // V^T cache: [b][g][dim][position]
+                uint16_t* vc = p.Vc + (((size_t)b * p.nkv + g) * p.hd + d4) * p.max_ctx + pos;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int b = b0 + j;
-                float v = 0.f;
-                if (b < p.B) {
-                    v = __ldcg(acc + (size_t)b * stride);
-                    __stcg(acc + (size_t)b * stride, 0.f);
-                }
-                y[j] = bf16_val(bf16_bits(v));  // the qkv tensor is bf16
-            }
-            if (kind == 2) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int b = b0 + j;
-                    if (b < p.B) {
-                        const int pos = __ldg(p.pos + b);
-                        if (pos >= 0 && pos < p.max_ctx)  // V^T cache: [b][g][dim][position]
-                            p.Vc[(((size_t)b * p.nkv + g) * p.hd + t) * p.max_ctx + pos] = bf16_bits(y[j]);
-                    }
-                }
+                for (int e = 0; e < 4; ++e) vc[(size_t)e * p.max_ctx] = bf16_bits(y[e]);
                 continue;
             }
-            // per-head RMSNorm: sums of squares over the head's 128 dims
+            float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float ss = y[j] * y[j];
+            for (int o2 = 16; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o2);
+            const float inv = 1.0f / sqrtf(ss / (float)p.hd + p.eps);
+            float other[4];
 #pragma unroll
-                for (int o2 = 16; o2 > 0; o2 >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o2);
-                if (lane == 0) red[w * 8 + j] = ss;
+            for (int e = 0; e < 4; ++e) {
+                y[e] = y[e] * inv * gam[e];
+                other[e] = __shfl_xor_sync(0xffffffffu, y[e], 16);
             }
-            exec_bar();
+            // (cos, sin) of frequencies (d4 & 63) .. +3 at this position
+            const float4* cs = reinterpret_cast<const float4*>(p.rope + (size_t)b * (p.hd / 2) + (d4 & 63));
+            const float4 c01 = __ldcg(cs), c23 = __ldcg(cs + 1);
+            const float cv[4] = {c01.x, c01.z, c23.x, c23.z}, sv[4] = {c01.y, c01.w, c23.y, c23.w};
+            ushort4 o;
+            uint16_t* oo = reinterpret_cast<uint16_t*>(&o);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float tot = red[j] + red[8 + j] + red[16 + j] + red[24 + j];
-                y[j] = y[j] * (1.0f / sqrtf(tot / (float)p.hd + p.eps)) * gam;
-                sy[j * 128 + t] = y[j];
+            for (int e = 0; e < 4; ++e)
+                oo[e] = bf16_bits(lane < 16 ? y[e] * cv[e] - other[e] * sv[e] : y[e] * cv[e] + other[e] * sv[e]);
+            if (kind == 0) {
+                const size_t qi = ((size_t)b * p.nq + n) * p.hd + d4;
+                *reinterpret_cast<ushort4*>(p.q + qi) = o;
+                if (p.out_q) *reinterpret_cast<ushort4*>(p.out_q + qi) = o;
+            } else {
+                *reinterpret_cast<ushort4*>(p.Kc + (((size_t)b * p.nkv + g) * p.max_ctx + pos) * p.hd + d4) = o;
             }
-            exec_bar();
-            // RoPE, rotate-half pairing: dim i with dim i + hd/2
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int b = b0 + j;
-                if (b >= p.B) continue;
-                const int pos = __ldg(p.pos + b);
-                if (pos < 0 || pos >= p.max_ctx) continue;
-                double sn, cs;
-                sincos((double)pos * inv_freq, &sn, &cs);
-                const float other = sy[j * 128 + (t ^ 64)];
-                const float r = t < 64 ? y[j] * (float)cs - other * (float)sn : y[j] * (float)cs + other * (float)sn;
-                if (kind == 0) {
-                    const size_t qi = ((size_t)b * p.nq + n) * p.hd + t;
-                    p.q[qi] = bf16_bits(r);
-                    if (p.out_q) p.out_q[qi] = bf16_bits(r);
-                } else {
-                    p.Kc[(((size_t)b * p.nkv + g) * p.max_ctx + pos) * p.hd + t] = bf16_bits(r);
-                }
-            }
-            exec_bar();  // sy / red are reused by the next 8 tokens
         }
         fence_proxy_async_global();  // the caches and q are read by TMA in the attention tasks
         int* ev = x.ctr + (unfused(p) ? p.ev_branch_all : p.ev_g + g);
@@ -544,9 +522,18 @@ struct Decode : WorkloadBase {
 
     __device__ static bool norm1(const Params& p, Ctx& x, TaskDesc& d, int b) {
         if (!group_wait(x, d, nullptr, 0, 312)) return false;
-        if (x.tid == 0) {
+        {
+            // the request's rotary (cos, sin) per frequency, for the Q and K
+            // branches: angle pos * base^(-2i / head_dim), in double
             const int pos = __ldg(p.pos + b);
-            if (pos < 0 || pos >= p.max_ctx) fail(x.ctl, ET_ERR_INVALID, 313, b, pos, p.max_ctx);
+            if (pos < 0 || pos >= p.max_ctx) {
+                if (x.tid == 0) fail(x.ctl, ET_ERR_INVALID, 313, b, pos, p.max_ctx);
+            } else if (x.tid < p.hd / 2) {
+                const double inv_freq = exp(-2.0 * (double)x.tid / (double)p.hd * log(p.rope_base));
+                double sn, cs;
+                sincos((double)pos * inv_freq, &sn, &cs);
+                p.rope[(size_t)b * (p.hd / 2) + x.tid] = make_float2((float)cs, (float)sn);
+            }
         }
         const uint16_t* xr = p.X + (size_t)b * p.hidden;
         float v[32];
@@ -576,34 +563,54 @@ struct Decode : WorkloadBase {
     __device__ static bool norm2(const Params& p, Ctx& x, TaskDesc& d, int b) {
         const int tgt = p.n_m * p.nkv;
         if (!group_wait(x, d, x.ctr + p.ev_o, tgt, 314)) return false;
-        const int nv = p.hidden / kExecThreads;
-        const size_t r0 = (size_t)b * p.hidden + x.tid * nv;
+        // thread t holds elements (j * 128 + t) * 8 .. +7, j < hidden / 1024:
+        // every load issued before the stores
+        const int nv = p.hidden / kExecThreads, n8 = nv / 8;  // n8 <= 4
+        const size_t row = (size_t)b * p.hidden;
+        float4 a[8];
+        uint4 xv[4];
         float v[32];
-        for (int i = 0; i < nv; i += 8) {
-            float xv[8];
-            bf16x8(*reinterpret_cast<const uint4*>(p.X + r0 + i), xv);
-            uint4 o;
-            uint16_t* oo = reinterpret_cast<uint16_t*>(&o);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const float a = __ldcg(p.h1acc + r0 + i + t);
-                __stcg(p.h1acc + r0 + i + t, 0.f);
-                oo[t] = bf16_bits(xv[t] + a);
-                v[i + t] = bf16_val(oo[t]);
+        for (int j = 0; j < 4; ++j)
+            if (j < n8) {
+                const size_t e = row + (size_t)(j * kExecThreads + x.tid) * 8;
+                a[2 * j] = __ldcg(reinterpret_cast<const float4*>(p.h1acc + e));
+                a[2 * j + 1] = __ldcg(reinterpret_cast<const float4*>(p.h1acc + e + 4));
+                xv[j] = *reinterpret_cast<const uint4*>(p.X + e);
             }
-            *reinterpret_cast<uint4*>(p.h1 + r0 + i) = o;
-            if (p.out_h1) *reinterpret_cast<uint4*>(p.out_h1 + r0 + i) = o;
-        }
-        const float inv = row_inv_rms(p, x, v, nv);
-        for (int i = 0; i < nv; i += 8) {
-            float gg[8];
-            bf16x8(*reinterpret_cast<const uint4*>(p.g2 + x.tid * nv + i), gg);
-            uint4 o;
-            uint16_t* oo = reinterpret_cast<uint16_t*>(&o);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) oo[t] = bf16_bits(v[i + t] * inv * gg[t]);
-            *reinterpret_cast<uint4*>(p.xn2 + r0 + i) = o;
-        }
+        for (int j = 0; j < 4; ++j)
+            if (j < n8) {
+                const size_t e = row + (size_t)(j * kExecThreads + x.tid) * 8;
+                __stcg(reinterpret_cast<float4*>(p.h1acc + e), make_float4(0.f, 0.f, 0.f, 0.f));
+                __stcg(reinterpret_cast<float4*>(p.h1acc + e + 4), make_float4(0.f, 0.f, 0.f, 0.f));
+                float xf[8];
+                bf16x8(xv[j], xf);
+                const float av[8] = {a[2 * j].x, a[2 * j].y, a[2 * j].z, a[2 * j].w,
+                                     a[2 * j + 1].x, a[2 * j + 1].y, a[2 * j + 1].z, a[2 * j + 1].w};
+                uint4 o;
+                uint16_t* oo = reinterpret_cast<uint16_t*>(&o);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    oo[t] = bf16_bits(xf[t] + av[t]);
+                    v[j * 8 + t] = bf16_val(oo[t]);
+                }
+                *reinterpret_cast<uint4*>(p.h1 + e) = o;
+                if (p.out_h1) *reinterpret_cast<uint4*>(p.out_h1 + e) = o;
+            }
+        const float inv = row_inv_rms(p, x, v, nv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (j < n8) {
+                const size_t c = (size_t)(j * kExecThreads + x.tid) * 8;
+                float gg[8];
+                bf16x8(*reinterpret_cast<const uint4*>(p.g2 + c), gg);
+                uint4 o;
+                uint16_t* oo = reinterpret_cast<uint16_t*>(&o);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) oo[t] = bf16_bits(v[j * 8 + t] * inv * gg[t]);
+                *reinterpret_cast<uint4*>(p.xn2 + row + c) = o;
+            }
         fence_proxy_async_global();  // xn2 is read by TMA in the gate/up tasks
         if (group_finish_notify(x, d, x.ctr + p.ev_n2, 1, p.B) && push_all(p))
             group_push(x, p.n_gu, [&](int n) { return task_word(ET_OP_DEC_GATEUP, n, 0); });
