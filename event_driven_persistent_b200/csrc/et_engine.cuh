@@ -57,7 +57,7 @@ struct SmemCtl {
     uint64_t ring_full[kRing];
     uint64_t ring_empty[kRing];
     uint64_t drain;
-    uint64_t s_full, p_full, o_full;  // attention stages: S in TMEM / P in smem / O in TMEM
+    uint64_t s_full[2], p_full, o_full;  // attention stages: S (two buffers) / P in smem / O in TMEM
     uint32_t tmem_base;
     int start_status;
     int bcast[8];
@@ -94,6 +94,10 @@ struct Ctx {
 
 // Defaults of the workload interface for what a workload does not use.
 struct WorkloadBase {
+    // engine paths a workload uses (the others are compiled out: a smaller
+    // megakernel has less code to fetch cold)
+    static constexpr bool kStream = false;  // stream / attention tasks
+    static constexpr bool kGather = false;  // tensor-core tasks with gathered B rows
     // stream tasks: stages that may be copied before the task's input wait,
     // the bytes stage s delivers, and the copies of stage s into `dst`
     // (completing on `bar`); `late` = issued after the input wait, so the
@@ -291,7 +295,8 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             mbar_init(&sc->ring_empty[r], 2);  // MMA warp + exec group
         }
         mbar_init(&sc->drain, 1);
-        mbar_init(&sc->s_full, 1);
+        mbar_init(&sc->s_full[0], 1);
+        mbar_init(&sc->s_full[1], 1);
         mbar_init(&sc->p_full, 1);
         mbar_init(&sc->o_full, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -451,7 +456,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             TaskDesc d = sc->pd;
             __syncwarp();
             if (brk) break;
-            if (r == 1 && d.valid && d.stream) {
+            if (W::kStream && r == 1 && d.valid && d.stream) {
                 // stream task: stages that do not depend on the task's input
                 // events first, then the wait, then the rest
                 bool ok = true;
@@ -497,11 +502,11 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 ok = sc->pok;
                 __syncwarp();
                 if (!ok) break;
-            } else if (r == 1 && d.valid && d.gemm) {
+            } else if (W::kGemm && r == 1 && d.valid && d.gemm) {
                 const CUtensorMap* am = W::a_map(p, d.a_map);
                 const uint32_t bbytes = 2u * (uint32_t)d.n * 128u;  // both K atoms
                 bool ok = true;
-                if (!d.gather) {
+                if (!(W::kGather && d.gather)) {
                     if (lane == 0) {
                         const CUtensorMap* bm = W::b_map(p, d.b_map);
                         // 1. weight tiles of the first stages, before the input
@@ -626,66 +631,80 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 TaskDesc d = sc->ring[slot];
                 mbar_arrive(&sc->ring_empty[slot]);
                 if (d.word == kExitWord) break;
-                if (d.valid && d.stream && !d.attn) {  // stages consumed by the exec group: keep the sequence
+                if (W::kStream && d.valid && d.stream && !d.attn) {  // stages consumed by the exec group: keep the sequence
                     for (int s = 0; s < d.nk; ++s, ++nst) alloc.next(d.sbytes);
                     continue;
                 }
-                if (d.valid && d.stream) {
-                    // attention stages: S = K Q^T into columns [0, 16) of the
-                    // task's accumulator (keys x query heads), then, once the
-                    // exec group has read S and written P (query heads x keys,
-                    // bf16) to its scratch, O = V^T P^T into columns [16, 32)
-                    // (head dims x query heads); the stage is free after that
+                if (W::kStream && d.valid && d.stream) {
+                    // attention stages (k = the run's count of attention stages
+                    // so far): S_k = K Q^T into TMEM columns [16 (k & 1), +16)
+                    // (keys x query heads), O_k = V^T P_k^T into columns
+                    // [32, 48) (head dims x query heads) once the exec group
+                    // has read S_k and written P_k (query heads x keys, bf16)
+                    // to its scratch.  S_{k+1} is issued before waiting for
+                    // P_k, so the exec group's softmax of stage k + 1 overlaps
+                    // O_k; the stage is free after O_k.
                     const uint32_t buf = g & 1;
                     if (!mbar_wait(&sc->acc_empty[buf], ((g >> 1) & 1) ^ 1, ctl, x.timeout_ns, 913)) break;
                     tc_fence_after();
-                    const uint32_t dS = sc->tmem_base + buf * kMaxN, dO = dS + 16;
+                    const uint32_t dT = sc->tmem_base + buf * kMaxN;
                     const uint32_t idesc = idesc_bf16_f32(128, 16);
                     const uint32_t pa = smem_u32(epi);
-                    bool ok = true;
-                    for (int s = 0; s < d.nk; ++s, ++nst, ++na) {
-                        const uint32_t ss = nst % kSlots;
-                        const uint32_t off = alloc.next(d.sbytes);
-                        if (!mbar_wait(&sc->full[ss], (nst / kSlots) & 1, ctl, x.timeout_ns, 914)) {
-                            ok = false;
-                            break;
-                        }
+                    const uint32_t nst0 = nst, na0 = na;
+                    auto issue_s = [&](int s, uint32_t off) -> bool {
+                        const uint32_t gs = nst0 + (uint32_t)s, k = na0 + (uint32_t)s;
+                        if (!mbar_wait(&sc->full[gs % kSlots], (gs / kSlots) & 1, ctl, x.timeout_ns, 914)) return false;
                         tc_fence_after();
-                        const uint32_t ka = smem_u32(arena + off), va = ka + kAttnVOff, qa = ka + kAttnQOff;
+                        const uint32_t ka = smem_u32(arena + off), qa = ka + kAttnQOff;
 #pragma unroll
                         for (int at = 0; at < 2; ++at) {
                             const uint64_t ad = sdesc_k128(ka + at * kAAtomBytes);
                             const uint64_t bd = sdesc_k128(qa + at * 16u * 128u);
 #pragma unroll
                             for (int kk = 0; kk < kAtomK / 16; ++kk)
-                                tc_mma_bf16(dS, ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
+                                tc_mma_bf16(dT + 16u * (k & 1), ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
                         }
-                        tc_commit(&sc->s_full);
+                        tc_commit(&sc->s_full[k & 1]);
                         issued_any = true;
-                        if (!mbar_wait(&sc->p_full, na & 1, ctl, x.timeout_ns, 915)) {
+                        return true;
+                    };
+                    bool ok = true;
+                    uint32_t off_cur = alloc.next(d.sbytes);
+                    ok = issue_s(0, off_cur);
+                    for (int s = 0; ok && s < d.nk; ++s) {
+                        uint32_t off_next = 0;
+                        if (s + 1 < d.nk) {
+                            off_next = alloc.next(d.sbytes);
+                            if (!(ok = issue_s(s + 1, off_next))) break;
+                        }
+                        if (!mbar_wait(&sc->p_full, (na0 + (uint32_t)s) & 1, ctl, x.timeout_ns, 915)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
+                        const uint32_t va = smem_u32(arena + off_cur) + kAttnVOff;
 #pragma unroll
                         for (int at = 0; at < 2; ++at) {
                             const uint64_t ad = sdesc_k128(va + at * kAAtomBytes);
                             const uint64_t bd = sdesc_k128(pa + at * 16u * 128u);
 #pragma unroll
                             for (int kk = 0; kk < kAtomK / 16; ++kk)
-                                tc_mma_bf16(dO, ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
+                                tc_mma_bf16(dT + 32u, ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
                         }
                         tc_commit(&sc->o_full);
-                        tc_commit(&sc->empty[ss]);
+                        tc_commit(&sc->empty[(nst0 + (uint32_t)s) % kSlots]);
+                        off_cur = off_next;
                     }
                     if (!ok) break;
+                    nst += (uint32_t)d.nk;
+                    na += (uint32_t)d.nk;
                     // one acc_full phase per use of an accumulator, attention
                     // tasks included: the epilogues' parity counts on it
                     tc_commit(&sc->acc_full[buf]);
                     ++g;
                     continue;
                 }
-                if (!(d.valid && d.gemm)) continue;
+                if (!(W::kGemm && d.valid && d.gemm)) continue;
                 const uint32_t buf = g & 1;
                 if (!mbar_wait(&sc->acc_empty[buf], ((g >> 1) & 1) ^ 1, ctl, x.timeout_ns, 911)) break;
                 tc_fence_after();
@@ -701,7 +720,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         break;
                     }
                     tc_fence_after();
-                    fence_proxy_async_smem();  // rows copied by cp.async (generic proxy) -> tensor core
+                    if (W::kGather && d.gather) fence_proxy_async_smem();  // rows copied by cp.async (generic proxy) -> tensor core
                     const uint32_t a0 = smem_u32(arena + off);
 #pragma unroll
                     for (int at = 0; at < 2; ++at) {
@@ -742,7 +761,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             if (d.word == kExitWord) break;
             if (!d.valid) continue;
             if (x.debug & ET_DEBUG_DELAY) debug_delay(d.word ^ (ra.epoch * 977u));
-            if (d.stream) {
+            if (W::kStream && d.stream) {
                 if (d.attn) {
                     const uint32_t buf = g & 1;
                     x.taddr = sc->tmem_base + buf * kMaxN + ((uint32_t)((warp & 3) * 32) << 16);
@@ -750,7 +769,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     ++g;
                 }
                 if (!W::stream_exec(p, x, d)) break;
-            } else if (d.gemm) {
+            } else if (W::kGemm && d.gemm) {
                 const uint32_t buf = g & 1;
                 const uint32_t par = (g >> 1) & 1;
                 if (x.tid == 0) sc->bcast[5] = mbar_wait(&sc->acc_full[buf], par, ctl, x.timeout_ns, 921);

@@ -41,6 +41,7 @@ constexpr int kKeysPerStage = 128;  // keys of one attention stage (the M of S =
 struct Decode : WorkloadBase {
     using Params = DecodeParams;
     static constexpr bool kGemm = true;
+    static constexpr bool kStream = true;
 
     __device__ static bool unfused(const Params& p) { return p.sched == ET_SCHED_UNFUSED; }
     __device__ static bool push_all(const Params& p) { return p.sched == ET_SCHED_DYNAMIC; }
@@ -186,11 +187,12 @@ struct Decode : WorkloadBase {
     // One attention split (exec group; the MMA warp runs the products).
     // Per stage of 128 keys: thread r (its warp's TMEM lane) reads the scores
     // of key r for every query head from S, the group takes the stage max and
-    // the online-softmax rescale, writes P = bf16(exp(s - max)) (query heads x
-    // keys, the 128-byte swizzled K-major layout of a tensor-core B operand)
-    // and, on a partial stage, zeroes the V^T columns of the missing keys;
-    // then thread r reads head dim r of every head from O = V^T P^T.  The
-    // normaliser sums the bf16 probabilities the product used.
+    // the online-softmax rescale; then it folds the previous stage's O (head
+    // dim r of every head) while the next stage's S is computed, writes P =
+    // bf16(exp(s - max)) (query heads x keys, the 128-byte swizzled K-major
+    // layout of a tensor-core B operand) and, on a partial stage, zeroes the
+    // V^T columns of the missing keys.  The normaliser sums the bf16
+    // probabilities the product used.
     __device__ static bool stream_exec(const Params& p, Ctx& x, TaskDesc& d) {
         const int bb = d.p[0], g = d.p[1], s = d.p[2];
         const int w = x.tid >> 5, lane = x.tid & 31;
@@ -201,22 +203,34 @@ struct Decode : WorkloadBase {
         for (int i = x.tid; i < 1024; i += kExecThreads)   // query-head rows grp..15 of P stay 0
             if (((i >> 5) & 15) >= grp) reinterpret_cast<uint32_t*>(P)[i] = 0u;
         const float scale = 0.08838834764831845f;  // 1 / sqrt(128)
-        float m[4], l[4], o[4];
+        float m[4], l[4], o[4], alpha_prev[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
             m[h] = -INFINITY;
             l[h] = 0.f;
             o[h] = 0.f;
+            alpha_prev[h] = 0.f;
         }
+        // fold O of attention stage k into o with that stage's rescale
+        auto fold = [&](uint32_t k) -> bool {
+            if (!exec_mbar_wait(x, &x.sc->o_full, k & 1, 317, 3)) return false;
+            tc_fence_after();
+            float ov[4];
+            __syncwarp();
+            tmem_ld4_wait(x.taddr + 32u, ov);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) o[h] = o[h] * alpha_prev[h] + ov[h];
+            return true;
+        };
         StageAlloc al = stream_alloc(d);
         for (int st = 0; st < d.nk; ++st) {
-            const uint32_t off = al.next(d.sbytes);
+            const uint32_t off = al.next(d.sbytes), k = x.na + (uint32_t)st;
             const int nks = stage_keys(d, st);
-            if (!exec_mbar_wait(x, &x.sc->s_full, x.na & 1, 316, 2)) return false;
+            if (!exec_mbar_wait(x, &x.sc->s_full[k & 1], (k >> 1) & 1, 316, 2)) return false;
             tc_fence_after();
             float sv[4];
             __syncwarp();
-            tmem_ld4_wait(x.taddr, sv);
+            tmem_ld4_wait(x.taddr + 16u * (k & 1), sv);
             const bool valid = r < nks;
             float mx[4];
 #pragma unroll
@@ -231,6 +245,7 @@ struct Decode : WorkloadBase {
                 for (int h = 0; h < 4; ++h) red[w * 4 + h] = mx[h];
             exec_bar();
             float alpha[4], ps[4];
+            uint16_t pb[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 float pv = 0.f;
@@ -240,19 +255,21 @@ struct Decode : WorkloadBase {
                     alpha[h] = expf(m[h] - mn);  // 0 on the first stage (m = -inf)
                     m[h] = mn;
                     if (valid) {
-                        const uint16_t pb = bf16_bits(expf(sv[h] - mn));
-                        pv = bf16_val(pb);
-                        *reinterpret_cast<uint16_t*>(P + (r >> 6) * 2048 + h * 128 +
-                                                     ((((r & 63) >> 3) ^ (h & 7)) << 4) + (r & 7) * 2) = pb;
-                    } else {
-                        *reinterpret_cast<uint16_t*>(P + (r >> 6) * 2048 + h * 128 +
-                                                     ((((r & 63) >> 3) ^ (h & 7)) << 4) + (r & 7) * 2) = 0;
+                        pb[h] = bf16_bits(expf(sv[h] - mn));
+                        pv = bf16_val(pb[h]);
                     }
                 }
                 ps[h] = pv;
 #pragma unroll
                 for (int o2 = 16; o2 > 0; o2 >>= 1) ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], o2);
             }
+            // the previous stage's O: its product has read P, which is then free
+            if (st > 0 && !fold(k - 1)) return false;
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                if (h < grp)
+                    *reinterpret_cast<uint16_t*>(P + (r >> 6) * 2048 + h * 128 + ((((r & 63) >> 3) ^ (h & 7)) << 4) +
+                                                 (r & 7) * 2) = pb[h];
             if (nks < kKeysPerStage) {
                 // V^T row r (head dim r): the columns of keys nks..127 to 0,
                 // after the stage's copies landed (that phase is already
@@ -260,9 +277,9 @@ struct Decode : WorkloadBase {
                 const uint32_t gs = d.st0 + (uint32_t)st;
                 if (!exec_mbar_wait(x, &x.sc->full[gs % kSlots], (gs / kSlots) & 1, 318, 5)) return false;
                 uint8_t* vr = x.arena + off + kAttnVOff + r * 128;
-                for (int k = nks; k < kKeysPerStage; ++k)
-                    *reinterpret_cast<uint16_t*>(vr + (k >> 6) * kAAtomBytes + ((((k & 63) >> 3) ^ (r & 7)) << 4) +
-                                                 (k & 7) * 2) = 0;
+                for (int kk = nks; kk < kKeysPerStage; ++kk)
+                    *reinterpret_cast<uint16_t*>(vr + (kk >> 6) * kAAtomBytes + ((((kk & 63) >> 3) ^ (r & 7)) << 4) +
+                                                 (kk & 7) * 2) = 0;
             }
             if (lane == 0)
 #pragma unroll
@@ -272,16 +289,13 @@ struct Decode : WorkloadBase {
             exec_bar();
             if (x.tid == 0) mbar_arrive(&x.sc->p_full);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) l[h] = l[h] * alpha[h] + red[16 + h] + red[20 + h] + red[24 + h] + red[28 + h];
-            if (!exec_mbar_wait(x, &x.sc->o_full, x.na & 1, 317, 3)) return false;
-            tc_fence_after();
-            float ov[4];
-            __syncwarp();
-            tmem_ld4_wait(x.taddr + 16, ov);
-#pragma unroll
-            for (int h = 0; h < 4; ++h) o[h] = o[h] * alpha[h] + ov[h];
-            ++x.na;
+            for (int h = 0; h < 4; ++h) {
+                l[h] = l[h] * alpha[h] + red[16 + h] + red[20 + h] + red[24 + h] + red[28 + h];
+                alpha_prev[h] = alpha[h];
+            }
         }
+        if (!fold(x.na + (uint32_t)d.nk - 1)) return false;
+        x.na += (uint32_t)d.nk;
         acc_release(x.acc_empty);
         const int tid = r;  // head dim of this thread
         // partial of this split: o (unnormalised), running max m, sum l

@@ -37,6 +37,7 @@ namespace et {
 struct Moe : WorkloadBase {
     using Params = MoeParams;
     static constexpr bool kGemm = true;
+    static constexpr bool kGather = true;
 
     __device__ static bool is_unfused(const Params& p) { return p.sched == ET_SCHED_UNFUSED; }
 

@@ -20,6 +20,7 @@ namespace et {
 struct MoeMlp : WorkloadBase {
     using Params = MoeMlpParams;
     static constexpr bool kGemm = true;
+    static constexpr bool kGather = true;
     static constexpr int kMlpMaps = 8;  // MLP tensor-map ids are offset by this
 
     __device__ static bool is_mlp(uint32_t word) {
