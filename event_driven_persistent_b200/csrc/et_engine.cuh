@@ -263,7 +263,7 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* arena = base;
-    uint8_t* scratch = arena + kArenaBytes;
+    uint8_t* scratch = arena + ((W::kGemm || W::kStream) ? kArenaBytes : 0);
     float* epi = reinterpret_cast<float*>(scratch);
     uint8_t* simt = scratch + kEpiBytes;
     SmemCtl* sc = reinterpret_cast<SmemCtl*>(scratch + kScratchBytes);

@@ -738,7 +738,7 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     in.max_T = g->d.max_T;
     in.n_ctas = g->n_ctas;
     in.threads = kThreads;
-    in.smem_bytes = kSmemBytes;
+    in.smem_bytes = g->d.kind == ET_GRAPH_SPLITK ? kSmemNoArenaBytes : kSmemBytes;
     in.fetch_batch = g->d.fetch_batch;
     in.hidden = g->d.hidden;
     in.inter = g->d.inter;

@@ -36,6 +36,9 @@ constexpr uint32_t kAttnVOff = 32768, kAttnQOff = 65536, kAttnStage = 65536 + 40
 constexpr int kEpiBytes = 64 * 33 * 4;   // gate/up exchange staging (start of the scratch)
 constexpr int kCtlBytes = 2048;          // mbarriers, task ring, broadcast words
 constexpr int kSmemBytes = 1024 /*align slack*/ + kArenaBytes + kScratchBytes + kCtlBytes;
+// a workload with neither tensor-core nor stream tasks has no stage arena and
+// asks only for its scratch and control block
+constexpr int kSmemNoArenaBytes = 1024 + kScratchBytes + kCtlBytes;
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above the sm_100 per-block limit");
 
 // Per-bucket static task lists: CSR over CTAs.  Hybrid schedules have a

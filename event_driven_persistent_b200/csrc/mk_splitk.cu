@@ -76,9 +76,9 @@ __global__ void __launch_bounds__(kThreads, 1) splitk_kernel(const __grid_consta
 
 // Called once per graph on its device: opt in to the shared-memory size.
 cudaError_t splitk_setup(int* max_blocks_per_sm) {
-    cudaError_t e = cudaFuncSetAttribute(splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemNoArenaBytes);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(max_blocks_per_sm, splitk_kernel, kThreads, kSmemBytes);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(max_blocks_per_sm, splitk_kernel, kThreads, kSmemNoArenaBytes);
 }
 
 // The two-launch control: the same two operators as plain kernels, one
@@ -116,7 +116,7 @@ cudaError_t launch_splitk_two(const float* A, int rows, int cols, int chunk, flo
 cudaError_t launch_splitk(const SplitKParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s) {
     // the launch's own status (not an unrelated error left pending earlier)
     void* args[] = {const_cast<SplitKParams*>(&p), const_cast<RunArgs*>(&ra)};
-    return cudaLaunchKernel(reinterpret_cast<const void*>(splitk_kernel), dim3(n_ctas), dim3(kThreads), args, kSmemBytes, s);
+    return cudaLaunchKernel(reinterpret_cast<const void*>(splitk_kernel), dim3(n_ctas), dim3(kThreads), args, kSmemNoArenaBytes, s);
 }
 
 }  // namespace et
