@@ -264,3 +264,31 @@ def test_moe_full_size(full_moe, sched, zipf, T):
             cache[(zipf, T, i, out["topk"][i].tobytes(), w_o[i].tobytes())] = row
     y_ref = np.stack([cache[(zipf, T, i, out["topk"][i].tobytes(), w_o[i].tobytes())] for i in toks])
     assert maxnorm_err(out["y"][toks], y_ref) <= TOL_Y
+
+
+@pytest.mark.parametrize("flags", ["trace", "trace+cta"])
+def test_cta_timing_records(small_inputs, flags):
+    """ET_DEBUG_CTA_TIMES adds one record per CTA (op ET_OP_CTA, a = CTA
+    index) with entry <= set-up done <= exit, and only together with
+    ET_DEBUG_TRACE; the task records are unchanged."""
+    d = small_inputs
+    dbg = et.ET_DEBUG_TRACE | (et.ET_DEBUG_CTA_TIMES if flags == "trace+cta" else 0)
+    g = et.et_build_graph(et.ET_GRAPH_MOE, "dynamic", 64, debug_flags=dbg, **SMALL)
+    try:
+        st, _ = run_moe(g, d, 21, 4, 16)
+        assert st == 0
+        tr = et.et_get_trace(g)
+        cta = [r for r in tr if r[0] == 60]
+        tasks = [r for r in tr if r[0] != 60]
+        assert tasks, "no task records"
+        if flags == "trace":
+            assert cta == []
+            return
+        n = et.et_get_info(g)["n_ctas"]
+        assert sorted(r[1] for r in cta) == list(range(n))
+        for r in cta:  # (op, a, b, sm, start, end, t_fetch, t_ready, t_acc, t_end)
+            assert r[6] <= r[7] <= r[9]
+        assert min(r[6] for r in cta) <= min(r[6] for r in tasks)
+        assert max(r[9] for r in cta) >= max(r[9] for r in tasks)
+    finally:
+        et.et_destroy_graph(g)
