@@ -212,8 +212,10 @@ struct Decode : WorkloadBase {
             alpha_prev[h] = 0.f;
         }
         // fold O of attention stage k into o with that stage's rescale
-        auto fold = [&](uint32_t k) -> bool {
-            if (!exec_mbar_wait(x, &x.sc->o_full, k & 1, 317, 3)) return false;
+        // (broadcast slot 3 inside the loop; 5 for the last fold, which follows
+        // the loop's last fold with no exec-group barrier in between)
+        auto fold = [&](uint32_t k, int slot) -> bool {
+            if (!exec_mbar_wait(x, &x.sc->o_full, k & 1, 317, slot)) return false;
             tc_fence_after();
             float ov[4];
             __syncwarp();
@@ -264,7 +266,7 @@ struct Decode : WorkloadBase {
                 for (int o2 = 16; o2 > 0; o2 >>= 1) ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], o2);
             }
             // the previous stage's O: its product has read P, which is then free
-            if (st > 0 && !fold(k - 1)) return false;
+            if (st > 0 && !fold(k - 1, 3)) return false;
 #pragma unroll
             for (int h = 0; h < 4; ++h)
                 if (h < grp)
@@ -294,7 +296,7 @@ struct Decode : WorkloadBase {
                 alpha_prev[h] = alpha[h];
             }
         }
-        if (!fold(x.na + (uint32_t)d.nk - 1)) return false;
+        if (!fold(x.na + (uint32_t)d.nk - 1, 5)) return false;
         x.na += (uint32_t)d.nk;
         acc_release(x.acc_empty);
         const int tid = r;  // head dim of this thread
