@@ -57,7 +57,7 @@ struct SmemCtl {
     uint64_t ring_full[kRing];
     uint64_t ring_empty[kRing];
     uint64_t drain;
-    uint64_t s_full[2], p_full, o_full;  // attention stages: S (two buffers) / P in smem / O in TMEM
+    uint64_t s_full[2], p_full[2], o_full[2];  // attention stages k: buffers k & 1 of S, P and O
     uint32_t tmem_base;
     int start_status;
     int bcast[8];
@@ -297,8 +297,10 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
         mbar_init(&sc->drain, 1);
         mbar_init(&sc->s_full[0], 1);
         mbar_init(&sc->s_full[1], 1);
-        mbar_init(&sc->p_full, 1);
-        mbar_init(&sc->o_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sc->p_full[b], 1);
+            mbar_init(&sc->o_full[b], 1);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
@@ -637,13 +639,14 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                 }
                 if (W::kStream && d.valid && d.stream) {
                     // attention stages (k = the run's count of attention stages
-                    // so far): S_k = K Q^T into TMEM columns [16 (k & 1), +16)
-                    // (keys x query heads), O_k = V^T P_k^T into columns
-                    // [32, 48) (head dims x query heads) once the exec group
-                    // has read S_k and written P_k (query heads x keys, bf16)
-                    // to its scratch.  S_{k+1} is issued before waiting for
-                    // P_k, so the exec group's softmax of stage k + 1 overlaps
-                    // O_k; the stage is free after O_k.
+                    // so far; buffer j = k & 1 of S, P and O): S_k = K Q^T into
+                    // TMEM columns [16 j, +16) (keys x query heads), O_k =
+                    // V^T P_k^T into columns [32 + 16 j, +16) (head dims x
+                    // query heads) once the exec group has read S_k and written
+                    // P_k (query heads x keys, bf16) to scratch + 4 KB * j.
+                    // S_{k+1} is issued before waiting for P_k, and the exec
+                    // group writes P_{k+1} while O_k runs; the stage is free
+                    // after O_k.
                     const uint32_t buf = g & 1;
                     if (!mbar_wait(&sc->acc_empty[buf], ((g >> 1) & 1) ^ 1, ctl, x.timeout_ns, 913)) break;
                     tc_fence_after();
@@ -677,7 +680,8 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                             off_next = alloc.next(d.sbytes);
                             if (!(ok = issue_s(s + 1, off_next))) break;
                         }
-                        if (!mbar_wait(&sc->p_full, (na0 + (uint32_t)s) & 1, ctl, x.timeout_ns, 915)) {
+                        const uint32_t k = na0 + (uint32_t)s, j = k & 1;
+                        if (!mbar_wait(&sc->p_full[j], (k >> 1) & 1, ctl, x.timeout_ns, 915)) {
                             ok = false;
                             break;
                         }
@@ -686,12 +690,12 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
 #pragma unroll
                         for (int at = 0; at < 2; ++at) {
                             const uint64_t ad = sdesc_k128(va + at * kAAtomBytes);
-                            const uint64_t bd = sdesc_k128(pa + at * 16u * 128u);
+                            const uint64_t bd = sdesc_k128(pa + 4096u * j + at * 16u * 128u);
 #pragma unroll
                             for (int kk = 0; kk < kAtomK / 16; ++kk)
-                                tc_mma_bf16(dT + 32u, ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
+                                tc_mma_bf16(dT + 32u + 16u * j, ad + 2 * kk, bd + 2 * kk, idesc, (at | kk) ? 1u : 0u);
                         }
-                        tc_commit(&sc->o_full);
+                        tc_commit(&sc->o_full[j]);
                         tc_commit(&sc->empty[(nst0 + (uint32_t)s) % kSlots]);
                         off_cur = off_next;
                     }

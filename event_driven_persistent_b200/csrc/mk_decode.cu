@@ -198,10 +198,10 @@ struct Decode : WorkloadBase {
         const int w = x.tid >> 5, lane = x.tid & 31;
         const int r = ((w + kExecWarp0) & 3) * 32 + lane;
         const int grp = p.grp;
-        uint8_t* P = reinterpret_cast<uint8_t*>(x.epi);  // [2 key atoms][16 rows][128 B]
-        float* red = x.epi + 1024;                          // [max: 4 warps x 4 heads][sum: same]
-        for (int i = x.tid; i < 1024; i += kExecThreads)   // query-head rows grp..15 of P stay 0
-            if (((i >> 5) & 15) >= grp) reinterpret_cast<uint32_t*>(P)[i] = 0u;
+        uint8_t* P0 = reinterpret_cast<uint8_t*>(x.epi);  // 2 x [2 key atoms][16 rows][128 B]
+        float* red = x.epi + 2048;                           // [max: 4 warps x 4 heads][sum: same]
+        for (int i = x.tid; i < 2048; i += kExecThreads)    // query-head rows grp..15 of both P stay 0
+            if (((i >> 5) & 15) >= grp) reinterpret_cast<uint32_t*>(P0)[i] = 0u;
         const float scale = 0.08838834764831845f;  // 1 / sqrt(128)
         float m[4], l[4], o[4], alpha_prev[4];
 #pragma unroll
@@ -215,11 +215,11 @@ struct Decode : WorkloadBase {
         // (broadcast slot 3 inside the loop; 5 for the last fold, which follows
         // the loop's last fold with no exec-group barrier in between)
         auto fold = [&](uint32_t k, int slot) -> bool {
-            if (!exec_mbar_wait(x, &x.sc->o_full, k & 1, 317, slot)) return false;
+            if (!exec_mbar_wait(x, &x.sc->o_full[k & 1], (k >> 1) & 1, 317, slot)) return false;
             tc_fence_after();
             float ov[4];
             __syncwarp();
-            tmem_ld4_wait(x.taddr + 32u, ov);
+            tmem_ld4_wait(x.taddr + 32u + 16u * (k & 1), ov);
 #pragma unroll
             for (int h = 0; h < 4; ++h) o[h] = o[h] * alpha_prev[h] + ov[h];
             return true;
@@ -228,6 +228,7 @@ struct Decode : WorkloadBase {
         for (int st = 0; st < d.nk; ++st) {
             const uint32_t off = al.next(d.sbytes), k = x.na + (uint32_t)st;
             const int nks = stage_keys(d, st);
+            uint8_t* P = P0 + 4096 * (k & 1);
             if (!exec_mbar_wait(x, &x.sc->s_full[k & 1], (k >> 1) & 1, 316, 2)) return false;
             tc_fence_after();
             float sv[4];
@@ -265,8 +266,6 @@ struct Decode : WorkloadBase {
 #pragma unroll
                 for (int o2 = 16; o2 > 0; o2 >>= 1) ps[h] += __shfl_xor_sync(0xffffffffu, ps[h], o2);
             }
-            // the previous stage's O: its product has read P, which is then free
-            if (st > 0 && !fold(k - 1, 3)) return false;
 #pragma unroll
             for (int h = 0; h < 4; ++h)
                 if (h < grp)
@@ -289,7 +288,10 @@ struct Decode : WorkloadBase {
             fence_proxy_async_smem();  // P and the zeroed V^T columns are read by the tensor core
             tc_fence_before();
             exec_bar();
-            if (x.tid == 0) mbar_arrive(&x.sc->p_full);
+            if (x.tid == 0) mbar_arrive(&x.sc->p_full[k & 1]);
+            // the previous stage's O, while this stage's product runs (its
+            // P buffer is then free for the stage after)
+            if (st > 0 && !fold(k - 1, 3)) return false;
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
                 l[h] = l[h] * alpha[h] + red[16 + h] + red[20 + h] + red[24 + h] + red[28 + h];
