@@ -177,7 +177,7 @@ def full_decode():
 
 
 @pytest.mark.parametrize("sched", ["static", "hybrid", "dynamic"])
-@pytest.mark.parametrize("B", [1, 16, 64])
+@pytest.mark.parametrize("B", [1, 16, 37, 64])
 def test_decode_full_size(full_decode, sched, B):
     d, wt, graphs = full_decode
     st, out = run_decode(graphs[sched], d, B, wt)
