@@ -40,7 +40,7 @@ class et_graph_desc(ctypes.Structure):
         "splitk_tile_rows")] + [("rms_eps", ctypes.c_float)] + [(n, ctypes.c_int) for n in (
             "fetch_batch", "debug_flags", "device", "n_ctas")] + [("timeout_ms", ctypes.c_float)] + [
             (n, ctypes.c_int) for n in ("n_heads", "n_kv_heads", "head_dim", "max_ctx")] + [
-            ("rope_base", ctypes.c_float), ("mlp_inter", ctypes.c_int)]
+            ("rope_base", ctypes.c_float), ("mlp_inter", ctypes.c_int), ("moe_xp_min_T", ctypes.c_int)]
 
 
 class et_graph_info(ctypes.Structure):

@@ -420,6 +420,8 @@ MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
 
 // MoE part of a graph: dims, events from ev0 (*ev_end = the next free
 // one), queue slots it may need (*qtasks), workspace; and its list slots.
+constexpr int kMoeXpMinT = 2048;  // default of et_graph_desc.moe_xp_min_T
+
 et_status setup_moe(et_graph* g, int ev0, int* ev_end, int* qtasks) {
     et_graph_desc& d = g->d;
     if (d.hidden <= 0) d.hidden = 2048;
@@ -483,6 +485,12 @@ et_status setup_moe(et_graph* g, int ev0, int* ev_end, int* qtasks) {
     ET_TRY(galloc(g, &p.Hm, pairs * p.inter));
     ET_TRY(galloc(g, &p.Yacc, (size_t)p.maxT * p.hidden));
     if (!make_map(&p.tm_hm, p.Hm, pairs, p.inter, 16)) return ET_ERR_CUDA;
+    if (d.moe_xp_min_T == 0) d.moe_xp_min_T = kMoeXpMinT;
+    p.Xp = nullptr;
+    if (d.moe_xp_min_T > 0 && p.maxT > p.tt && p.maxT >= d.moe_xp_min_T && p.hidden <= 2048) {  // row copy: <= 8 x 16 B per lane
+        ET_TRY(galloc(g, &p.Xp, pairs * p.hidden));
+        if (!make_map(&p.tm_xp, p.Xp, pairs, p.hidden, 16)) return ET_ERR_CUDA;
+    }
     return ET_OK;
 }
 void moe_slots(et_graph* g, const MoeParams& p, int Tb, std::vector<Slot>& s) {
@@ -874,6 +882,7 @@ et_status moe_run_params(et_graph* g, int T, const uint16_t* X, const uint16_t* 
     p.cb = mb.cb;      // (static lists and dynamic alike)
     p.n_cb = cdiv(T, p.cb);
     p.f_max = mb.f_max;
+    p.use_xp = p.Xp != nullptr && p.n_tt > 1 && T >= g->d.moe_xp_min_T;
     return ET_OK;
 }
 

@@ -52,13 +52,14 @@ struct MlpParams {
 // one token tile covers T, the whole grouping), SC scan, GR(g) grouping,
 // S1(f, n) stage-1 tile (token rows gathered from X), S2(f, n) stage-2
 // tile, CB(b) combine.
-enum { MOE_MAP_WR = 0, MOE_MAP_W1 = 1, MOE_MAP_W2 = 2, MOE_MAP_X = 3, MOE_MAP_HM = 4 };
+enum { MOE_MAP_WR = 0, MOE_MAP_W1 = 1, MOE_MAP_W2 = 2, MOE_MAP_X = 3, MOE_MAP_HM = 4, MOE_MAP_XP = 5 };
 struct MoeParams {
     CUtensorMap tm_wr;  // Wr [E, H], box 64 x 64
     CUtensorMap tm_w1;  // W1 [E*2I, H], box 64 x 64
     CUtensorMap tm_w2;  // W2 [E*H, I], box 64 x 64
     CUtensorMap tm_x;   // X  [T, H], box 64 x 16
     CUtensorMap tm_hm;  // Hm [maxT*k, I] (workspace), box 64 x 16
+    CUtensorMap tm_xp;  // Xp [maxT*k, H] (workspace), box 64 x 16
     const uint16_t* X;
     const float* bias;
     uint16_t* Y;
@@ -83,6 +84,8 @@ struct MoeParams {
     int32_t* pos;       // [maxT*k]
     int32_t* scal;      // [8]: 0 = total m-tiles, 1 = stage-2 tasks were pushed early
     uint16_t* Hm;       // [maxT*k, I] stage-1 output, grouped order
+    uint16_t* Xp;       // [maxT*k, H] X rows in grouped order (null when the graph never stages them)
+    int use_xp;         // this run: grouping tasks write Xp, stage 1 reads it by TMA
     float* Yacc;        // [maxT, H] fp32 combine accumulator (kept zero between runs)
     int T, hidden, inter, E, k, maxT;
     int tt, n_tt, n_kc, tkt, n_tk, bm, n1_tile, n_n1, n2_tile, n_n2, cb, n_cb;

@@ -99,7 +99,11 @@ struct Moe : WorkloadBase {
                 d.a_map = MOE_MAP_W1;
                 d.a_row0 = e * 2 * p.inter + b * p.n1_tile;
                 d.a_row1 = e * 2 * p.inter + p.inter + b * p.n1_tile;
-                d.gather = 1;  // token rows straight from X through perm
+                if (p.use_xp) {  // token rows staged in grouped order by the grouping tasks
+                    d.b_map = MOE_MAP_XP;
+                } else {
+                    d.gather = 1;  // token rows straight from X through perm
+                }
                 d.nk = p.hidden / kTileK;
             } else {
                 d.a_map = MOE_MAP_W2;
@@ -133,7 +137,7 @@ struct Moe : WorkloadBase {
         return id == MOE_MAP_WR ? &p.tm_wr : (id == MOE_MAP_W1 ? &p.tm_w1 : &p.tm_w2);
     }
     __device__ static const CUtensorMap* b_map(const Params& p, int id) {
-        return id == MOE_MAP_X ? &p.tm_x : &p.tm_hm;
+        return id == MOE_MAP_X ? &p.tm_x : (id == MOE_MAP_XP ? &p.tm_xp : &p.tm_hm);
     }
 
     // Push the stage-1 tasks of m-tiles [f0, f0 + nf) and, when stage 2 goes
@@ -578,7 +582,30 @@ struct Moe : WorkloadBase {
             p.perm[row] = pair;
             p.pos[pair] = row;
             if (p.out_perm) p.out_perm[row] = pair;
+            sm.tk[t * p.k + s] = row;  // the expert is no longer needed: keep the row for the X copy
         }
+    }
+
+    // Xp rows of a grouping tile's pairs: each token's X row (read once) to the
+    // grouped row of each of its k picks.  Warp w takes tokens w, w + 4, ...;
+    // lanes cover the row in 16-byte pieces.  Exec group, after place_pairs.
+    __device__ static void stage_rows(const Params& p, Ctx& x, const RouteSmem& sm, int t0, int ntok) {
+        exec_bar();  // the rows placed by every thread
+        const int w = x.tid >> 5, lane = x.tid & 31, nv = p.hidden / 8;
+        for (int t = w; t < ntok; t += kExecThreads / 32) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.X + (size_t)(t0 + t) * p.hidden);
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (lane + 32 * u < nv) v[u] = __ldg(src + lane + 32 * u);
+            for (int s = 0; s < p.k; ++s) {
+                uint4* dst = reinterpret_cast<uint4*>(p.Xp + (size_t)sm.tk[t * p.k + s] * p.hidden);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (lane + 32 * u < nv) dst[lane + 32 * u] = v[u];
+            }
+        }
+        fence_proxy_async_global();  // Xp is read by TMA in stage 1
     }
 
     // SC: expert counts from the per-tile pair counts, the CSRs and each
@@ -656,6 +683,7 @@ struct Moe : WorkloadBase {
         if (e < p.E) sm.base[e] = __ldcg(p.goff + (size_t)g * p.E + e);
         load_tile_picks(p, x, sm, t0, ntok);
         place_pairs(p, x, sm, t0, ntok);
+        if (p.use_xp) stage_rows(p, x, sm, t0, ntok);
         const int cnt = e < p.E ? tile_count(sm, e) : 0;
         if (!x.dynamic) {
             group_finish_notify(x, d, x.ctr + p.ev_grp, 1, p.n_tt);

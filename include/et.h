@@ -119,6 +119,11 @@ typedef struct {
     float rope_base;     /* rotary embedding base [500000] */
     /* MoE -> dense MLP (ET_GRAPH_MOE_MLP); the MoE dims above, the MLP's width = hidden */
     int mlp_inter;       /* dense MLP intermediate width [6144] */
+    /* MoE: from this T on (when several 128-token grouping tiles exist) each grouping task
+       also copies its tokens' rows of X into a permuted copy in grouped order, and stage 1
+       loads its token rows from there by TMA instead of gathering them from X for every
+       column tile [2048; -1 = never] */
+    int moe_xp_min_T;
 } et_graph_desc;
 
 typedef struct et_graph et_graph; /* opaque, library-owned */

@@ -395,6 +395,8 @@ def moe_dataflow(topk, n_kc, tkt, tt, bm, n_n1, n_n2, cb, E):
     # stable grouping by brute force: expert-major, ascending token
     order = [(t, s) for e in range(E) for t in range(T) for s in range(k) if int(topk[t, s]) == e]
     row_of = {pair: r for r, pair in enumerate(order)}
+    # ("row", r): grouped row r placed (its pair index, and, where the device
+    # stages stage-1 rows in grouped order, its copy of the token's X row)
     all_route = {("route", t) for t in range(T)}
     for j in range(_cdiv(T, tkt)):
         toks = range(j * tkt, min(T, (j + 1) * tkt))

@@ -159,6 +159,42 @@ def test_moe_dependency_order(small_inputs, sched, T):
         et.et_destroy_graph(g)
 
 
+@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid"])
+@pytest.mark.parametrize("T", [150, 300])
+def test_moe_staged_rows(small_inputs, sched, T):
+    """Stage-1 token rows staged once in grouped order by the grouping tasks
+    (moe_xp_min_T lowered so that small dims take that path): Y against the
+    grouped oracle, and dependency order and event counts as above."""
+    d = small_inputs
+    g = et.et_build_graph(et.ET_GRAPH_MOE, sched, 512, debug_flags=et.ET_DEBUG_TRACE | et.ET_DEBUG_DELAY,
+                          moe_xp_min_T=129, **SMALL)
+    try:
+        st, out = run_moe(g, d, T, 4, 16)
+        assert st == 0
+        w_o, grp = check_routing(d, out, 4, 16, T)
+        y_ref = oracle.moe_grouped(d["X"][:T], d["W1"], d["W2"], out["topk"], w_o, grp["indptr"], grp["perm"])
+        assert maxnorm_err(out["y"], y_ref) <= TOL_Y
+        info = et.et_get_info(g)
+        trace = et.et_get_trace(g)
+        n_kc = max(r[2] for r in trace if r[0] == dag.OP_MOE_ROUTER) + 1
+        n_n1, n_n2 = 128 // info["moe_n1_tile"], 256 // info["moe_n2_tile"]
+        counts = et.et_get_event_counts(g)
+        n_cb = sum(1 for kind, _, _ in counts if kind == 26)  # the run's combine blocks (size bucket)
+        cb = 1 if n_cb == T else -(-T // n_cb)
+        graph, _ = dag.moe_graph(out["topk"], 16, info["moe_tt"], n_kc, info["moe_tkt"], info["moe_gt"], info["moe_bm"],
+                                 n_n1, n_n2, cb, sched)
+        errs = dag.check_trace(graph, trace)
+        assert errs == [], errs[:5]
+        rw = dag.moe_dataflow(out["topk"], n_kc, info["moe_tkt"], info["moe_tt"], info["moe_bm"], n_n1, n_n2,
+                              cb, 16)
+        errs = dag.check_dataflow(rw, trace)
+        assert errs == [], errs[:5]
+        errs = dag.check_event_counts(graph, counts)
+        assert errs == [], errs[:5]
+    finally:
+        et.et_destroy_graph(g)
+
+
 @pytest.mark.parametrize("sched", ["static", "dynamic"])
 def test_moe_timeout_reports(small_inputs, sched):
     d = small_inputs
