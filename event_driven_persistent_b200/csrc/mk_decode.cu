@@ -353,13 +353,26 @@ struct Decode : WorkloadBase {
             inv[tid] = 1.0f / ls;
         }
         exec_bar();
-        // thread t = dim t: the splits' partial outputs, loads independent of each other
-        for (int h = 0; h < p.grp; ++h) {
-            float os = 0.f;
-#pragma unroll 4
-            for (int s = 0; s < ns; ++s) os = fmaf(wgt[s * p.grp + h], __ldcg(base + ((size_t)s * p.grp + h) * stride + tid), os);
-            p.attn[(size_t)bb * p.nq * p.hd + (size_t)(g * p.grp + h) * p.hd + tid] = bf16_bits(os * inv[h]);
+        // thread t = dim t: the splits' partial outputs of every head, eight
+        // splits' loads issued together before their sums
+        float os[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int s0 = 0; s0 < ns; s0 += 8) {
+            float v[8][4];
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    v[s][h] = (s0 + s < ns && h < p.grp) ? __ldcg(base + ((size_t)(s0 + s) * p.grp + h) * stride + tid)
+                                                         : 0.f;
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    if (s0 + s < ns && h < p.grp) os[h] = fmaf(wgt[(s0 + s) * p.grp + h], v[s][h], os[h]);
         }
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            if (h < p.grp) p.attn[(size_t)bb * p.nq * p.hd + (size_t)(g * p.grp + h) * p.hd + tid] = bf16_bits(os[h] * inv[h]);
         fence_proxy_async_global();  // attn is read by TMA in the o-proj tasks
         int* ev = x.ctr + (unfused(p) ? p.ev_merge_all : p.ev_ag + g);
         const int tgt = unfused(p) ? p.B * p.nkv : p.B;
