@@ -297,7 +297,7 @@ et_status build_splitk(et_graph* g) {
     if (d.splitk_cols <= 0) d.splitk_cols = 128;
     if (d.splitk_chunk <= 0) d.splitk_chunk = 32;
     if (d.splitk_tile_rows <= 0) d.splitk_tile_rows = 32;
-    if (d.fetch_batch <= 0) d.fetch_batch = 4;
+    if (d.fetch_batch <= 0) d.fetch_batch = 1;
     const int nt_max = cdiv(d.max_T, d.splitk_tile_rows);
     const int nch = cdiv(d.splitk_cols, d.splitk_chunk);
     if (nt_max > 0xFFFF || nch > 0x3FF) return ET_ERR_UNSUPPORTED;

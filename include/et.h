@@ -105,7 +105,7 @@ typedef struct {
     int splitk_chunk;    /* split-K K-chunk [32] */
     int splitk_tile_rows;/* split-K rows per task [32] */
     float rms_eps;       /* MLP RMSNorm epsilon [1e-5] */
-    int fetch_batch;     /* dynamic: tasks claimed per atomic pop [workload default] */
+    int fetch_batch;     /* dynamic: tasks claimed per atomic pop [1] */
     int debug_flags;     /* ET_DEBUG_* */
     int device;          /* CUDA device ordinal */
     int n_ctas;          /* persistent CTAs [0 = one per SM] */

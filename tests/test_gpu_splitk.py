@@ -52,6 +52,26 @@ def test_splitk_config_parity(sched):
         et.et_destroy_graph(g)
 
 
+@pytest.mark.parametrize("fetch_batch", [1, 2, 4])
+def test_splitk_batched_pops(fetch_batch):
+    """The dynamic schedule with F queue slots reserved per atomic pop
+    (several tasks per CTA in flight from one reservation): results, and
+    dependency order with random delays."""
+    g = et.et_build_graph(et.ET_GRAPH_SPLITK, "dynamic", 512, fetch_batch=fetch_batch,
+                          debug_flags=et.ET_DEBUG_TRACE | et.ET_DEBUG_DELAY)
+    try:
+        A = W.splitk_inputs(512)
+        for _ in range(2):
+            st, B, C = run(g, A)
+            assert st == 0
+            check(A, B, C)
+        graph = dag.splitk_graph(512, 128, 32, 32, "dynamic")
+        errs = dag.check_trace(graph, et.et_get_trace(g))
+        assert errs == [], errs[:5]
+    finally:
+        et.et_destroy_graph(g)
+
+
 @pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid"])
 @pytest.mark.parametrize("rows", [1, 31, 33, 1000, 4096])
 def test_splitk_ragged_and_symbolic_rows(sched, rows):
