@@ -42,13 +42,28 @@ struct SplitK : WorkloadBase {
             if (!group_wait(x, d, nullptr, 0, 0)) return false;  // no input event
             const int c0 = j * p.chunk;
             const int nc = min(p.chunk, p.cols - c0);
-            for (int r = warp; r < nr; r += kExecThreads / 32) {
-                const float* row = p.A + (size_t)(r0 + r) * p.cols + c0;
+            // four threads per row, each summing columns q*8 .. q*8+7 of every
+            // 32-column block of the chunk (independent loads), then two shuffles
+            const int q = lane & 3;
+            for (int rb = 0; rb < nr; rb += kExecThreads / 4) {
+                const int r = rb + (x.tid >> 2);
                 float s = 0.f;
-                for (int c = lane; c < nc; c += 32) s += row[c];
+                if (r < nr) {
+                    const float* row = p.A + (size_t)(r0 + r) * p.cols + c0;
+                    for (int cb = 0; cb < nc; cb += 32) {
+                        float v[8];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                if (lane == 0) p.Bp[(size_t)(r0 + r) * p.n_chunks + j] = s;
+                        for (int e = 0; e < 8; ++e) {
+                            const int c = cb + q * 8 + e;
+                            v[e] = c < nc ? row[c] : 0.f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s += v[e];
+                    }
+                }
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                if (r < nr && q == 0) p.Bp[(size_t)(r0 + r) * p.n_chunks + j] = s;
             }
             int* ev = x.ctr + (p.unfused ? p.ev_all : p.ev_base + i);
             const int tgt = p.unfused ? p.n_tiles * p.n_chunks : target(p, i);
