@@ -130,6 +130,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t tx) 
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(tx)
                  : "memory");
 }
+// raise the phase's expected transaction bytes without arriving
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t tx) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(tx) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
     uint32_t ok;
     asm volatile(

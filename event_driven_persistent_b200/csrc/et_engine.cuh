@@ -244,6 +244,35 @@ __device__ __forceinline__ StageAlloc stream_alloc(const TaskDesc& d) {
     return a;
 }
 
+// B rows of one stage for tiles of more than 32 rows (all 32 lanes of the
+// producer warp call): eight lanes per row, so one copy instruction covers
+// the 128-byte K atom of four rows (four whole lines); lane l holds the
+// addresses of rows l, l + 32, l + 64 and l + 96 (null past the task's
+// rows) and hands them to the lanes that copy them.  The 32-row blocks are
+// a rolled loop: the code stays small.
+__device__ __forceinline__ void gather_rows_wide(uint8_t* bdst, uint32_t atom, int n, int kx, int lane,
+                                                 const uint16_t* const (&rows)[4]) {
+    const int sub = lane >> 3, cc = lane & 7;
+#pragma unroll 1
+    for (int i = 0; 32 * i < n; ++i) {
+        const uint16_t* r = i == 0 ? rows[0] : i == 1 ? rows[1] : i == 2 ? rows[2] : rows[3];
+        const unsigned long long mine = reinterpret_cast<unsigned long long>(r);
+        const uint16_t* src[8];  // all eight hand-offs first: independent
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+            src[g] = reinterpret_cast<const uint16_t*>(__shfl_sync(0xffffffffu, mine, 4 * g + sub));
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const int rr = 32 * i + 4 * g + sub;
+            if (src[g] && rr < n) {
+                uint8_t* dr = bdst + rr * 128 + ((cc ^ (rr & 7)) << 4);
+                cp_async16(dr, src[g] + kx + cc * 8);
+                cp_async16(dr + atom, src[g] + kx + kAtomK + cc * 8);
+            }
+        }
+    }
+}
+
 // Megakernel body.  W supplies the task semantics:
 //   W::fetch_init(p, idx)              initial dynamic task word for slot idx
 //   W::derive(p, x, word, d)           fill a TaskDesc (warp 0; may wait in
@@ -389,8 +418,11 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     tma_load_2d(bdst + at * atom + rb * 128, bm2, &sc->full[slot2], kx + at * kAtomK, dd.b_row0 + rb, pol);
         };
         auto issue_a = [&](uint32_t slot2, uint32_t off, const CUtensorMap* am2, const TaskDesc& dd, int stage,
-                           uint32_t tx, uint64_t pol) {
-            mbar_arrive_expect_tx(&sc->full[slot2], tx);
+                           uint32_t tx, uint64_t pol, bool arrive = true) {
+            if (arrive)
+                mbar_arrive_expect_tx(&sc->full[slot2], tx);
+            else
+                mbar_expect_tx(&sc->full[slot2], tx);
             ++armed[slot2];
             uint8_t* dst = arena + off;
             const int kx = dd.k0 + stage * kTileK;
@@ -548,9 +580,10 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     ok = sc->pok;
                     __syncwarp();
                 } else {
-                    // B rows gathered through an index list: every lane copies
-                    // up to 4 rows per stage with cp.async into the 128-byte
-                    // swizzled layout; lane 0 adds the weight tile by TMA.
+                    // B rows gathered through an index list, copied with
+                    // cp.async into the 128-byte swizzled layout (a lane per
+                    // row for tiles of up to 32 rows, else eight lanes per
+                    // row); lane 0 adds the weight tile by TMA first.
                     // The rows' index list is read first: its L2 round trip
                     // overlaps the hand-off.  (A gathered task's inputs are
                     // complete when it is derived: derive waits for them, or
@@ -584,22 +617,28 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                         const uint32_t sl = sc->pslot, of = sc->poff;
                         __syncwarp();
                         if (!ok) break;
+                        // the weight tile first (its bytes expected, no arrival
+                        // yet), then the rows; the phase completes only after
+                        // lane 0's arrival, which follows every lane's copies
+                        if (lane == 0) issue_a(sl, of, am, d, s, kAStageBytes, pol_w, false);
                         const int kx = d.k0 + s * kTileK;
                         uint8_t* bdst = arena + of + kAStageBytes;
                         const uint32_t atom = (uint32_t)d.n * 128u;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int rr = lane + 32 * i;
-                            if (rows[i]) {
-                                const uint16_t* src = rows[i] + kx;
+                        if (d.n <= 32) {
+                            // up to 32 rows: a lane copies its own row
+                            if (rows[0]) {
+                                const uint16_t* src = rows[0] + kx;
 #pragma unroll
                                 for (int c = 0; c < 16; ++c)
-                                    cp_async16(bdst + (c >> 3) * atom + rr * 128 + (((c & 7) ^ (rr & 7)) << 4), src + c * 8);
+                                    cp_async16(bdst + (c >> 3) * atom + lane * 128 + (((c & 7) ^ (lane & 7)) << 4),
+                                               src + c * 8);
                             }
+                        } else {
+                            gather_rows_wide(bdst, atom, d.n, kx, lane, rows);
                         }
                         cp_async_mbar_arrive(&sc->full[sl]);
                         __syncwarp();
-                        if (lane == 0) issue_a(sl, of, am, d, s, kAStageBytes, pol_w);
+                        if (lane == 0) mbar_arrive(&sc->full[sl]);
                     }
                 }
                 if (!ok) break;
