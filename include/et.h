@@ -144,7 +144,9 @@ typedef struct {
     int moe_n2_tile;     /* output columns per stage-2 task */
     int moe_cb;          /* tokens per combine task at this graph's max_T; a run whose size
                             bucket (the power of two >= T, capped at max_T) is <= 256 uses 1 */
-    int dec_split;       /* decode: keys per attention split task */
+    int dec_split;       /* decode: keys per attention split task of the last run (before any run:
+                            the graph's, 512); the dynamic and hybrid schedules double it from
+                            B = 8 and quadruple it from B = 32, static lists keep the graph's */
     int dec_qkv_kc;      /* decode: K chunks of a QKV head tile */
     int dec_o_kc;        /* decode: K columns per o-proj task (the heads of one KV group) */
 } et_graph_info;

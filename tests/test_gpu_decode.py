@@ -110,16 +110,19 @@ def test_decode_symbolic_B_repeated_runs(small_inputs, sched):
         et.et_destroy_graph(g)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic", "hybrid", "unfused"])
-def test_decode_dependency_order(small_inputs, sched):
+@pytest.mark.parametrize("sched,B", [("static", 5), ("dynamic", 5), ("hybrid", 5), ("unfused", 5),
+                                     ("dynamic", 12), ("hybrid", 40), ("static", 40)])
+def test_decode_dependency_order(small_inputs, sched, B):
+    """Trace order, data flow and event counts against the oracle's task
+    graph; B = 12 and 40 run the longer queued splits (1024 and 2048 keys)."""
     d = small_inputs
-    B = 5
-    g = et.et_build_graph(et.ET_GRAPH_DECODE, sched, 8, max_ctx=600,
+    g = et.et_build_graph(et.ET_GRAPH_DECODE, sched, max(B, 8), max_ctx=600,
                           debug_flags=et.ET_DEBUG_TRACE | et.ET_DEBUG_DELAY, **SMALL)
     try:
         st, out = run_decode(g, d, B)
         assert st == 0
         info = et.et_get_info(g)
+        assert info["dec_split"] == (512 if sched in ("static", "unfused") or B < 8 else (1024 if B < 32 else 2048))
         kw = dict(nq=4, nkv=2, n_kc=info["dec_qkv_kc"], split=info["dec_split"], n_m=1024 // 128,
                   n_gu=512 // info["mlp_gu_tile"], gu_tile=info["mlp_gu_tile"], kchunk=info["mlp_kchunk"],
                   n_c=512 // info["mlp_kchunk"])
