@@ -605,7 +605,10 @@ et_status build_decode(et_graph* g) {
     p.rope_base = (double)d.rope_base;
     p.n_heads = p.nq + 2 * p.nkv;
     const int kt = p.hidden / kTileK;
-    p.n_kc = kt % 4 == 0 ? 4 : (kt % 2 == 0 ? 2 : 1);
+    // QKV K chunks: as many as keep every (head tile, chunk) task in one wave
+    // over the CTAs (chunks of kt / n_kc stages, rounded: 10 or 11 of the 32
+    // stages for 48 head tiles on 148 SMs), so no CTA streams two tasks
+    p.n_kc = std::max(1, std::min(kt, g->n_ctas / p.n_heads));
     p.o_kc = p.grp * p.hd;
     p.gu_tile = 64;
     p.kchunk = d.inter % 1024 == 0 ? 1024 : (d.inter % 256 == 0 ? 256 : 128);

@@ -67,8 +67,10 @@ struct Decode : WorkloadBase {
             d.b_map = DEC_MAP_XN;
             d.b_row0 = 0;
             d.n = tok_n(p);
-            d.k0 = b * (p.hidden / p.n_kc);
-            d.nk = p.hidden / p.n_kc / kTileK;
+            // K chunk b: stages [b kt / n_kc, (b + 1) kt / n_kc) of the kt
+            const int kt = p.hidden / kTileK, s0 = b * kt / p.n_kc;
+            d.k0 = s0 * kTileK;
+            d.nk = (b + 1) * kt / p.n_kc - s0;
         } else if (op == ET_OP_DEC_ATTN) {
             const int bb = a / p.nkv, g = a % p.nkv, s = b;
             d.valid = 0;

@@ -147,7 +147,8 @@ typedef struct {
     int dec_split;       /* decode: keys per attention split task of the last run (before any run:
                             the graph's, 512); the dynamic and hybrid schedules double it from
                             B = 8 and quadruple it from B = 32, static lists keep the graph's */
-    int dec_qkv_kc;      /* decode: K chunks of a QKV head tile */
+    int dec_qkv_kc;      /* decode: K chunks of a QKV head tile (as many as keep every QKV task in
+                            one wave over the CTAs; chunk c = stages [c kt / n, (c + 1) kt / n)) */
     int dec_o_kc;        /* decode: K columns per o-proj task (the heads of one KV group) */
 } et_graph_info;
 
