@@ -58,6 +58,7 @@ struct SmemCtl {
     uint64_t ring_empty[kRing];
     uint64_t drain;
     uint64_t s_full[2], p_full[2], o_full[2];  // attention stages k: buffers k & 1 of S, P and O
+    uint64_t gready[kSlots];  // gathered stage reserved and its weight tile issued (warp 0 -> gather warp)
     uint32_t tmem_base;
     int start_status;
     int bcast[8];
@@ -321,9 +322,10 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
         }
         for (int r = 0; r < kRing; ++r) {
             mbar_init(&sc->ring_full[r], 1);
-            mbar_init(&sc->ring_empty[r], 2);  // MMA warp + exec group
+            mbar_init(&sc->ring_empty[r], W::kGather ? 3 : 2);  // MMA warp + exec group (+ gather warp)
         }
         mbar_init(&sc->drain, 1);
+        for (int s = 0; s < kSlots; ++s) mbar_init(&sc->gready[s], 1);
         mbar_init(&sc->s_full[0], 1);
         mbar_init(&sc->s_full[1], 1);
         for (int b = 0; b < 2; ++b) {
@@ -383,7 +385,6 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             lend = ra.lists.off[blockIdx.x + 1];
         }
         int qn = 0, qe = 0;
-        bool any_gather = false;
         // lane 0: stage bookkeeping (global stage count, arena ranges of the
         // last kSlots stages, arms per slot for the exit drain)
         uint32_t nst = 0, tail = 0;  // stages reserved so far; oldest stage not yet seen consumed
@@ -580,66 +581,36 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
                     ok = sc->pok;
                     __syncwarp();
                 } else {
-                    // B rows gathered through an index list, copied with
-                    // cp.async into the 128-byte swizzled layout (a lane per
-                    // row for tiles of up to 32 rows, else eight lanes per
-                    // row); lane 0 adds the weight tile by TMA first.
-                    // The rows' index list is read first: its L2 round trip
-                    // overlaps the hand-off.  (A gathered task's inputs are
-                    // complete when it is derived: derive waits for them, or
-                    // the queue holds the task only once they are.)
-                    any_gather = true;
-                    const uint16_t* rows[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) rows[i] = W::gather_row(p, d, lane + 32 * i);
+                    // B rows gathered through an index list: the gather warp
+                    // copies them.  Per stage this warp reserves the stage,
+                    // raises its expected bytes by the weight tile's without
+                    // arriving, issues the weight tile and signals gready; the
+                    // gather warp's arrival (after its row copies) completes
+                    // the phase.  The weight stream never waits on the rows.
+                    // (A gathered task's inputs are complete when it is
+                    // derived: derive waits for them, or the queue holds the
+                    // task only once they are.)
                     if (lane == 0) {
                         ok = W::gemm_wait(p, x, d);
                         if (ok && (x.debug & ET_DEBUG_TRACE)) {
                             d.start = take_ticket(ctl);
                             d.t_ready = globaltimer();
                         }
+                        d.st0 = nst;  // the task's first stage: the gather warp follows from it
                         sc->ring[slot] = d;
                         mbar_arrive(&sc->ring_full[slot]);
+                        for (int s = 0; ok && s < d.nk; ++s) {
+                            uint32_t sl = 0, of = 0;
+                            ok = reserve(stage_bytes(d.n), &sl, &of);
+                            if (!ok) break;
+                            issue_a(sl, of, am, d, s, kAStageBytes, pol_w, false);
+                            mbar_arrive(&sc->gready[sl]);
+                        }
                         sc->pok = ok;
                     }
                     __syncwarp();
                     ok = sc->pok;
                     __syncwarp();
-                    for (int s = 0; s < d.nk && ok; ++s) {
-                        if (lane == 0) {
-                            uint32_t sl = 0, of = 0;
-                            sc->pok = reserve(stage_bytes(d.n), &sl, &of);
-                            sc->pslot = sl;
-                            sc->poff = of;
-                        }
-                        __syncwarp();
-                        ok = sc->pok;
-                        const uint32_t sl = sc->pslot, of = sc->poff;
-                        __syncwarp();
-                        if (!ok) break;
-                        // the weight tile first (its bytes expected, no arrival
-                        // yet), then the rows; the phase completes only after
-                        // lane 0's arrival, which follows every lane's copies
-                        if (lane == 0) issue_a(sl, of, am, d, s, kAStageBytes, pol_w, false);
-                        const int kx = d.k0 + s * kTileK;
-                        uint8_t* bdst = arena + of + kAStageBytes;
-                        const uint32_t atom = (uint32_t)d.n * 128u;
-                        if (d.n <= 32) {
-                            // up to 32 rows: a lane copies its own row
-                            if (rows[0]) {
-                                const uint16_t* src = rows[0] + kx;
-#pragma unroll
-                                for (int c = 0; c < 16; ++c)
-                                    cp_async16(bdst + (c >> 3) * atom + lane * 128 + (((c & 7) ^ (lane & 7)) << 4),
-                                               src + c * 8);
-                            }
-                        } else {
-                            gather_rows_wide(bdst, atom, d.n, kx, lane, rows);
-                        }
-                        cp_async_mbar_arrive(&sc->full[sl]);
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sc->full[sl]);
-                    }
                 }
                 if (!ok) break;
             } else {
@@ -651,7 +622,6 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             if (r == 0) break;
         }
         // drain: every armed stage's copies must land before the CTA exits
-        if (any_gather) cp_async_wait_all();
         if (lane == 0)
             for (int s = 0; s < kSlots; ++s)
                 if (armed[s]) {
@@ -788,7 +758,68 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             }
         }
         __syncwarp();
-    } else if (!skip && warp >= kExecWarp0) {
+    } else if (!skip && W::kGather && warp == kGatherWarp) {
+        // ------------------------------------------------------ row gather
+        // Follows the task ring.  For each gathered task, the B rows of every
+        // stage once warp 0 has reserved it and issued its weight tile
+        // (gready; warp 0 cannot reuse a slot before this warp's arrival on
+        // it, so one parity bit per slot tracks the phases): cp.async into
+        // the 128-byte swizzled layout, a lane per row for tiles of up to 32
+        // rows, else eight lanes per row; the last arrival completes the
+        // stage's full phase.
+        uint32_t gpar = 0;
+        for (uint32_t it = 0;; ++it) {
+            const uint32_t slot = it % kRing;
+            int okw = 1;
+            if (lane == 0) okw = mbar_wait(&sc->ring_full[slot], (it / kRing) & 1, ctl, x.timeout_ns, 930);
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            __syncwarp();  // lane 0's acquire orders the other lanes' reads of the entry
+            if (!okw) break;
+            const TaskDesc d = sc->ring[slot];
+            __syncwarp();  // every lane has the entry before lane 0 frees it
+            if (lane == 0) mbar_arrive(&sc->ring_empty[slot]);
+            if (d.word == kExitWord) break;
+            if (!(d.valid && d.gemm && d.gather)) continue;
+            const uint16_t* rows[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rows[i] = W::gather_row(p, d, lane + 32 * i);
+            const uint32_t atom = (uint32_t)d.n * 128u;
+            bool ok = true;
+            for (int s = 0; s < d.nk; ++s) {
+                const uint32_t sl = (d.st0 + (uint32_t)s) % kSlots;
+                uint32_t of = 0;
+                int okg = 1;
+                if (lane == 0) {
+                    okg = mbar_wait(&sc->gready[sl], (gpar >> sl) & 1u, ctl, x.timeout_ns, 931);
+                    of = sc->r_off[sl];
+                }
+                if (!__shfl_sync(0xffffffffu, okg, 0)) {
+                    ok = false;
+                    break;
+                }
+                of = __shfl_sync(0xffffffffu, of, 0);
+                gpar ^= 1u << sl;
+                const int kx = d.k0 + s * kTileK;
+                uint8_t* bdst = arena + of + kAStageBytes;
+                if (d.n <= 32) {
+                    if (rows[0]) {
+                        const uint16_t* src = rows[0] + kx;
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            cp_async16(bdst + (c >> 3) * atom + lane * 128 + (((c & 7) ^ (lane & 7)) << 4), src + c * 8);
+                    }
+                } else {
+                    gather_rows_wide(bdst, atom, d.n, kx, lane, rows);
+                }
+                cp_async_mbar_arrive(&sc->full[sl]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sc->full[sl]);
+            }
+            if (!ok) break;
+        }
+        cp_async_wait_all();  // every copy landed before the CTA exits
+        __syncwarp();
+    } else if (!skip && warp >= kExecWarp0 && warp < kExecWarp0 + kExecThreads / 32) {
         // ------------------------------------------------- epilogue / CUDA-core
         // Every decision that can end the loop is taken by exec thread 0 and
         // broadcast, so the four warps never split around a named barrier.

@@ -760,7 +760,7 @@ et_status et_build_graph(const et_graph_desc* desc, et_graph** out) {
     in.sched = g->d.sched;
     in.max_T = g->d.max_T;
     in.n_ctas = g->n_ctas;
-    in.threads = kThreads;
+    in.threads = (desc->kind == ET_GRAPH_MOE || desc->kind == ET_GRAPH_MOE_MLP) ? kThreadsGather : kThreads;
     in.smem_bytes = g->d.kind == ET_GRAPH_SPLITK ? kSmemNoArenaBytes : kSmemBytes;
     in.fetch_batch = g->d.fetch_batch;
     in.hidden = g->d.hidden;

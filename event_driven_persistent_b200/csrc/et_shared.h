@@ -9,8 +9,11 @@ namespace et {
 typedef et_trace_record TraceRec;
 
 // Launch shape of every megakernel: warp 0 fetches tasks and drives TMA,
-// warp 1 issues tcgen05 MMAs, warps 2..5 run epilogues and CUDA-core tasks.
+// warp 1 issues tcgen05 MMAs, warps 2..5 run epilogues and CUDA-core tasks;
+// workloads with gathered B rows add warp 6, which copies those rows.
 constexpr int kThreads = 192;
+constexpr int kGatherWarp = 6;
+constexpr int kThreadsGather = kThreads + 32;
 constexpr int kExecThreads = 128;
 constexpr int kExecWarp0 = 2;
 constexpr int kRing = 2;           // task ring depth (warp 0 runs one task ahead)

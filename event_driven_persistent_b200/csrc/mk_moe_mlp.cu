@@ -56,20 +56,20 @@ struct MoeMlp : WorkloadBase {
     }
 };
 
-__global__ void __launch_bounds__(kThreads, 1) moe_mlp_kernel(const __grid_constant__ MoeMlpParams p, const RunArgs ra) {
+__global__ void __launch_bounds__(kThreadsGather, 1) moe_mlp_kernel(const __grid_constant__ MoeMlpParams p, const RunArgs ra) {
     megakernel_body<MoeMlp>(p, ra);
 }
 
 cudaError_t moe_mlp_setup(int* max_blocks_per_sm) {
     cudaError_t e = cudaFuncSetAttribute(moe_mlp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(max_blocks_per_sm, moe_mlp_kernel, kThreads, kSmemBytes);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(max_blocks_per_sm, moe_mlp_kernel, kThreadsGather, kSmemBytes);
 }
 
 cudaError_t launch_moe_mlp(const MoeMlpParams& p, const RunArgs& ra, int n_ctas, cudaStream_t s) {
     // the launch's own status (not an unrelated error left pending earlier)
     void* args[] = {const_cast<MoeMlpParams*>(&p), const_cast<RunArgs*>(&ra)};
-    return cudaLaunchKernel(reinterpret_cast<const void*>(moe_mlp_kernel), dim3(n_ctas), dim3(kThreads), args,
+    return cudaLaunchKernel(reinterpret_cast<const void*>(moe_mlp_kernel), dim3(n_ctas), dim3(kThreadsGather), args,
                             kSmemBytes, s);
 }
 
