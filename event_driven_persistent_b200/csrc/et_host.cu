@@ -420,7 +420,11 @@ MoeShape moe_shape(const et_graph* g, const MoeParams& p, int T) {
 
 // MoE part of a graph: dims, events from ev0 (*ev_end = the next free
 // one), queue slots it may need (*qtasks), workspace; and its list slots.
-constexpr int kMoeXpMinT = 2048;  // default of et_graph_desc.moe_xp_min_T
+// Default of et_graph_desc.moe_xp_min_T: never.  Staged rows paid off while
+// the producer warp gathered stage-1 rows itself (T = 4096: 1294 -> 1198 us);
+// with the gather warp, gathering is faster at every T (T = 2048: 728 -> 592
+// us, T = 4096: 1190 -> 987 us without them).
+constexpr int kMoeXpMinT = -1;
 
 et_status setup_moe(et_graph* g, int ev0, int* ev_end, int* qtasks) {
     et_graph_desc& d = g->d;

@@ -122,7 +122,7 @@ typedef struct {
     /* MoE: from this T on (when several 128-token grouping tiles exist) each grouping task
        also copies its tokens' rows of X into a permuted copy in grouped order, and stage 1
        loads its token rows from there by TMA instead of gathering them from X for every
-       column tile [2048; -1 = never] */
+       column tile [0 = the default: never; -1 = never] */
     int moe_xp_min_T;
 } et_graph_desc;
 
