@@ -115,6 +115,10 @@ struct WorkloadBase {
     __device__ static void stream_late(const P&, const TaskDesc&, int, uint8_t*, uint64_t*, uint64_t) {}
     template <class P>
     __device__ static bool stream_exec(const P&, Ctx&, TaskDesc&) { return false; }
+    // B operand map with a 64-row box (the same tensor as b_map), for the
+    // 64-row chunks of wide token tiles: one copy instead of four; null = none
+    template <class P>
+    __device__ static const CUtensorMap* b_map_wide(const P&, int) { return nullptr; }
 };
 
 __device__ __forceinline__ void exec_bar() { named_bar_sync(1, kExecThreads); }
@@ -413,10 +417,15 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
             uint8_t* bdst = arena + off + kAStageBytes;
             const uint32_t atom = (uint32_t)dd.n * 128u;
             const int kx = dd.k0 + stage * kTileK;
-            for (int rb = 0; rb < dd.n; rb += 16)
+            const CUtensorMap* bw = W::b_map_wide(p, dd.b_map);
+            for (int rb = 0; rb < dd.n;) {
+                const bool wide = bw != nullptr && rb + 64 <= dd.n;  // a 64-row box where one fits
 #pragma unroll
                 for (int at = 0; at < 2; ++at)
-                    tma_load_2d(bdst + at * atom + rb * 128, bm2, &sc->full[slot2], kx + at * kAtomK, dd.b_row0 + rb, pol);
+                    tma_load_2d(bdst + at * atom + rb * 128, wide ? bw : bm2, &sc->full[slot2], kx + at * kAtomK,
+                                dd.b_row0 + rb, pol);
+                rb += wide ? 64 : 16;
+            }
         };
         auto issue_a = [&](uint32_t slot2, uint32_t off, const CUtensorMap* am2, const TaskDesc& dd, int stage,
                            uint32_t tx, uint64_t pol, bool arrive = true) {

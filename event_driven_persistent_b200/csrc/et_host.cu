@@ -489,6 +489,7 @@ et_status setup_moe(et_graph* g, int ev0, int* ev_end, int* qtasks) {
     ET_TRY(galloc(g, &p.Hm, pairs * p.inter));
     ET_TRY(galloc(g, &p.Yacc, (size_t)p.maxT * p.hidden));
     if (!make_map(&p.tm_hm, p.Hm, pairs, p.inter, 16)) return ET_ERR_CUDA;
+    if (!make_map(&p.tm_hm64, p.Hm, pairs, p.inter, 64)) return ET_ERR_CUDA;
     if (d.moe_xp_min_T == 0) d.moe_xp_min_T = kMoeXpMinT;
     p.Xp = nullptr;
     if (d.moe_xp_min_T > 0 && p.maxT > p.tt && p.maxT >= d.moe_xp_min_T && p.hidden <= 2048) {  // row copy: <= 8 x 16 B per lane

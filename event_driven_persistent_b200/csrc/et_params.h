@@ -59,6 +59,7 @@ struct MoeParams {
     CUtensorMap tm_w2;  // W2 [E*H, I], box 64 x 64
     CUtensorMap tm_x;   // X  [T, H], box 64 x 16
     CUtensorMap tm_hm;  // Hm [maxT*k, I] (workspace), box 64 x 16
+    CUtensorMap tm_hm64;  // Hm, box 64 x 64 (stage-2 token tiles of 64 rows and more)
     CUtensorMap tm_xp;  // Xp [maxT*k, H] (workspace), box 64 x 16
     const uint16_t* X;
     const float* bias;

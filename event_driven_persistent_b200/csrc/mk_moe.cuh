@@ -139,6 +139,9 @@ struct Moe : WorkloadBase {
     __device__ static const CUtensorMap* b_map(const Params& p, int id) {
         return id == MOE_MAP_X ? &p.tm_x : (id == MOE_MAP_XP ? &p.tm_xp : &p.tm_hm);
     }
+    __device__ static const CUtensorMap* b_map_wide(const Params& p, int id) {
+        return id == MOE_MAP_HM ? &p.tm_hm64 : nullptr;
+    }
 
     // Push the stage-1 tasks of m-tiles [f0, f0 + nf) and, when stage 2 goes
     // early, their stage-2 tasks right after (exec group or single thread).
