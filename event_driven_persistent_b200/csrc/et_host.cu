@@ -360,6 +360,9 @@ et_status setup_mlp(et_graph* g, MlpParams& p, int hidden, int inter, int maxB, 
     ET_TRY(galloc(g, &p.yacc, (size_t)p.maxB * p.hidden));
     if (!make_map(&p.tm_xn, p.xn, rows, p.hidden, 16)) return ET_ERR_CUDA;
     if (!make_map(&p.tm_h, p.h, rows, p.inter, 16)) return ET_ERR_CUDA;
+    p.wide_b = rows >= 64;
+    if (p.wide_b && (!make_map(&p.tm_xn64, p.xn, rows, p.hidden, 64) || !make_map(&p.tm_h64, p.h, rows, p.inter, 64)))
+        return ET_ERR_CUDA;
     return ET_OK;
 }
 int mlp_queue_tasks(const MlpParams& p) { return p.maxB + p.n_gu + p.n_m * p.n_c + p.n_m; }
@@ -667,6 +670,11 @@ et_status build_decode(et_graph* g) {
     if (!make_map(&p.tm_xn2, p.xn2, rows, p.hidden, 16)) return ET_ERR_CUDA;
     if (!make_map(&p.tm_hm, p.hm, rows, p.inter, 16)) return ET_ERR_CUDA;
     if (!make_map(&p.tm_q, p.q, (uint64_t)p.maxB * p.nq, p.hd, 16)) return ET_ERR_CUDA;
+    p.wide_b = rows >= 64;
+    if (p.wide_b && (!make_map(&p.tm_xn64, p.xn, rows, p.hidden, 64) ||
+                     !make_map(&p.tm_attn64, p.attn, rows, (uint64_t)p.nq * p.hd, 64) ||
+                     !make_map(&p.tm_xn2_64, p.xn2, rows, p.hidden, 64) || !make_map(&p.tm_hm64, p.hm, rows, p.inter, 64)))
+        return ET_ERR_CUDA;
     int mb = 0;
     ET_CU(decode_setup(&mb));
     if (mb < 1) return ET_ERR_UNSUPPORTED;

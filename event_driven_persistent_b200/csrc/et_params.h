@@ -31,6 +31,8 @@ struct MlpParams {
     CUtensorMap tm_wd;   // Wd  [H, I], box 64 x 64
     CUtensorMap tm_xn;   // xn  [maxB, H] (workspace), box 64 x 16
     CUtensorMap tm_h;    // h   [maxB, I] (workspace), box 64 x 16
+    CUtensorMap tm_xn64, tm_h64;  // the same, box 64 x 64 (wide_b)
+    int wide_b;          // 1 = the workspaces hold 64 rows or more: 64-row boxes for wide token tiles
     const uint16_t* X;
     const uint16_t* gamma;
     uint16_t* xn;
@@ -123,6 +125,8 @@ struct DecodeParams {
     CUtensorMap tm_kc;   // K cache as [B nkv max_ctx, hd], box 64 x 128 (this run's Kc)
     CUtensorMap tm_vt;   // V^T cache as [B nkv hd, max_ctx], box 64 x 128 (this run's Vc)
     CUtensorMap tm_q;    // q as [maxB nq, hd], box 64 x 16
+    CUtensorMap tm_xn64, tm_attn64, tm_xn2_64, tm_hm64;  // workspace activations, box 64 x 64 (wide_b)
+    int wide_b;          // 1 = the workspaces hold 64 rows or more: 64-row boxes for wide token tiles
     // inputs / outputs
     const uint16_t* X;
     const int32_t* pos;        // [B] tokens already cached per request (= the new token's position)

@@ -152,6 +152,11 @@ struct Decode : WorkloadBase {
     __device__ static const CUtensorMap* b_map(const Params& p, int id) {
         return id == DEC_MAP_XN ? &p.tm_xn : (id == DEC_MAP_ATTN ? &p.tm_attn : (id == DEC_MAP_XN2 ? &p.tm_xn2 : &p.tm_hm));
     }
+    __device__ static const CUtensorMap* b_map_wide(const Params& p, int id) {
+        if (!p.wide_b) return nullptr;
+        return id == DEC_MAP_XN ? &p.tm_xn64
+                                : (id == DEC_MAP_ATTN ? &p.tm_attn64 : (id == DEC_MAP_XN2 ? &p.tm_xn2_64 : &p.tm_hm64));
+    }
 
     // ------------------------------------------------------------ stream
     // Stages of an attention split whose keys were cached before this step

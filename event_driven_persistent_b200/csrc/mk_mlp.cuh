@@ -74,6 +74,9 @@ struct Mlp : WorkloadBase {
     __device__ static const CUtensorMap* b_map(const Params& p, int id) {
         return id == MLP_MAP_XN ? &p.tm_xn : &p.tm_h;
     }
+    __device__ static const CUtensorMap* b_map_wide(const Params& p, int id) {
+        return !p.wide_b ? nullptr : (id == MLP_MAP_XN ? &p.tm_xn64 : &p.tm_h64);
+    }
 
     __device__ static bool epilogue(const Params& p, Ctx& x, TaskDesc& d, uint32_t taddr, uint64_t* acc_empty) {
         const int op = task_op(d.word), a = task_a(d.word), c = task_b(d.word);

@@ -44,6 +44,9 @@ struct MoeMlp : WorkloadBase {
     __device__ static const CUtensorMap* a_map(const Params& p, int id) {
         return id >= kMlpMaps ? Mlp::a_map(p.mlp, id - kMlpMaps) : Moe::a_map(p.moe, id);
     }
+    __device__ static const CUtensorMap* b_map_wide(const Params& p, int id) {
+        return id >= kMlpMaps ? Mlp::b_map_wide(p.mlp, id - kMlpMaps) : Moe::b_map_wide(p.moe, id);
+    }
     __device__ static const CUtensorMap* b_map(const Params& p, int id) {
         return id >= kMlpMaps ? Mlp::b_map(p.mlp, id - kMlpMaps) : Moe::b_map(p.moe, id);
     }
