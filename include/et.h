@@ -130,7 +130,10 @@ typedef struct et_graph et_graph; /* opaque, library-owned */
 
 /* Tile parameters of a built graph (what the task coordinates mean). */
 typedef struct {
-    int kind, sched, max_T, n_ctas, threads, smem_bytes, fetch_batch;
+    int kind, sched, max_T, n_ctas;
+    int threads;         /* per CTA: 192 (224 in the MoE graphs, which add a warp that copies
+                            gathered token rows) */
+    int smem_bytes, fetch_batch;
     int hidden, inter, n_experts, top_k;
     int splitk_cols, splitk_chunk, splitk_tile_rows;
     int mlp_gu_tile;     /* intermediate columns per gate/up task */
