@@ -18,6 +18,9 @@
 //   warps 2..5      epilogues (tcgen05.ld of the accumulator, fused
 //                   element-wise math, stores, notify/push) and all CUDA-core
 //                   tasks (norm, reductions, top-k, grouping, combine).
+//   warp 6          (workloads with gathered B rows only) the cp.async row
+//                   copies of gathered stages, so that warp 0's weight
+//                   stream never waits on them.
 //
 // Tasks flow from warp 0 to the others through a 2-deep ring in shared
 // memory guarded by mbarriers.
@@ -33,7 +36,7 @@ struct TaskDesc {
     int valid;       // 0 = a static slot with nothing to do at this size
     uint32_t start;  // trace ticket taken after the task's wait
     int gemm;        // 1 = tensor-core task
-    int gather;      // 1 = B rows gathered through W::gather_row (cp.async), else B by TMA
+    int gather;      // 1 = B rows gathered through W::gather_row (cp.async, gather warp), else B by TMA
     uint64_t t_fetch, t_ready, t_acc;  // trace timestamps (ns)
     int a_map, a_row0, a_row1;  // A: tensor map id, rows of the two 64-row boxes
     int b_map, b_row0;          // B: tensor map id, first row
@@ -250,7 +253,7 @@ __device__ __forceinline__ StageAlloc stream_alloc(const TaskDesc& d) {
 }
 
 // B rows of one stage for tiles of more than 32 rows (all 32 lanes of the
-// producer warp call): eight lanes per row, so one copy instruction covers
+// gather warp call): eight lanes per row, so one copy instruction covers
 // the 128-byte K atom of four rows (four whole lines); lane l holds the
 // addresses of rows l, l + 32, l + 64 and l + 96 (null past the task's
 // rows) and hands them to the lanes that copy them.  The 32-row blocks are
@@ -378,8 +381,8 @@ __device__ __forceinline__ void megakernel_body(const typename W::Params& p, con
 
     if (!skip && warp == 0) {
         // ---------------------------------------------------- task source + loads
-        // Lane 0 leads (task fetch, waits, TMA, ring); for tasks whose B rows
-        // are gathered through an index list, all 32 lanes issue the row copies.
+        // Lane 0 leads (task fetch, waits, TMA, ring); the other lanes follow
+        // (the B rows of gathered tasks are copied by the gather warp).
         const uint64_t pol_w = policy_evict_first();
         const uint64_t pol_a = policy_evict_last();
         // phase 0: list part A; 1: ready queue; 2: list part B
